@@ -1,0 +1,479 @@
+#!/usr/bin/env python3
+"""Benchmark of the KDA forward pass on B200: chunked-prefill tokens/s with its HBM roofline fraction,
+plus the fused decode step's state GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {1,2,3,4,5}] [--impl {ours,reference}]
+
+One step = one pass of the forward pass over one batch of the workload with inputs resident in
+HBM: one ``kda_chunk_fwd`` call for the prefill workloads (1-4), one ``kda_recurrent_step`` call for
+the decode workload (5).  Rank 0 prints ONE JSON line.  With N > 1 (launched by torch.distributed.run)
+every rank runs the same workload on its own GPU over its own independent (b, hv) shard -- the
+forward pass has no exchange step, so there is no collective on the data path (weak scaling);
+a barrier and a MAX all-reduce of the device times are the only communication.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from kimi_delta_attention_33_b200.inputs import GATE_STANDARD, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "KDA fwd tokens/s (chunked prefill) & decode-step state GB/s, % of roofline, 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+PREFILL_KERNEL_FILES = {"simt": "kimi_delta_attention_33_b200/csrc/kda_chunk_simt.cu",
+                        "tc": "kimi_delta_attention_33_b200/csrc/kda_chunk_tc.cu"}
+DECODE_KERNEL_FILE = "kimi_delta_attention_33_b200/csrc/kda_decode.cu"
+
+
+# ------------------------------------------------------------------------ algorithmic counts ---
+
+def elt_bytes(w):
+    return 2 if w.dtype == torch.bfloat16 else 4
+
+
+def prefill_bytes(w) -> int:
+    """Bytes the forward pass must move: q, k once per H head, v, g_raw, beta, A_log, dt_bias and S0
+    (when given) read; o and S_T written.  Per-chunk states and intermediates are not counted."""
+    e = elt_bytes(w)
+    B, T, H, HV, K, V = w.B, w.T, w.H, w.HV, w.K, w.V
+    rd = 2 * B * T * H * K * e + B * T * HV * V * e + B * T * HV * K * e + B * T * HV * e + HV * 4 + HV * K * 4
+    if w.S0_std is not None:
+        rd += B * HV * K * V * 4
+    wr = B * T * HV * V * e + B * HV * K * V * 4
+    return rd + wr
+
+
+def prefill_flops(w) -> float:
+    """2 flops per multiply-add, triangles counted half: A, R, W, U (C*K/2 or C*V/2 each), the solve
+    (C^2/6), the three K x V state products and A.E (C*V/2), per token and value head."""
+    C, K, V = w.chunk, w.K, w.V
+    per = 2 * (4 * (C * K / 2) + C * C / 6 + 3 * K * V + C * V / 2)
+    return per * w.B * w.T * w.HV
+
+
+def decode_bytes(w) -> int:
+    """Per decode step: S read and written (fp32), q, k per H head, v, g_raw, beta, A_log, dt_bias, o."""
+    e = elt_bytes(w)
+    B, H, HV, K, V = w.B, w.H, w.HV, w.K, w.V
+    return (2 * B * HV * K * V * 4 + 2 * B * H * K * e + B * HV * V * e + B * HV * K * e + B * HV * e + HV * 4
+            + HV * K * 4 + B * HV * V * e)
+
+
+# -------------------------------------------------------------------------------- peaks etc ----
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1632.8)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, 1590.0, "fallback"
+
+
+def _sha(path):
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def ncu_traffic(kernel_file: str, wid: int):
+    """DRAM bytes per launch from the committed ncu summary, or None when absent or stale."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    ent = table.get(f"{kernel_file}#{wid}")
+    if not ent or ent.get("source_sha256") != _sha(kernel_file):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------------- clocks -----
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.period, self.stop_evt, self.thread, self.max_mhz = period_s, threading.Event(), None, None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.get_reasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return None
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ distributed ---
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- our arm -------
+
+def _step_inputs_decode(x, w, dev):
+    """Per-step contiguous slices [steps, B, ...] of the decode token stream."""
+    return {n: x[n].to(dev).transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
+
+
+def run_ours(args, ws, rank, local):
+    from kimi_delta_attention_33_b200 import kda
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    torch.manual_seed(0)
+    x = make_inputs(w, seed=1000 + w.wid + 7919 * rank, device=str(dev))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    hbm_peak, _, peak_kind = measured_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    if w.is_decode:
+        steps_in = _step_inputs_decode(x, w, dev)
+        S = x["S0"].clone()
+        o = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
+        nsteps = steps_in["q"].shape[0]
+
+        def step(i):
+            t = i % nsteps
+            kda.recurrent_step(steps_in["q"][t], steps_in["k"][t], steps_in["v"][t], steps_in["g"][t],
+                               steps_in["beta"][t], S, x["A_log"], x["dt_bias"], gate_mode=w.gate_mode,
+                               lower_bound=w.lower_bound, o=o)
+        units_per_step = w.B                    # one token per sequence per step
+        bytes_per_launch = decode_bytes(w)
+        kernel_file, flush_needed = DECODE_KERNEL_FILE, False   # 512 MiB of state >> L2
+    else:
+        ws_bytes = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+        o = torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev)
+        S_T = torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev)
+
+        def step(i):
+            kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["S0"],
+                          chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o, S_T=S_T,
+                          workspace=workspace)
+        units_per_step = w.B * w.T
+        bytes_per_launch = prefill_bytes(w)
+        kernel_file = PREFILL_KERNEL_FILES["tc" if kda.uses_tensor_cores(w.K, w.V, w.chunk) else "simt"]
+        flush_needed = prefill_bytes(w) < 2 * (126 << 20)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if not w.is_decode:
+        kda.read_status(workspace)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            if flush_needed:
+                flush.zero_()
+            evs[i][0].record(stream)
+            step(args.warmup + i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(step_ms), ws)
+    ms_per_step = total_ms / args.steps
+    value = ws * units_per_step * args.steps / (total_ms / 1e3)
+    kern_s = (sum(step_ms) / args.steps) / 1e3     # one launch of our kernel per step
+    achieved = bytes_per_launch / kern_s / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": ncu_traffic(kernel_file, w.wid),
+            "kernel_file": kernel_file, "algorithmic_bytes_per_launch": bytes_per_launch}
+    if not w.is_decode:
+        roof["algorithmic_flops_per_launch"] = prefill_flops(w)
+        roof["achieved_tflops"] = round(prefill_flops(w) / kern_s / 1e12, 2)
+
+    e2e = run_e2e(args, w, x, dev, kda) if rank == 0 else None
+    decode_extra = None
+    if not w.is_decode and not args.no_decode_extra and rank == 0:
+        decode_extra = run_decode_extra(args, dev, kda, hbm_peak)
+    cpu = cpu_baseline(w) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": workload_config(w, ws, flush_needed), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clk.summary()}
+        if decode_extra is not None:
+            line["decode"] = decode_extra
+        print(json.dumps(line), flush=True)
+
+
+def workload_config(w, ws, flushed):
+    return {"workload": f"workload {w.wid}: {w.name}", "B": w.B, "T": w.T, "H": w.H, "HV": w.HV, "K": w.K,
+            "V": w.V, "chunk": w.chunk, "gate": "standard" if w.gate_mode == GATE_STANDARD else "safe",
+            "inputs": "bf16" if w.dtype == torch.bfloat16 else "fp32", "state": "fp32",
+            "S0": w.S0_std is not None, "l2": ("flushed between timed steps (256 MiB write)" if flushed
+                                               else "inputs larger than L2"),
+            "parallelism": f"dp{ws} (independent (b, hv) shards per GPU, no collective)"}
+
+
+def run_e2e(args, w, x, dev, kda):
+    """Same metric through the public API with host buffers: pinned H2D of the step's inputs, the call,
+    D2H of the step's result, all inside the timed region."""
+    stream = torch.cuda.current_stream(dev)
+    names = ("q", "k", "v", "g", "beta")
+    if w.is_decode:
+        host = {n: x[n][:, 0].contiguous().cpu().pin_memory() for n in names}
+        devb = {n: torch.empty_like(host[n], device=dev) for n in names}
+        S = x["S0"].clone()
+        o_dev = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
+        o_host = torch.empty(o_dev.shape, dtype=w.dtype).pin_memory()
+        units = w.B
+
+        def call():
+            for n in names:
+                devb[n].copy_(host[n], non_blocking=True)
+            kda.recurrent_step(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"], S, x["A_log"], x["dt_bias"],
+                               gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o_dev)
+            o_host.copy_(o_dev, non_blocking=True)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = o_host.numel() * o_host.element_size()
+    else:
+        inputs = names + (("S0",) if x["S0"] is not None else ())
+        host = {n: x[n].cpu().pin_memory() for n in inputs}
+        devb = {n: torch.empty_like(host[n], device=dev) for n in inputs}
+        ws_bytes = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+        o_dev = torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev)
+        S_dev = torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev)
+        o_host = torch.empty(o_dev.shape, dtype=w.dtype).pin_memory()
+        S_host = torch.empty(S_dev.shape, dtype=torch.float32).pin_memory()
+        units = w.B * w.T
+
+        def call():
+            for n in inputs:
+                devb[n].copy_(host[n], non_blocking=True)
+            kda.chunk_fwd(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"], x["A_log"], x["dt_bias"],
+                          devb.get("S0"), chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o_dev,
+                          S_T=S_dev, workspace=workspace)
+            o_host.copy_(o_dev, non_blocking=True)
+            S_host.copy_(S_dev, non_blocking=True)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in inputs)
+        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+    for _ in range(max(args.warmup, 1)):
+        call()
+    torch.cuda.synchronize(dev)
+    n = max(3, min(args.steps, 50))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    sec = a.elapsed_time(b) / 1e3 / n
+    return {"value": round(units / sec, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+def run_decode_extra(args, dev, kda, hbm_peak):
+    """The decode workload's step, measured in the same run: state GB/s against the HBM roofline."""
+    w = WORKLOADS[5]
+    x = make_inputs(w, device=str(dev))
+    steps_in = _step_inputs_decode(x, w, dev)
+    S = x["S0"].clone()
+    o = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t):
+        kda.recurrent_step(steps_in["q"][t], steps_in["k"][t], steps_in["v"][t], steps_in["g"][t],
+                           steps_in["beta"][t], S, x["A_log"], x["dt_bias"], gate_mode=w.gate_mode,
+                           lower_bound=w.lower_bound, o=o)
+    for t in range(3):
+        step(t)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for t in range(w.decode_steps):
+        step(t)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    sec = a.elapsed_time(b) / 1e3 / w.decode_steps
+    gbs = decode_bytes(w) / sec / 1e9
+    return {"workload": f"workload 5: {w.name}", "steps": w.decode_steps, "us_per_step": round(sec * 1e6, 2),
+            "tokens_per_s": round(w.B / sec, 1), "state_GBps": round(gbs, 1), "peak": hbm_peak,
+            "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_step": decode_bytes(w),
+            "traffic": ncu_traffic(DECODE_KERNEL_FILE, 5)}
+
+
+# ------------------------------------------------------------------------ CPU oracle legs -----
+
+def _oracle_sample(w, budget_s: float):
+    """A bounded sample of the workload for the float64 oracle: a subset of (b, hv) pairs over a prefix
+    of the tokens, sized to roughly `budget_s` seconds on this host.  Returns the callable and a
+    description; the callable returns the number of workload tokens it stands for (token-heads / HV)."""
+    import oracle
+    threads = max(1, oracle.num_threads())
+    per_token_head = 7.0 * w.K * w.V          # double flops of one recurrence step
+    rate = 0.8e9 * threads                    # rough oracle speed, only used to size the sample
+    T = w.T
+    max_th = budget_s * rate / per_token_head
+    pairs = max(1, min(w.pairs, int(max_th // T)))
+    if pairs == 1 and T > max_th:
+        T = max(16, int(max_th))
+    pairs = min(pairs, w.pairs)
+    sub = w.scaled(T=T)
+    x = make_inputs(sub)
+    G = w.HV // w.H
+    sel = [(b, hv) for b in range(w.B) for hv in range(w.HV)][:pairs]
+
+    def run():
+        for b, hv in sel:
+            h = hv // G
+            s0 = None if x["S0"] is None else x["S0"][b:b + 1, hv:hv + 1]
+            oracle.forward(x["q"][b:b + 1, :, h:h + 1], x["k"][b:b + 1, :, h:h + 1], x["v"][b:b + 1, :, hv:hv + 1],
+                           x["g"][b:b + 1, :, hv:hv + 1], x["beta"][b:b + 1, :, hv:hv + 1], x["A_log"][hv:hv + 1],
+                           x["dt_bias"][hv:hv + 1], s0, gate_mode=w.gate_mode, lower_bound=w.lower_bound)
+        return pairs * T / w.HV
+
+    desc = (f"{pairs} of {w.pairs} (b, hv) pairs x {T} of {w.T} tokens"
+            f" ({pairs * T} token-heads = {pairs * T / w.HV:.1f} workload tokens), one pair per oracle call")
+    return run, desc, threads
+
+
+def cpu_baseline(w):
+    run, desc, threads = _oracle_sample(w, budget_s=4.0)
+    t0 = time.perf_counter()
+    tokens, reps = 0.0, 0
+    while True:
+        tokens += run()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= 10.0 or reps >= 50:
+            break
+    return {"value": round(tokens / el, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{desc}; repeated {reps}x in {el:.1f} s on {os.cpu_count()} host cores",
+            "host_cpu_count": os.cpu_count()}
+
+
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores, on this arm's workload, metric and unit."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    run, desc, threads = _oracle_sample(w, budget_s=2.0)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    tokens = sum(run() for _ in range(args.steps))
+    el = time.perf_counter() - t0
+    v = round(tokens / el, 2)
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                      "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                      "config": workload_config(w, 1, False),
+                      "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                       "sample": desc + " per step"},
+                      "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-extra", action="store_true")
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = {1: 200, 2: 200, 3: 20, 4: 10, 5: 128}[args.workload] if args.impl == "ours" else 10
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    ws, rank, local = dist_setup()
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention forward library.
+ *
+ * The operation (KDA notes, "KDA 递归核心", §逐步公式 steps 1-4; KDA ledger DER1):
+ * every (sequence b, value head hv) keeps a key-major state S in R^{K x V};
+ * for each token t
+ *     S_dec = exp(g_t) (.) S_{t-1}          decay, one factor per KEY channel (row of S)
+ *     r_t   = v_t - k_t . S_dec             delta-rule residual
+ *     S_t   = S_dec + (beta_t k_t) (x) r_t  rank-1 write
+ *     o_t   = scale * q_t . S_t             read-out, scale = 1/sqrt(K) by default
+ * Grouped value attention (KDA notes, "KDA 递归核心", input-tensor table:
+ * q, k are repeat_interleave'd to HV heads): value head hv reads q/k head
+ * hv / (HV/H).  The gate (KDA notes, "Gate 激活", table "两种 Gate"):
+ *     input = g_raw + dt_bias[hv, :],  rate = exp(A_log[hv])
+ *     SAFE      g = lower_bound * sigmoid(rate * input)     in [lower_bound, 0]
+ *     STANDARD  g = -rate * softplus(input)                 in (-inf, 0]
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense, contiguous, row-major DEVICE buffers with the
+ *     shapes given per argument; the caller owns and allocates all of them.
+ *     The library never allocates, never frees and keeps no pointer after
+ *     the call returns.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
+ *     the legacy default stream).  No entry point synchronises the device,
+ *     except kda_read_status, which exists to do so.
+ *   - Arguments are validated on the host before anything is launched.  On an
+ *     invalid argument nothing is launched and KDA_ERR_INVALID_ARG or
+ *     KDA_ERR_UNSUPPORTED is returned; a launch failure returns KDA_ERR_CUDA.
+ *     kda_last_error() then describes the failure (thread-local string).
+ *   - No C++ exception crosses this interface.
+ *   - Per-token tensors (q, k, v, g, beta, o) share one dtype (`dtype`);
+ *     A_log, dt_bias and the state are always float32.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary-compatible with cudaStream_t. */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null pointer, bad shape or bad value; nothing launched     */
+    KDA_ERR_UNSUPPORTED = 2, /* valid but outside the built kernels (K, V, chunk, dtype)  */
+    KDA_ERR_CUDA = 3,        /* a CUDA call failed; kda_last_error() names it             */
+    KDA_ERR_TIMEOUT = 4      /* a bounded on-device wait gave up (see kda_read_status)   */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Mirrors the op's `use_gate_in_kernel` / `safe_gate` switches (KDA notes, "Gate 激活",
+ * §Gate 在 API 中的位置): NONE means `g` already holds the log-space decay. */
+typedef enum { KDA_GATE_NONE = 0, KDA_GATE_SAFE = 1, KDA_GATE_STANDARD = 2 } kda_gate_mode;
+
+/* Thread-local description of the last failure on the calling thread ("" if none). */
+const char* kda_last_error(void);
+
+/* Library version string. */
+const char* kda_version(void);
+
+/*
+ * kda_gate -- the gate activation alone (KDA notes, "Gate 激活", code box
+ * kda_gate_reference and table "两种 Gate").
+ *   g_raw    [B, T, HV, K]  dtype           raw gate projection
+ *   A_log    [HV]           float32         head-wise log rate
+ *   dt_bias  [HV, K]        float32 or NULL (NULL: no bias)
+ *   mode     KDA_GATE_SAFE or KDA_GATE_STANDARD (NONE is INVALID_ARG)
+ *   lower_bound  SAFE only: finite and < 0, else INVALID_ARG
+ *   g_out    [B, T, HV, K]  float32         log-space decay, written
+ * B, T, HV, K >= 1 (B*T*HV*K < 2^31).
+ */
+kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, const float* dt_bias,
+                    int B, int T, int HV, int K, kda_gate_mode mode, float lower_bound,
+                    float* g_out, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
+ * for these sizes (always >= 256: the first 256 bytes hold the on-device status
+ * word read by kda_read_status).  Returns 0 for sizes kda_chunk_fwd rejects.
+ */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk);
+
+/*
+ * kda_chunk_fwd -- chunked prefill (DeltaNet-family digest, sections "Chunkwise
+ * KDA" and "Chunkwise Triton pipeline"): the same result as running the
+ * recurrence above token by token, computed C tokens at a time with the
+ * in-chunk cumulative log-decay, the triangular solve for the in-chunk delta
+ * errors and one state update per chunk.
+ *   q, k     [B, T, H, K]   dtype
+ *   v        [B, T, HV, V]  dtype
+ *   g        [B, T, HV, K]  dtype   g_raw when gate_mode != NONE, else the log decay (<= 0)
+ *   beta     [B, T, HV]     dtype   write strength (the op applies no sigmoid)
+ *   A_log    [HV] float32, dt_bias [HV, K] float32 or NULL -- used when gate_mode != NONE
+ *            (A_log may be NULL only when gate_mode == NONE)
+ *   S0       [B, HV, K, V]  float32 initial state, or NULL for zeros
+ *   chunk    16 or 64 (the pages' default is 64)
+ *   scale    read-out scale; <= 0 selects 1/sqrt(K)
+ *   o        [B, T, HV, V]  dtype, written; must not alias any input
+ *   S_T      [B, HV, K, V]  float32 final state, written; or NULL.  May alias S0
+ *            (in-place state update).
+ *   workspace, workspace_bytes  >= kda_chunk_fwd_workspace_size(...) bytes of
+ *            caller-owned device memory, 256-byte aligned; contents need no
+ *            initialisation and are scratch after the call.
+ * Constraints: HV % H == 0; K, V in {16, 32, 64, 128}; T >= 1 (a last partial
+ * chunk is handled); every pointer 16-byte aligned.
+ * Calls that share one workspace must be ordered on one stream.
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* A_log, const float* dt_bias,
+                         const float* S0, int B, int T, int H, int HV, int K, int V, int chunk,
+                         kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
+                         void* o, float* S_T, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream);
+
+/*
+ * kda_read_status -- synchronises `stream`, then reads the status word a
+ * kda_chunk_fwd call left in `workspace` and clears it.  Returns KDA_OK, or
+ * KDA_ERR_TIMEOUT if a bounded on-device wait of that call gave up (its
+ * outputs are then undefined), or KDA_ERR_CUDA.
+ */
+kda_status kda_read_status(const void* workspace, kda_stream_t stream);
+
+/*
+ * kda_recurrent_step -- one decode step for a batch of sequences, fused
+ * (DeltaNet-family digest, "decode के लिए fused recurrent Triton kernel": the
+ * recurrent schedule for decode and stateful serving).  S is read once and
+ * written once, in place.
+ *   q, k     [B, H, K]      dtype   (one token per sequence, i.e. [B, 1, H, K])
+ *   v        [B, HV, V]     dtype
+ *   g        [B, HV, K]     dtype   g_raw when gate_mode != NONE, else the log decay
+ *   beta     [B, HV]        dtype
+ *   A_log, dt_bias          as for kda_chunk_fwd
+ *   S        [B, HV, K, V]  float32, read and overwritten with S_t
+ *   o        [B, HV, V]     dtype, written; must not alias any input
+ * Constraints: HV % H == 0; K, V in {16, 32, 64, 128}; every pointer 16-byte aligned.
+ */
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, const float* A_log, const float* dt_bias,
+                              int B, int H, int HV, int K, int V, kda_gate_mode gate_mode,
+                              float lower_bound, float scale, kda_dtype dtype, float* S, void* o,
+                              kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,156 @@
+// kda_api.cu -- the C ABI declared in include/kda.h: host-side validation, kernel choice,
+// status codes and the thread-local error string.  No exception crosses this file's
+// extern "C" functions and nothing here allocates device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "kda_internal.h"
+
+#define KDA_VERSION_STRING "kda-b200 0.1.0 (sm_100a)"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+kda_status fail(kda_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+kda_status ok() {
+    g_err[0] = '\0';
+    return KDA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool kv_dim_ok(int x) { return x == 16 || x == 32 || x == 64 || x == 128; }
+
+kda_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Validation shared by the prefill and decode entry points.
+kda_status check_common(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        const float* A_log, int B, int H, int HV, int K, int V, int gate_mode, float lower_bound,
+                        int dtype, const void* o) {
+    if (!q || !k || !v || !g || !beta || !o) return fail(KDA_ERR_INVALID_ARG, "null tensor pointer (q, k, v, g, beta and o are required)");
+    if (B < 1 || H < 1 || HV < 1 || K < 1 || V < 1) return fail(KDA_ERR_INVALID_ARG, "sizes must be >= 1 (B=%d H=%d HV=%d K=%d V=%d)", B, H, HV, K, V);
+    if (HV % H != 0) return fail(KDA_ERR_INVALID_ARG, "HV (%d) must be a multiple of H (%d)", HV, H);
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (gate_mode != KDA_GATE_NONE && gate_mode != KDA_GATE_SAFE && gate_mode != KDA_GATE_STANDARD)
+        return fail(KDA_ERR_INVALID_ARG, "unknown gate mode %d", gate_mode);
+    if (gate_mode != KDA_GATE_NONE && !A_log) return fail(KDA_ERR_INVALID_ARG, "A_log is required when the gate is applied in the op");
+    if (gate_mode == KDA_GATE_SAFE && !(std::isfinite(lower_bound) && lower_bound < 0.0f))
+        return fail(KDA_ERR_INVALID_ARG, "safe gate needs a finite lower_bound < 0 (got %g)", (double)lower_bound);
+    if (!kv_dim_ok(K) || !kv_dim_ok(V)) return fail(KDA_ERR_UNSUPPORTED, "K and V must each be 16, 32, 64 or 128 (K=%d V=%d)", K, V);
+    return KDA_OK;
+}
+
+constexpr size_t kStatusBytes = 256;
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_last_error(void) { return g_err; }
+
+const char* kda_version(void) { return KDA_VERSION_STRING; }
+
+kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, const float* dt_bias, int B, int T,
+                    int HV, int K, kda_gate_mode mode, float lower_bound, float* g_out, kda_stream_t stream) {
+    if (!g_raw || !A_log || !g_out) return fail(KDA_ERR_INVALID_ARG, "null pointer (g_raw, A_log and g_out are required)");
+    if (B < 1 || T < 1 || HV < 1 || K < 1) return fail(KDA_ERR_INVALID_ARG, "sizes must be >= 1");
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (mode != KDA_GATE_SAFE && mode != KDA_GATE_STANDARD) return fail(KDA_ERR_INVALID_ARG, "kda_gate needs SAFE or STANDARD mode");
+    if (mode == KDA_GATE_SAFE && !(std::isfinite(lower_bound) && lower_bound < 0.0f))
+        return fail(KDA_ERR_INVALID_ARG, "safe gate needs a finite lower_bound < 0 (got %g)", (double)lower_bound);
+    const long long n = (long long)B * T * HV * K;
+    if (n >= (1ll << 31)) return fail(KDA_ERR_UNSUPPORTED, "B*T*HV*K must be < 2^31");
+    kda::GateArgs a{g_raw, (int)dtype, A_log, dt_bias, n, HV, K, (int)mode, lower_bound, g_out, (cudaStream_t)stream};
+    cudaError_t e = kda::launch_gate(a);
+    if (e != cudaSuccess) return cuda_fail(e, "gate kernel launch");
+    return ok();
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk) {
+    if (B < 1 || T < 1 || H < 1 || HV < 1 || HV % H != 0 || !kv_dim_ok(K) || !kv_dim_ok(V)) return 0;
+    if (chunk != 16 && chunk != 64) return 0;
+    return kStatusBytes;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         const float* A_log, const float* dt_bias, const float* S0, int B, int T, int H, int HV,
+                         int K, int V, int chunk, kda_gate_mode gate_mode, float lower_bound, float scale,
+                         kda_dtype dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream) {
+    kda_status s = check_common(q, k, v, g, beta, A_log, B, H, HV, K, V, (int)gate_mode, lower_bound, (int)dtype, o);
+    if (s != KDA_OK) return s;
+    if (T < 1) return fail(KDA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    if (chunk != 16 && chunk != 64) return fail(KDA_ERR_UNSUPPORTED, "chunk must be 16 or 64 (got %d)", chunk);
+    if ((long long)B * T * HV * (K > V ? K : V) >= (1ll << 40)) return fail(KDA_ERR_UNSUPPORTED, "tensor too large");
+    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, S0, o, S_T, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace of at least %zu bytes is required (got %zu)", need, workspace_bytes);
+    if (o == q || o == k || o == v || o == g || o == beta) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
+    if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
+    kda::ChunkArgs a{q, k, v, g, beta, A_log, dt_bias, S0, B, T, H, HV, K, V, chunk, (int)gate_mode, lower_bound,
+                     scale, (int)dtype, o, S_T, static_cast<unsigned int*>(workspace),
+                     static_cast<char*>(workspace) + kStatusBytes, workspace_bytes - kStatusBytes,
+                     (cudaStream_t)stream};
+    cudaError_t e;
+    if (kda::chunk_tc_supported(a)) {
+        e = kda::launch_chunk_tc(a);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel launch");
+    } else {
+        e = kda::launch_chunk_simt(a);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk kernel launch");
+    }
+    return ok();
+}
+
+kda_status kda_read_status(const void* workspace, kda_stream_t stream) {
+    if (!workspace) return fail(KDA_ERR_INVALID_ARG, "null workspace");
+    unsigned int word = 0;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read-back");
+    if (word != kda::STATUS_OK) {
+        const unsigned int zero = 0;
+        cudaMemcpy(const_cast<void*>(workspace), &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        return fail(KDA_ERR_TIMEOUT, "an on-device wait gave up (status word 0x%x); outputs are undefined", word);
+    }
+    return ok();
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                              const float* A_log, const float* dt_bias, int B, int H, int HV, int K, int V,
+                              kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype, float* S,
+                              void* o, kda_stream_t stream) {
+    kda_status s = check_common(q, k, v, g, beta, A_log, B, H, HV, K, V, (int)gate_mode, lower_bound, (int)dtype, o);
+    if (s != KDA_OK) return s;
+    if (!S) return fail(KDA_ERR_INVALID_ARG, "null state pointer S");
+    if ((long long)B * HV >= (1ll << 31)) return fail(KDA_ERR_UNSUPPORTED, "B*HV must be < 2^31");
+    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, S, o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    if (o == q || o == k || o == v || o == g || o == beta || o == S) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
+    if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
+    kda::DecodeArgs a{q, k, v, g, beta, A_log, dt_bias, B, H, HV, K, V, (int)gate_mode, lower_bound, scale,
+                      (int)dtype, S, o, (cudaStream_t)stream};
+    cudaError_t e = kda::launch_decode_step(a);
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// kda_common.cuh -- small device helpers shared by the KDA kernels (not by the oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// ---- element load / store for the two per-token dtypes -------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Loads 4 consecutive elements (16-byte aligned for float, 8-byte aligned for bf16) as float4.
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+// ---- gate activation (KDA notes, "Gate 激活", table "两种 Gate") ------------------------------
+// input = g_raw + dt_bias, rate = exp(A_log):
+//   SAFE      g = L * sigmoid(rate * input)
+//   STANDARD  g = -rate * softplus(input), softplus(x) = max(x,0) + log1p(exp(-|x|))
+// NONE returns the input unchanged (it is already the log-space decay).
+__device__ __forceinline__ float gate_value(float graw, float bias, float rate, int mode, float lower_bound) {
+    const float x = graw + bias;
+    if (mode == KDA_GATE_SAFE) {
+        return lower_bound / (1.0f + expf(-rate * x));
+    } else if (mode == KDA_GATE_STANDARD) {
+        const float sp = fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+        return -rate * sp;
+    }
+    return graw;
+}
+
+}  // namespace kda

@@ -1,0 +1,59 @@
+// kda_internal.h -- argument bundles and launcher declarations between the C ABI and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+struct DecodeArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    int B, H, HV, K, V;
+    int gate_mode;
+    float lower_bound, scale;
+    int dtype;
+    float* S;
+    void* o;
+    cudaStream_t stream;
+};
+
+struct ChunkArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias, *S0;
+    int B, T, H, HV, K, V, chunk;
+    int gate_mode;
+    float lower_bound, scale;
+    int dtype;
+    void* o;
+    float* S_T;
+    unsigned int* status;  // device status word (first bytes of the workspace)
+    void* scratch;         // workspace beyond the status block
+    size_t scratch_bytes;
+    cudaStream_t stream;
+};
+
+struct GateArgs {
+    const void* g_raw;
+    int dtype;
+    const float *A_log, *dt_bias;
+    long long n;  // B*T*HV*K
+    int HV, K;
+    int gate_mode;
+    float lower_bound;
+    float* g_out;
+    cudaStream_t stream;
+};
+
+// Status word values written by kernels with bounded waits.
+enum : unsigned int { STATUS_OK = 0u, STATUS_TIMEOUT = 1u };
+
+cudaError_t launch_decode_step(const DecodeArgs& a);
+cudaError_t launch_gate(const GateArgs& a);
+cudaError_t launch_chunk_simt(const ChunkArgs& a);
+bool chunk_tc_supported(const ChunkArgs& a);
+cudaError_t launch_chunk_tc(const ChunkArgs& a);
+
+}  // namespace kda

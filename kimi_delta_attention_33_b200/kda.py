@@ -1,0 +1,171 @@
+"""Python binding of ``libkda.so`` (the C ABI in ``include/kda.h``).
+
+Argument marshalling only: every step of the forward pass runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  There is
+no fallback of any kind -- importing this module raises if the shared library is
+missing, and each call raises ``KdaError`` with the library's own message when
+the C ABI returns an error status.
+
+Functions mirror the C entry points:
+
+* ``gate(g_raw, A_log, dt_bias, mode, lower_bound)``  -> float32 log decay
+* ``chunk_fwd(q, k, v, g, beta, ...)``                 -> (o, S_T)
+* ``recurrent_step(q, k, v, g, beta, S, ...)``         -> o  (S updated in place)
+* ``read_status(workspace)``                           -> synchronise and check the device status word
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+GATE_NONE, GATE_SAFE, GATE_STANDARD = 0, 1, 2
+F32, BF16 = 0, 1
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+                4: "KDA_ERR_TIMEOUT"}
+
+# Every symbol include/kda.h declares, in declaration order.
+EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
+           "kda_read_status", "kda_recurrent_step")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kimi_delta_attention_33_b200.build` "
+                      "(this package has no fallback path)")
+
+lib = ctypes.CDLL(LIB_PATH)
+_vp, _fp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+lib.kda_last_error.restype = ctypes.c_char_p
+lib.kda_last_error.argtypes = []
+lib.kda_version.restype = ctypes.c_char_p
+lib.kda_version.argtypes = []
+lib.kda_gate.restype = _i
+lib.kda_gate.argtypes = [_vp, _i, _fp, _fp, _i, _i, _i, _i, _i, _f, _fp, _vp]
+lib.kda_chunk_fwd_workspace_size.restype = _sz
+lib.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
+lib.kda_chunk_fwd.restype = _i
+lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, _vp, _fp, _vp,
+                                                                                  _sz, _vp]
+lib.kda_read_status.restype = _i
+lib.kda_read_status.argtypes = [_vp, _vp]
+lib.kda_recurrent_step.restype = _i
+lib.kda_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, _fp, _vp, _vp]
+
+
+def version() -> str:
+    return lib.kda_version().decode()
+
+
+def last_error() -> str:
+    return lib.kda_last_error().decode()
+
+
+def _check(status: int):
+    if status != OK:
+        raise KdaError(status, last_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise KdaError(ERR_UNSUPPORTED, f"per-token tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise KdaError(ERR_INVALID_ARG, "tensors must be contiguous CUDA tensors")
+
+
+def gate(g_raw: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor | None = None, *, mode: int = GATE_SAFE,
+         lower_bound: float | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Gate activation.  g_raw [B, T, HV, K] -> float32 log decay of the same shape."""
+    _require_cuda(g_raw, A_log, dt_bias)
+    B, T, HV, K = g_raw.shape
+    if out is None:
+        out = torch.empty(g_raw.shape, dtype=torch.float32, device=g_raw.device)
+    lb = float("nan") if lower_bound is None else float(lower_bound)
+    _check(lib.kda_gate(_ptr(g_raw), _dtype_code(g_raw), _ptr(A_log), _ptr(dt_bias), B, T, HV, K, int(mode), lb,
+                        _ptr(out), _stream(g_raw.device)))
+    return out
+
+
+def workspace_size(B, T, H, HV, K, V, chunk) -> int:
+    return int(lib.kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk))
+
+
+def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int = 64,
+              gate_mode: int = GATE_NONE, lower_bound: float | None = None, scale: float | None = None,
+              output_final_state: bool = True, S_T: torch.Tensor | None = None, o: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None):
+    """Chunked prefill.  q, k [B,T,H,K]; v [B,T,HV,V]; g [B,T,HV,K] (g_raw if gate_mode != NONE);
+    beta [B,T,HV]; S0 [B,HV,K,V] fp32 or None.  Returns ``(o, S_T)`` (``S_T`` None unless requested)."""
+    _require_cuda(q, k, v, g, beta, A_log, dt_bias, S0)
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, T, HV, V), dtype=q.dtype, device=q.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((B, HV, K, V), dtype=torch.float32, device=q.device)
+    need = workspace_size(B, T, H, HV, K, V, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    lb = float("nan") if lower_bound is None else float(lower_bound)
+    sc = -1.0 if scale is None else float(scale)
+    _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias), _ptr(S0),
+                             B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q), _ptr(o),
+                             _ptr(S_T), _ptr(workspace), workspace.numel(), _stream(q.device)))
+    return o, S_T
+
+
+def read_status(workspace: torch.Tensor):
+    """Synchronise the current stream and raise ``KdaError`` if a chunk call's bounded wait gave up."""
+    _check(lib.kda_read_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: int = GATE_NONE,
+                   lower_bound: float | None = None, scale: float | None = None, o: torch.Tensor | None = None):
+    """One fused decode step.  q, k [B,H,K] (or [B,1,H,K]); v [B,HV,V]; g [B,HV,K]; beta [B,HV];
+    S [B,HV,K,V] fp32 updated in place.  Returns o [B,HV,V] (shaped like v)."""
+    _require_cuda(q, k, v, g, beta, S, A_log, dt_bias)
+    B, H, K = q.shape[0], q.shape[-2], q.shape[-1]
+    HV, V = v.shape[-2], v.shape[-1]
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    lb = float("nan") if lower_bound is None else float(lower_bound)
+    sc = -1.0 if scale is None else float(scale)
+    _check(lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                                  B, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q), _ptr(S), _ptr(o),
+                                  _stream(q.device)))
+    return o
+
+
+def uses_tensor_cores(K: int, V: int, chunk: int) -> bool:
+    """Whether kda_chunk_fwd runs these sizes on the tensor-core kernel (else the CUDA-core kernel)."""
+    return False
+
+
+def default_scale(K: int) -> float:
+    return 1.0 / math.sqrt(K)

@@ -36,6 +36,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kda_oracle.c")
 _LIB = os.path.join(_HERE, "libkda_oracle.so")
+# The mutation tests point this at a deliberately broken build of a copy of kda_oracle.c.
+_LIB_OVERRIDE = os.environ.get("KDA_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -60,8 +62,11 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+            if _LIB_OVERRIDE:
+                lib = ctypes.CDLL(_LIB_OVERRIDE)
+            else:
+                build()
+                lib = ctypes.CDLL(_LIB)
             dp = ctypes.POINTER(ctypes.c_double)
             lib.kda_oracle_gate.argtypes = [dp, dp, dp, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_double, dp]

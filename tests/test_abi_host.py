@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol
+``include/kda.h`` declares, and rejects bad arguments with the documented status before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kimi_delta_attention_33_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+FAKE = 0x10000  # a 16-byte-aligned non-null address; validation fails before anything touches it
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", text)
+
+
+def test_header_declarations_are_all_exported():
+    names = _declared()
+    assert names, "no declarations parsed"
+    assert tuple(names) == kda.EXPORTS
+    for n in names:
+        assert hasattr(kda.lib, n), f"{n} not exported by libkda.so"
+
+
+def test_version_and_empty_error():
+    assert "sm_100a" in kda.version()
+    assert isinstance(kda.last_error(), str)
+
+
+def _chunk(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, A_log=FAKE, dt_bias=FAKE, S0=None, B=1, T=64, H=2, HV=2,
+             K=128, V=128, chunk=64, gate=kda.GATE_SAFE, lb=-5.0, scale=-1.0, dtype=kda.BF16, o=FAKE * 2,
+             S_T=None, ws=FAKE * 3, ws_bytes=1 << 20, stream=None)
+    a.update(over)
+    return kda.lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["A_log"], a["dt_bias"], a["S0"], a["B"],
+                                 a["T"], a["H"], a["HV"], a["K"], a["V"], a["chunk"], a["gate"], a["lb"], a["scale"],
+                                 a["dtype"], a["o"], a["S_T"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _step(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, A_log=FAKE, dt_bias=None, B=4, H=2, HV=4, K=128, V=128,
+             gate=kda.GATE_SAFE, lb=-5.0, scale=-1.0, dtype=kda.BF16, S=FAKE * 4, o=FAKE * 2, stream=None)
+    a.update(over)
+    return kda.lib.kda_recurrent_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["A_log"], a["dt_bias"], a["B"],
+                                      a["H"], a["HV"], a["K"], a["V"], a["gate"], a["lb"], a["scale"], a["dtype"],
+                                      a["S"], a["o"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), kda.ERR_INVALID_ARG),
+    (dict(o=None), kda.ERR_INVALID_ARG),
+    (dict(HV=3), kda.ERR_INVALID_ARG),
+    (dict(B=0), kda.ERR_INVALID_ARG),
+    (dict(T=0), kda.ERR_INVALID_ARG),
+    (dict(K=48), kda.ERR_UNSUPPORTED),
+    (dict(V=256), kda.ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.ERR_UNSUPPORTED),
+    (dict(lb=float("nan")), kda.ERR_INVALID_ARG),
+    (dict(lb=0.5), kda.ERR_INVALID_ARG),
+    (dict(A_log=None), kda.ERR_INVALID_ARG),
+    (dict(gate=7), kda.ERR_INVALID_ARG),
+    (dict(dtype=5), kda.ERR_INVALID_ARG),
+    (dict(v=FAKE + 4), kda.ERR_INVALID_ARG),
+    (dict(ws=None), kda.ERR_INVALID_ARG),
+    (dict(ws_bytes=16), kda.ERR_INVALID_ARG),
+    (dict(o=FAKE), kda.ERR_INVALID_ARG),
+])
+def test_chunk_fwd_rejects_bad_arguments(over, status):
+    assert _chunk(**over) == status
+    assert kda.last_error() != ""
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(S=None), kda.ERR_INVALID_ARG),
+    (dict(beta=None), kda.ERR_INVALID_ARG),
+    (dict(HV=6, H=4), kda.ERR_INVALID_ARG),
+    (dict(K=100), kda.ERR_UNSUPPORTED),
+    (dict(gate=kda.GATE_SAFE, lb=float("inf")), kda.ERR_INVALID_ARG),
+    (dict(o=FAKE * 4), kda.ERR_INVALID_ARG),
+    (dict(S=FAKE * 4 + 8), kda.ERR_INVALID_ARG),
+])
+def test_recurrent_step_rejects_bad_arguments(over, status):
+    assert _step(**over) == status
+    assert kda.last_error() != ""
+
+
+def test_gate_rejects_bad_arguments():
+    L = kda.lib
+    assert L.kda_gate(None, kda.BF16, FAKE, None, 1, 1, 1, 16, kda.GATE_SAFE, -5.0, FAKE, None) == kda.ERR_INVALID_ARG
+    assert L.kda_gate(FAKE, kda.BF16, FAKE, None, 1, 1, 1, 16, kda.GATE_NONE, -5.0, FAKE, None) == kda.ERR_INVALID_ARG
+    assert L.kda_gate(FAKE, kda.BF16, FAKE, None, 1, 1, 1, 16, kda.GATE_SAFE, float("nan"), FAKE,
+                      None) == kda.ERR_INVALID_ARG
+    assert L.kda_gate(FAKE, kda.BF16, FAKE, None, 0, 1, 1, 16, kda.GATE_STANDARD, 0.0, FAKE,
+                      None) == kda.ERR_INVALID_ARG
+
+
+def test_workspace_size():
+    assert kda.workspace_size(2, 1024, 4, 8, 128, 128, 64) >= 256
+    assert kda.workspace_size(1, 64, 2, 2, 16, 16, 16) >= 256
+    assert kda.workspace_size(1, 64, 2, 3, 16, 16, 16) == 0
+    assert kda.workspace_size(1, 64, 2, 2, 16, 16, 32) == 0
+    assert kda.workspace_size(1, 64, 2, 2, 24, 16, 16) == 0
+
+
+def test_read_status_rejects_null():
+    assert kda.lib.kda_read_status(None, None) == kda.ERR_INVALID_ARG
