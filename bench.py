@@ -196,6 +196,8 @@ def run_ours(args, ws, rank, local):
     from kimi_delta_attention_33_b200 import kda
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
+    if args.B is not None:
+        w = w.scaled(B=args.B)
     torch.manual_seed(0)
     x = make_inputs(w, seed=1000 + w.wid + 7919 * rank, device=str(dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -262,7 +264,7 @@ def run_ours(args, ws, rank, local):
         roof["algorithmic_flops_per_launch"] = prefill_flops(w)
         roof["achieved_tflops"] = round(prefill_flops(w) / kern_s / 1e12, 2)
 
-    e2e = run_e2e(args, w, x, dev, kda) if rank == 0 else None
+    e2e = run_e2e(args, w, x, dev, kda) if (rank == 0 and not args.no_e2e) else None
     decode_extra = None
     if not w.is_decode and not args.no_decode_extra and rank == 0:
         decode_extra = run_decode_extra(args, dev, kda, hbm_peak)
@@ -459,6 +461,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-extra", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--B", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {1: 200, 2: 200, 3: 20, 4: 10, 5: 128}[args.workload] if args.impl == "ours" else 10

@@ -99,6 +99,13 @@ def _require_cuda(*ts):
             raise KdaError(ERR_INVALID_ARG, "tensors must be contiguous CUDA tensors")
 
 
+def _require_out(t, shape, dtype):
+    if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise KdaError(ERR_INVALID_ARG, f"output tensor must be a contiguous CUDA tensor of shape {tuple(shape)} "
+                                        f"and dtype {dtype} (got {tuple(t.shape)}, {t.dtype}, "
+                                        f"contiguous={t.is_contiguous()})")
+
+
 def gate(g_raw: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor | None = None, *, mode: int = GATE_SAFE,
          lower_bound: float | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
     """Gate activation.  g_raw [B, T, HV, K] -> float32 log decay of the same shape."""
@@ -106,6 +113,7 @@ def gate(g_raw: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor | None 
     B, T, HV, K = g_raw.shape
     if out is None:
         out = torch.empty(g_raw.shape, dtype=torch.float32, device=g_raw.device)
+    _require_out(out, g_raw.shape, torch.float32)
     lb = float("nan") if lower_bound is None else float(lower_bound)
     _check(lib.kda_gate(_ptr(g_raw), _dtype_code(g_raw), _ptr(A_log), _ptr(dt_bias), B, T, HV, K, int(mode), lb,
                         _ptr(out), _stream(g_raw.device)))
@@ -129,6 +137,9 @@ def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int
         o = torch.empty((B, T, HV, V), dtype=q.dtype, device=q.device)
     if S_T is None and output_final_state:
         S_T = torch.empty((B, HV, K, V), dtype=torch.float32, device=q.device)
+    _require_out(o, (B, T, HV, V), q.dtype)
+    if S_T is not None:
+        _require_out(S_T, (B, HV, K, V), torch.float32)
     need = workspace_size(B, T, H, HV, K, V, chunk)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
@@ -154,6 +165,8 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
     HV, V = v.shape[-2], v.shape[-1]
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    _require_out(o, v.shape, q.dtype)
+    _require_out(S, (B, HV, K, V), torch.float32)
     lb = float("nan") if lower_bound is None else float(lower_bound)
     sc = -1.0 if scale is None else float(scale)
     _check(lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),

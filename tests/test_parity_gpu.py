@@ -85,13 +85,14 @@ def _decode_run(w, x, steps):
     """`steps` consecutive kda_recurrent_step calls on the workload's [B, steps, ...] token stream."""
     xd = to_dev(x)
     S = xd["S0"].clone() if xd["S0"] is not None else torch.zeros(w.B, w.HV, w.K, w.V, device="cuda")
-    outs = torch.empty(w.B, steps, w.HV, w.V, dtype=w.dtype, device="cuda")
+    outs = []
     for t in range(steps):
-        kda.recurrent_step(xd["q"][:, t].contiguous(), xd["k"][:, t].contiguous(), xd["v"][:, t].contiguous(),
-                           xd["g"][:, t].contiguous(), xd["beta"][:, t].contiguous(), S, xd["A_log"], xd["dt_bias"],
-                           gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=outs[:, t])
+        outs.append(kda.recurrent_step(xd["q"][:, t].contiguous(), xd["k"][:, t].contiguous(),
+                                       xd["v"][:, t].contiguous(), xd["g"][:, t].contiguous(),
+                                       xd["beta"][:, t].contiguous(), S, xd["A_log"], xd["dt_bias"],
+                                       gate_mode=w.gate_mode, lower_bound=w.lower_bound))
     torch.cuda.synchronize()
-    return outs, S
+    return torch.stack(outs, dim=1), S
 
 
 def test_workload5_decode_sampled():
@@ -286,6 +287,15 @@ def test_read_status_ok_after_call():
     ws = torch.zeros(kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk), dtype=torch.uint8, device="cuda")
     _run_chunk(x, w, workspace=ws)
     kda.read_status(ws)
+
+
+def test_non_contiguous_output_rejected():
+    w = _small(T=64)
+    x = to_dev(make_inputs(w))
+    big = torch.empty(w.B, 2 * w.T, w.HV, w.V, dtype=w.dtype, device="cuda")
+    with pytest.raises(kda.KdaError):
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["S0"], chunk=64,
+                      gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=big[:, ::2])
 
 
 def test_invalid_call_launches_nothing():
