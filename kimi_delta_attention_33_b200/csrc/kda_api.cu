@@ -107,7 +107,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                      scale, (int)dtype, o, S_T, static_cast<unsigned int*>(workspace),
                      static_cast<char*>(workspace) + kStatusBytes, workspace_bytes - kStatusBytes,
                      (cudaStream_t)stream};
-    cudaError_t e;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "status word reset");
     if (kda::chunk_tc_supported(a)) {
         e = kda::launch_chunk_tc(a);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel launch");

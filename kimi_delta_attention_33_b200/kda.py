@@ -127,7 +127,7 @@ def workspace_size(B, T, H, HV, K, V, chunk) -> int:
 def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int = 64,
               gate_mode: int = GATE_NONE, lower_bound: float | None = None, scale: float | None = None,
               output_final_state: bool = True, S_T: torch.Tensor | None = None, o: torch.Tensor | None = None,
-              workspace: torch.Tensor | None = None):
+              workspace: torch.Tensor | None = None, check_status: bool = False):
     """Chunked prefill.  q, k [B,T,H,K]; v [B,T,HV,V]; g [B,T,HV,K] (g_raw if gate_mode != NONE);
     beta [B,T,HV]; S0 [B,HV,K,V] fp32 or None.  Returns ``(o, S_T)`` (``S_T`` None unless requested)."""
     _require_cuda(q, k, v, g, beta, A_log, dt_bias, S0)
@@ -148,6 +148,8 @@ def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int
     _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias), _ptr(S0),
                              B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q), _ptr(o),
                              _ptr(S_T), _ptr(workspace), workspace.numel(), _stream(q.device)))
+    if check_status:
+        read_status(workspace)
     return o, S_T
 
 
@@ -175,9 +177,9 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
     return o
 
 
-def uses_tensor_cores(K: int, V: int, chunk: int) -> bool:
+def uses_tensor_cores(K: int, V: int, chunk: int, dtype: torch.dtype = torch.bfloat16) -> bool:
     """Whether kda_chunk_fwd runs these sizes on the tensor-core kernel (else the CUDA-core kernel)."""
-    return False
+    return dtype == torch.bfloat16 and K == 128 and chunk == 64 and V in (64, 128)
 
 
 def default_scale(K: int) -> float:

@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _run_chunk(xd, w, **kw):
+    kw.setdefault("check_status", "workspace" not in kw)
     return kda.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"], xd["S0"],
                          chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, **kw)
 
