@@ -55,4 +55,17 @@ __device__ __forceinline__ float gate_value(float graw, float bias, float rate, 
     return graw;
 }
 
+// The same gate with the fast hardware exponential / division / logarithm (relative error ~1e-6,
+// far below the tf32 operand rounding of the tensor-core path that uses it).
+__device__ __forceinline__ float gate_value_fast(float graw, float bias, float rate, int mode, float lower_bound) {
+    const float x = graw + bias;
+    if (mode == KDA_GATE_SAFE) {
+        return __fdividef(lower_bound, 1.0f + __expf(-rate * x));
+    } else if (mode == KDA_GATE_STANDARD) {
+        const float sp = fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x)));
+        return -rate * sp;
+    }
+    return graw;
+}
+
 }  // namespace kda

@@ -43,6 +43,24 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
+// Same MMA with the A operand read from TMEM (row m in lane m, contraction index along columns;
+// the tensor core takes the top 19 bits of each fp32 word, i.e. truncates it to tf32).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// D[M x N] (+)= A_tmem[M x 8*ksteps] * B[N x 8*ksteps]^T: one K = 8 step per 8 TMEM columns of A.
+__device__ __forceinline__ void gemm_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, uint32_t b_sbo,
+                                             uint32_t idesc, int ksteps, bool accumulate) {
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_tf32_ts(d_tmem, a_tmem + 8u * ks, smem_desc(b_addr + ks * 256u, b_sbo), idesc,
+                    (ks > 0 || accumulate) ? 1u : 0u);
+}
+
 // D[M x N] (+)= A[M x 8*ksteps] * B[N x 8*ksteps]^T, operands in the tiling above.
 __device__ __forceinline__ void gemm_tf32(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
                                           uint32_t b_sbo, uint32_t idesc, int ksteps, bool accumulate) {

@@ -179,7 +179,7 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
 
 def uses_tensor_cores(K: int, V: int, chunk: int, dtype: torch.dtype = torch.bfloat16) -> bool:
     """Whether kda_chunk_fwd runs these sizes on the tensor-core kernel (else the CUDA-core kernel)."""
-    return dtype == torch.bfloat16 and K == 128 and chunk == 64 and V in (64, 128)
+    return dtype == torch.bfloat16 and K == 128 and chunk == 64 and V == 128
 
 
 def default_scale(K: int) -> float:
