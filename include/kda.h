@@ -125,6 +125,37 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
  */
 kda_status kda_read_status(const void* workspace, kda_stream_t stream);
 
+/* Size, in bytes, of the built-in workspace behind kda_chunk_fwd_noalloc. */
+#define KDA_NOALLOC_SCRATCH_BYTES 4096
+
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it is an interface convenience of this library.
+ * Who needs it: code that only ever holds pointers to buffers owned by someone else -- e.g. a
+ * host application or plugin handed its tensors by an outer runtime that keeps a fixed
+ * device-memory budget and exposes no allocator, or a latency-critical serving loop in which
+ * allocating on the call path is not allowed -- and so has no workspace to pass.
+ * Arguments, layouts, results and errors are those of kda_chunk_fwd without the workspace: the
+ * library supplies it from a fixed array of KDA_NOALLOC_SCRATCH_BYTES bytes of device memory that
+ * is part of the library (every GPU that loads the library holds it until the process exits).
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.
+ *   - The first call on a device resolves the array's device address on that device
+ *     (cudaGetSymbolAddress with the device current); make that first call before any stream
+ *     capture.
+ *   - Sizes that would need more workspace than KDA_NOALLOC_SCRATCH_BYTES return
+ *     KDA_ERR_UNSUPPORTED with a message; nothing is launched.
+ *   - Every call uses the same array and leaves its contents behind; each call clears the part
+ *     that must start at zero (the status word).  Calls whose work overlaps on the GPU (for
+ *     example on two streams at once) race on the array: order them on one stream.  The status
+ *     word is internal, so a bounded on-device wait that gives up cannot be read back through
+ *     kda_read_status here.
+ */
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                 const void* beta, const float* A_log, const float* dt_bias,
+                                 const float* S0, int B, int T, int H, int HV, int K, int V, int chunk,
+                                 kda_gate_mode gate_mode, float lower_bound, float scale,
+                                 kda_dtype dtype, void* o, float* S_T, kda_stream_t stream);
+
 /*
  * kda_recurrent_step -- one decode step for a batch of sequences, fused
  * (DeltaNet-family digest, "decode के लिए fused recurrent Triton kernel": the

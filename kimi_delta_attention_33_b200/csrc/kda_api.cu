@@ -57,6 +57,10 @@ constexpr size_t kStatusBytes = 256;
 
 }  // namespace
 
+namespace kda {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace kda
+
 extern "C" {
 
 const char* kda_last_error(void) { return g_err; }

@@ -50,6 +50,9 @@ struct GateArgs {
 // Status word values written by kernels with bounded waits.
 enum : unsigned int { STATUS_OK = 0u, STATUS_TIMEOUT = 1u };
 
+// Sets the thread-local message kda_last_error() returns.
+void set_last_error(const char* msg);
+
 cudaError_t launch_decode_step(const DecodeArgs& a);
 cudaError_t launch_gate(const GateArgs& a);
 cudaError_t launch_chunk_simt(const ChunkArgs& a);

@@ -1,0 +1,75 @@
+// kda_noalloc.cu -- kda_chunk_fwd for callers that cannot allocate device memory.
+//
+// Some callers only ever hold pointers to buffers that someone else owns: a host application
+// or plugin that receives its tensors from an outer runtime with a fixed device-memory budget
+// and no allocator to hand out, or a latency-critical serving loop where allocating on the call
+// path is forbidden.  Such a caller cannot provide the workspace kda_chunk_fwd asks for.  This
+// entry point supplies that workspace itself, from a fixed array in device memory that is part
+// of this library (every GPU that loads the library holds it until the process exits), and then
+// runs exactly the same prefill as kda_chunk_fwd.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "kda_internal.h"
+
+namespace {
+
+// Upper bound on the workspace kda_chunk_fwd may need; larger requests are rejected.
+constexpr size_t kScratchBytes = KDA_NOALLOC_SCRATCH_BYTES;
+
+// The workspace of every kda_chunk_fwd_noalloc call.  In host code this name is only a
+// stand-in for the symbol, not a device address: its address on the current device comes
+// from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                            const void* beta, const float* A_log, const float* dt_bias,
+                                            const float* S0, int B, int T, int H, int HV, int K, int V, int chunk,
+                                            kda_gate_mode gate_mode, float lower_bound, float scale,
+                                            kda_dtype dtype, void* o, float* S_T, kda_stream_t stream) {
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk);
+    char msg[192];
+    if (need > kScratchBytes) {
+        // kda_chunk_fwd's own validation reports the sizes it rejects outright (need == 0).
+        snprintf(msg, sizeof(msg), "kda_chunk_fwd_noalloc: these sizes need %zu bytes of workspace, more than the "
+                 "built-in %zu bytes", need, kScratchBytes);
+        kda::set_last_error(msg);
+        return KDA_ERR_UNSUPPORTED;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        snprintf(msg, sizeof(msg), "kda_chunk_fwd_noalloc: cudaGetDevice failed (%s)", cudaGetErrorString(e));
+        kda::set_last_error(msg);
+        return KDA_ERR_CUDA;
+    }
+    void* scratch = nullptr;
+    {
+        // One-time set-up per device, with that device current: resolve the array's device address.
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_scratch_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess || p == nullptr) {
+                snprintf(msg, sizeof(msg), "kda_chunk_fwd_noalloc: cudaGetSymbolAddress failed (%s)",
+                         cudaGetErrorString(e));
+                kda::set_last_error(msg);
+                return KDA_ERR_CUDA;
+            }
+            g_scratch_ptr[dev] = p;
+        }
+        scratch = g_scratch_ptr[dev];
+    }
+    // kda_chunk_fwd clears the status word at the start of the array before launching; nothing else
+    // in the array needs to start at zero.
+    return kda_chunk_fwd(q, k, v, g, beta, A_log, dt_bias, S0, B, T, H, HV, K, V, chunk, gate_mode, lower_bound,
+                         scale, dtype, o, S_T, scratch, kScratchBytes, stream);
+}

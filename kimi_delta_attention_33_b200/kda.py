@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Every symbol include/kda.h declares, in declaration order.
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
-           "kda_read_status", "kda_recurrent_step")
+           "kda_read_status", "kda_chunk_fwd_noalloc", "kda_recurrent_step")
 
 
 class KdaError(RuntimeError):
@@ -60,6 +60,9 @@ lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7
                                                                                   _sz, _vp]
 lib.kda_read_status.restype = _i
 lib.kda_read_status.argtypes = [_vp, _vp]
+lib.kda_chunk_fwd_noalloc.restype = _i
+lib.kda_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, _vp, _fp,
+                                                                                          _vp]
 lib.kda_recurrent_step.restype = _i
 lib.kda_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, _fp, _vp, _vp]
 
@@ -150,6 +153,29 @@ def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int
                              _ptr(S_T), _ptr(workspace), workspace.numel(), _stream(q.device)))
     if check_status:
         read_status(workspace)
+    return o, S_T
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int = 64,
+                      gate_mode: int = GATE_NONE, lower_bound: float | None = None, scale: float | None = None,
+                      S_T: torch.Tensor | None = None, o: torch.Tensor | None = None):
+    """``chunk_fwd`` through ``kda_chunk_fwd_noalloc``: the library supplies the workspace from its own
+    fixed device array, for callers that cannot allocate one.  Outputs are still passed in (or made
+    here by torch when omitted)."""
+    _require_cuda(q, k, v, g, beta, A_log, dt_bias, S0)
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, T, HV, V), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, HV, K, V), dtype=torch.float32, device=q.device)
+    _require_out(o, (B, T, HV, V), q.dtype)
+    _require_out(S_T, (B, HV, K, V), torch.float32)
+    lb = float("nan") if lower_bound is None else float(lower_bound)
+    sc = -1.0 if scale is None else float(scale)
+    _check(lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                                     _ptr(S0), B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q),
+                                     _ptr(o), _ptr(S_T), _stream(q.device)))
     return o, S_T
 
 
