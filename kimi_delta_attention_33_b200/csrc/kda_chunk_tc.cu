@@ -24,7 +24,7 @@
 // State side, transposed so the state stays in TMEM and feeds the tensor core directly.
 // One CTA owns one (b, hv) pair: TMEM D4[v][d] holds S_c^T diag(e^rho) (lane = value column v).
 //   M1  D1[128 x 64] = [Qhat; -Khat] Kchk^T                  -> A (rows 0-63), -R/beta (rows 64-127)
-//   T = (I + R)^{-1} on the CUDA cores (16 x 16 diagonal blocks, then two doubling steps), Tb = T diag(beta)
+//   T = (I + R)^{-1} on the CUDA cores (block doubling, 2 x 2 up to 64 x 64), Tb = T diag(beta)
 //   M3  D3[v][i]    = D4 (A from TMEM) . [Qhat; -Khat]^T      -> (Qtil S_c)^T (i < 64), -(Ktil S_c)^T (i >= 64)
 //   M2  D2[v][j]    = V^T Tb^T                                -> U^T
 //   M4  D2         += D3[:, 64:] (A from TMEM) Tb^T           -> E^T = (U - Tb Ktil S_c)^T
@@ -98,6 +98,45 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
 
 __device__ __forceinline__ float bf16_bits_to_f32(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
 
+// One doubling step of the unit-lower-triangular inverse, in place over the strictly-lower part
+// stored with row pitch RP: every diagonal block of size 2 HS, [[Ta, 0], [C, Td]], whose diagonal
+// sub-blocks already hold their inverses, gets its lower-left block -Td C Ta (Ta, Td with implicit
+// unit diagonals).  X = C Ta goes through the scratch sX.
+template <int HS>
+__device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid) {
+    constexpr int CNT = (CH / (2 * HS)) * HS * HS;
+    constexpr int ITERS = (CNT + TC_THREADS - 1) / TC_THREADS;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int e = tid + TC_THREADS * it;
+        if (CNT % TC_THREADS == 0 || e < CNT) {
+            const int c = e % HS, r = (e / HS) % HS, base = (e / (HS * HS)) * 2 * HS;
+            const float* Crow = sRT + (base + HS + r) * RP + base;
+            float acc = Crow[c];
+#pragma unroll
+            for (int m = 1; m < HS; ++m)
+                if (m > c) acc += Crow[m] * sRT[(base + m) * RP + base + c];
+            sX[e] = acc;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int e = tid + TC_THREADS * it;
+        if (CNT % TC_THREADS == 0 || e < CNT) {
+            const int c = e % HS, r = (e / HS) % HS, blk = e / (HS * HS), base = blk * 2 * HS;
+            const float* Drow = sRT + (base + HS + r) * RP + base + HS;
+            const float* Xb = sX + blk * HS * HS;
+            float acc = Xb[r * HS + c];
+#pragma unroll
+            for (int m = 0; m < HS - 1; ++m)
+                if (m < r) acc += Drow[m] * Xb[m * HS + c];
+            sRT[(base + HS + r) * RP + base + c] = -acc;
+        }
+    }
+    __syncthreads();
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -118,7 +157,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::GM);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
-    const bf16* sG = reinterpret_cast<const bf16*>(smem + L::AT);
+    const bf16* sG = reinterpret_cast<const bf16*>(smem + L::GM);  // g tile staging (bf16 [64][128])
     uint32_t* sFlag = reinterpret_cast<uint32_t*>(smem + L::FLAG);
     const uint32_t s_base = smem_u32(smem);
     const uint32_t mbar = s_base + L::MBAR;
@@ -153,57 +192,67 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     uint32_t phase = 0;
     bool aborted = false;
 
-    for (int t0 = 0; t0 < T && !aborted; t0 += CH) {
-        const int n = min(CH, T - t0);
-        const int m_ref = (n - 1) >> 1;
-        const size_t tok0 = (size_t)b * T + t0;
-
-        // ---- P1: issue every global load of this chunk before any arithmetic -------------------
-        uint4 qr[4], kr[4], gr[4];
+    // Input staging.  A chunk's g and v tiles go to GM by cp.async, issued while the tensor core runs
+    // the previous chunk's state chain (GM is idle then); its q, k and beta go to registers, loaded
+    // right after that chain completes.  Rows past T are zero-filled.
+    const uint32_t gm_addr = s_base + L::GM;
+    auto prefetch_gv = [&](int tc0) {
+        const int nn = min(CH, T - tc0);
+        const size_t tk0 = (size_t)b * T + tc0;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int u = tid + TC_THREADS * it;
+            const int i = u >> 4, c = u & 15;
+            const bool ok = i < nn;
+            cp_async16(gm_addr + i * 256 + c * 16, ok ? g + (tk0 + i) * g_row + (size_t)hv * KD + 8 * c : g, ok ? 16u : 0u);
+            cp_async16(gm_addr + 16384 + i * 256 + c * 16, ok ? v + (tk0 + i) * v_row + (size_t)hv * VD + 8 * c : v,
+                       ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    uint4 qr[4], kr[4];
+    float bload;
+    auto load_qkb = [&](int tc0) {
+        const int nn = min(CH, T - tc0);
+        const size_t tk0 = (size_t)b * T + tc0;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
             const int u = tid + TC_THREADS * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
             qr[it] = make_uint4(0u, 0u, 0u, 0u);
             kr[it] = qr[it];
-            if (i < n) {
-                qr[it] = __ldg(reinterpret_cast<const uint4*>(q + (tok0 + i) * qk_row + (size_t)h * KD + 8 * d8));
-                kr[it] = __ldg(reinterpret_cast<const uint4*>(k + (tok0 + i) * qk_row + (size_t)h * KD + 8 * d8));
+            if (i < nn) {
+                qr[it] = __ldg(reinterpret_cast<const uint4*>(q + (tk0 + i) * qk_row + (size_t)h * KD + 8 * d8));
+                kr[it] = __ldg(reinterpret_cast<const uint4*>(k + (tk0 + i) * qk_row + (size_t)h * KD + 8 * d8));
             }
-            const int gi = u >> 4, gc = u & 15;
-            gr[it] = make_uint4(0u, 0u, 0u, 0u);
-            if (gi < n) gr[it] = __ldg(reinterpret_cast<const uint4*>(g + (tok0 + gi) * g_row + (size_t)hv * KD + 8 * gc));
         }
-        // value tile, one value column per thread, tokens 4 jq .. 4 jq + 3 for jq = tid/128 + 2 x
-        const int vc = tid & (VD - 1), jq0 = tid >> 7;
-        unsigned short vv[32];
-        {
-            const unsigned short* vp = reinterpret_cast<const unsigned short*>(v) + (size_t)hv * VD + vc;
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int j = 4 * (jq0 + 2 * x) + r;
-                    vv[4 * x + r] = (j < n) ? __ldg(vp + (tok0 + j) * v_row) : (unsigned short)0;
-                }
-        }
-        const float bload = (tid < n) ? to_f32(beta[(tok0 + tid) * HV + hv]) : 0.f;  // tid < n <= 64
+        bload = (tid < nn) ? to_f32(beta[(tk0 + tid) * HV + hv]) : 0.f;  // tid < nn <= 64
+    };
+    prefetch_gv(0);
+    load_qkb(0);
 
-        // ---- P2: gate + in-chunk inclusive cumulative log decay (two threads per channel) -------
+    for (int t0 = 0; t0 < T && !aborted; t0 += CH) {
+        const int n = min(CH, T - t0);
+        const int m_ref = (n - 1) >> 1;
+        const size_t tok0 = (size_t)b * T + t0;
+
+        // ---- P2: the chunk's g and v tiles arrived in GM by cp.async; V^T -> VE, beta ----------
+        cp_async_wait_all();
+        __syncthreads();
+        {
+            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::GM + 16384);
+            const int vc = tid & (VD - 1), jq0 = tid >> 7;  // one value column, token quads jq0 + 2 x
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
-            *reinterpret_cast<uint4*>(smem + L::AT + (u >> 4) * (KD * 2) + (u & 15) * 16) = gr[it];
-        }
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-            const int jq = jq0 + 2 * x;
-            *reinterpret_cast<uint4*>(smem + L::VE + cm_off(vc, 4 * jq, CH)) =
-                make_uint4(to_tf32(bf16_bits_to_f32(vv[4 * x])), to_tf32(bf16_bits_to_f32(vv[4 * x + 1])),
-                           to_tf32(bf16_bits_to_f32(vv[4 * x + 2])), to_tf32(bf16_bits_to_f32(vv[4 * x + 3])));
+            for (int x = 0; x < 8; ++x) {
+                const int j = 4 * (jq0 + 2 * x);
+                *reinterpret_cast<uint4*>(smem + L::VE + cm_off(vc, j, CH)) =
+                    make_uint4(to_tf32(bf16_bits_to_f32(sVs[(j + 0) * VD + vc])),
+                               to_tf32(bf16_bits_to_f32(sVs[(j + 1) * VD + vc])),
+                               to_tf32(bf16_bits_to_f32(sVs[(j + 2) * VD + vc])),
+                               to_tf32(bf16_bits_to_f32(sVs[(j + 3) * VD + vc])));
+            }
         }
         if (tid < CH) sBeta[tid] = bload;
-        __syncthreads();
         const int gd = tid & (KD - 1), gh = tid >> 7;  // gate channel, token half
         float gv[32];
         {
@@ -367,81 +416,13 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         __syncthreads();
 
-        // ---- P6: T = (I + R)^{-1}, in place over R --------------------------------------------
-        // (a) the four 16 x 16 diagonal blocks, one column per thread (64 threads);
-        // (b) two doubling steps: the inverse of [[Ta, 0], [C, Td]] has lower-left block -Td C Ta,
-        //     with Ta, Td the already inverted diagonal blocks (unit diagonals implicit).
-        {
-            float col[16];
-            const int blk = (tid >> 4) & 3, c = tid & 15, base = 16 * blk;
-            if (tid < 64) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int m = 0; m < r; ++m) acc += (m >= c) ? sRT[(base + r) * RP + base + m] * col[m] : 0.f;
-                    col[r] = (r < c) ? 0.f : ((r == c) ? 1.f : -acc);
-                }
-            }
-            __syncthreads();
-            if (tid < 64) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (r > c) sRT[(base + r) * RP + base + c] = col[r];
-            }
-        }
-        __syncthreads();
-        {   // doubling step 16 -> 32: blocks at base 0 and 32
-            const int r = tid >> 4, c = tid & 15;
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int base = 32 * x;
-                const float* Crow = sRT + (base + 16 + r) * RP + base;
-                float acc = Crow[c];
-#pragma unroll
-                for (int m = 1; m < 16; ++m)
-                    if (m > c) acc += Crow[m] * sRT[(base + m) * RP + base + c];
-                sX[x * 256 + r * 16 + c] = acc;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int base = 32 * x;
-                const float* Drow = sRT + (base + 16 + r) * RP + base + 16;
-                const float* Xb = sX + x * 256;
-                float acc = Xb[r * 16 + c];
-#pragma unroll
-                for (int m = 0; m < 15; ++m)
-                    if (m < r) acc += Drow[m] * Xb[m * 16 + c];
-                sRT[(base + 16 + r) * RP + base + c] = -acc;
-            }
-        }
-        __syncthreads();
-        {   // doubling step 32 -> 64
-            const int c = tid & 31;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int r = (tid >> 5) + 8 * x;
-                const float* Crow = sRT + (32 + r) * RP;
-                float acc = Crow[c];
-#pragma unroll
-                for (int m = 1; m < 32; ++m)
-                    if (m > c) acc += Crow[m] * sRT[m * RP + c];
-                sX[r * 32 + c] = acc;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int r = (tid >> 5) + 8 * x;
-                const float* Drow = sRT + (32 + r) * RP + 32;
-                float acc = sX[r * 32 + c];
-#pragma unroll
-                for (int m = 0; m < 31; ++m)
-                    if (m < r) acc += Drow[m] * sX[m * 32 + c];
-                sRT[(32 + r) * RP + c] = -acc;
-            }
-        }
-        __syncthreads();
+        // ---- P6: T = (I + R)^{-1}, in place over R, by six doubling steps (block sizes 2 .. 64) --
+        tri_inverse_step<1>(sRT, sX, tid);
+        tri_inverse_step<2>(sRT, sX, tid);
+        tri_inverse_step<4>(sRT, sX, tid);
+        tri_inverse_step<8>(sRT, sX, tid);
+        tri_inverse_step<16>(sRT, sX, tid);
+        tri_inverse_step<32>(sRT, sX, tid);
         // Tb = T diag(beta) as tf32 into AT rows 64-127
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
@@ -458,6 +439,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         fence_proxy_async();
         cta_sync_tc();
+        if (t0 + CH < T) prefetch_gv(t0 + CH);  // GM (R/T) is no longer needed by this chunk
 
         // ---- state chain: M3, M2, M4, M5, M6 back to back (fast path) --------------------------
         if (tid == 0) {
@@ -502,6 +484,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             if (!__syncthreads_and(ok)) { aborted = true; break; }
             phase ^= 1u;
         }
+
+        if (t0 + CH < T) load_qkb(t0 + CH);
 
         // ---- outputs: O^T in D3 columns 0-63 (lane = value column) ----------------------------
         {

@@ -147,6 +147,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t a, const uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16-byte asynchronous global -> shared copy; src_bytes < 16 zero-fills the rest (0: all zeros).
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // Round-to-nearest fp32 -> tf32 (low 13 mantissa bits cleared); the tensor core reads the rest.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
