@@ -48,7 +48,7 @@ constexpr int TC_THREADS = 256;
 constexpr int KD = 128;  // key dimension handled by this kernel
 constexpr int VD = 128;  // value dimension handled by this kernel (one CTA owns all of it)
 constexpr int CH = 64;   // chunk length handled by this kernel
-constexpr int RP = 65;   // row pitch (floats) of the R / T scratch
+constexpr int RP = 68;   // row pitch (floats) of the R / T scratch: 16-byte aligned rows
 constexpr float SPAN_LIMIT = 40.0f;
 constexpr uint32_t WAIT_POLLS = 1u << 26;
 
@@ -134,6 +134,93 @@ __device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid)
             sRT[(base + HS + r) * RP + base + c] = -acc;
         }
     }
+    __syncthreads();
+}
+
+// The last two doubling steps with one column per lane and four rows per thread: X = C Ta and the
+// new block -Td X, accumulating over m with loads of four consecutive row entries at a time.
+// Step 16 -> 32 (two blocks, at 0 and 32): warp w serves block w / 4 and rows 4 (w % 4) .. + 3 of its
+// 16 x 16 lower-left block; lane = column (lane % 16) and row pair (lane / 16).
+__device__ __forceinline__ void tri_inverse_step16(float* sRT, float* sX, int tid) {
+    const int w = tid >> 5, lane = tid & 31;
+    const int base = 32 * (w >> 2), c = lane & 15;
+    const int r0 = 4 * (w & 3) + 2 * (lane >> 4);  // rows r0, r0 + 1 of the 16 x 16 lower-left block
+    float acc[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) acc[x] = sRT[(base + 16 + r0 + x) * RP + base + c];
+#pragma unroll
+    for (int m4 = 0; m4 < 16; m4 += 4) {
+        float a[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) a[t] = (m4 + t > c) ? sRT[(base + m4 + t) * RP + base + c] : 0.f;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const float4 cr = *reinterpret_cast<const float4*>(sRT + (base + 16 + r0 + x) * RP + base + m4);
+            acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) sX[(w >> 2) * 256 + (r0 + x) * 16 + c] = acc[x];
+    __syncthreads();
+    const float* Xb = sX + (w >> 2) * 256;
+#pragma unroll
+    for (int x = 0; x < 2; ++x) acc[x] = Xb[(r0 + x) * 16 + c];
+#pragma unroll
+    for (int m4 = 0; m4 < 16; m4 += 4) {
+        float xm[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) xm[t] = Xb[(m4 + t) * 16 + c];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const float4 dr = *reinterpret_cast<const float4*>(sRT + (base + 16 + r0 + x) * RP + base + 16 + m4);
+            const int r = r0 + x;
+            acc[x] += (m4 + 0 < r ? dr.x * xm[0] : 0.f) + (m4 + 1 < r ? dr.y * xm[1] : 0.f) +
+                      (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) sRT[(base + 16 + r0 + x) * RP + base + c] = -acc[x];
+    __syncthreads();
+}
+
+// Step 32 -> 64 (one block): warp w serves rows 4 w + {0..3}, lane = column.
+__device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int tid) {
+    const int w = tid >> 5, c = tid & 31, r0 = 4 * w;
+    float acc[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) acc[x] = sRT[(32 + r0 + x) * RP + c];
+#pragma unroll
+    for (int m4 = 0; m4 < 32; m4 += 4) {
+        float a[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) a[t] = (m4 + t > c) ? sRT[(m4 + t) * RP + c] : 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float4 cr = *reinterpret_cast<const float4*>(sRT + (32 + r0 + x) * RP + m4);
+            acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) sX[(r0 + x) * 32 + c] = acc[x];
+    __syncthreads();
+#pragma unroll
+    for (int x = 0; x < 4; ++x) acc[x] = sX[(r0 + x) * 32 + c];
+#pragma unroll
+    for (int m4 = 0; m4 < 32; m4 += 4) {
+        if (m4 >= r0 + 3) break;  // warp-uniform: no row of this warp reaches these m
+        float xm[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) xm[t] = sX[(m4 + t) * 32 + c];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float4 dr = *reinterpret_cast<const float4*>(sRT + (32 + r0 + x) * RP + 32 + m4);
+            const int r = r0 + x;
+            acc[x] += (m4 + 0 < r ? dr.x * xm[0] : 0.f) + (m4 + 1 < r ? dr.y * xm[1] : 0.f) +
+                      (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) sRT[(32 + r0 + x) * RP + c] = -acc[x];
     __syncthreads();
 }
 
@@ -292,7 +379,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             else sig = rho;
             sRho[d] = rho;
             sSig[d] = sig;
-            sERho[d] = __expf(rho);
+            sERho[d] = sFpend[d] * __expf(rho);  // D4 rescale: previous chunk's pending factor and e^rho
             sESig[d] = __expf(sig);
             sFnext[d] = __expf(sGam[gidx(CH - 1, d)] - sig);  // pending per-key factor of D4 after this chunk
         }
@@ -342,7 +429,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-                row.r[c] = __float_as_uint(sFpend[d0 + c] * sERho[d0 + c] * __uint_as_float(row.r[c]));
+                row.r[c] = __float_as_uint(sERho[d0 + c] * __uint_as_float(row.r[c]));
             row.store(taddr(tmem, 32 * wq, L::D4 + d0));
         }
         tmem_wait_st();
@@ -421,18 +508,20 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         tri_inverse_step<2>(sRT, sX, tid);
         tri_inverse_step<4>(sRT, sX, tid);
         tri_inverse_step<8>(sRT, sX, tid);
-        tri_inverse_step<16>(sRT, sX, tid);
-        tri_inverse_step<32>(sRT, sX, tid);
+        tri_inverse_step16(sRT, sX, tid);
+        tri_inverse_step32(sRT, sX, tid);
         // Tb = T diag(beta) as tf32 into AT rows 64-127
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             const int u = tid + TC_THREADS * x;
             const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
             uint32_t w[4];
+            const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
+            const float tr[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
                 const int j = 4 * j4 + t;
-                const float tv = (j < i) ? sRT[i * RP + j] : (j == i ? 1.f : 0.f);
+                const float tv = (j < i) ? tr[t] : (j == i ? 1.f : 0.f);
                 w[t] = to_tf32(tv * sBeta[j]);
             }
             *reinterpret_cast<uint4*>(smem + L::AT + cm_off(64 + i, 4 * j4, CH)) = make_uint4(w[0], w[1], w[2], w[3]);
