@@ -68,7 +68,9 @@ struct TcLayout {
     static constexpr uint32_t MBAR = BETA + 256;  // 8 B
     static constexpr uint32_t TBASE = MBAR + 8;   // 4 B
     static constexpr uint32_t FLAG = TBASE + 4;   // 4 B
-    static constexpr uint32_t BYTES = FLAG + 4;
+    static constexpr uint32_t VS = VEC + 4096;    // bf16 [64][128] staging of the next chunk's v tile
+    static constexpr uint32_t BYTES = VS + 64 * VD * 2;
+    static_assert(FLAG + 4 <= VS, "vector region");
     // TMEM columns (all accumulators M = 128: TMEM lane = row)
     static constexpr int D4 = 0;     // state^T [v][d], 128 columns
     static constexpr int D3 = 128;   // [v][i]: 0-63 outputs, 64-127 -P
@@ -279,29 +281,27 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     uint32_t phase = 0;
     bool aborted = false;
 
-    // Input staging.  A chunk's g and v tiles go to GM by cp.async, issued while the tensor core runs
-    // the previous chunk's state chain (GM is idle then); its q, k and beta go to registers, loaded
-    // right after that chain completes.  Rows past T are zero-filled.
+    // Input staging and the gate, one chunk ahead.  While the tensor core runs chunk c's state chain
+    // (which reads X1, AT, X2, VE and TMEM only), the CUDA cores load chunk c+1's q, k, v, beta into
+    // registers, bring its g tile into GM by cp.async, and run its gate and in-chunk cumulative decay
+    // into GM.  Rows past T are zero-filled.
     const uint32_t gm_addr = s_base + L::GM;
-    auto prefetch_gv = [&](int tc0) {
+    uint4 qr[4], kr[4];
+    float bload;
+    const int vc = tid & (VD - 1), jq0 = tid >> 7;  // value column, first token quad (quads jq0 + 2 x)
+    auto load_inputs = [&](int tc0) {
         const int nn = min(CH, T - tc0);
         const size_t tk0 = (size_t)b * T + tc0;
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
+        for (int it = 0; it < 4; ++it) {  // g tile -> GM staging, v tile -> VS staging, bf16 [64][128]
             const int u = tid + TC_THREADS * it;
             const int i = u >> 4, c = u & 15;
             const bool ok = i < nn;
             cp_async16(gm_addr + i * 256 + c * 16, ok ? g + (tk0 + i) * g_row + (size_t)hv * KD + 8 * c : g, ok ? 16u : 0u);
-            cp_async16(gm_addr + 16384 + i * 256 + c * 16, ok ? v + (tk0 + i) * v_row + (size_t)hv * VD + 8 * c : v,
+            cp_async16(s_base + L::VS + i * 256 + c * 16, ok ? v + (tk0 + i) * v_row + (size_t)hv * VD + 8 * c : v,
                        ok ? 16u : 0u);
         }
         cp_async_commit();
-    };
-    uint4 qr[4], kr[4];
-    float bload;
-    auto load_qkb = [&](int tc0) {
-        const int nn = min(CH, T - tc0);
-        const size_t tk0 = (size_t)b * T + tc0;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
             const int u = tid + TC_THREADS * it;
@@ -315,20 +315,72 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         bload = (tid < nn) ? to_f32(beta[(tk0 + tid) * HV + hv]) : 0.f;  // tid < nn <= 64
     };
-    prefetch_gv(0);
-    load_qkb(0);
+    // Gate + inclusive in-chunk cumulative log decay of the chunk at tc0 (two threads per key channel),
+    // its beta, the fast/exact decision and the per-channel vectors.  Uses sFpend, the pending state
+    // factor the chunk starts from.  Returns whether the chunk takes the exact path.
+    auto stage_gate = [&](int tc0) -> bool {
+        const int nn = min(CH, T - tc0), mr = (nn - 1) >> 1;
+        cp_async_wait_all();
+        __syncthreads();
+        if (tid < CH) sBeta[tid] = bload;
+        const int gd = tid & (KD - 1), gh = tid >> 7;
+        float gv[32];
+        {
+            const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int i = 32 * gh + r;
+                const float x = (i < nn) ? gate_value_fast(__bfloat162float(sG[i * KD + gd]), bias, rate, gate_mode,
+                                                           lower_bound)
+                                         : 0.f;
+                acc += x;
+                gv[r] = acc;
+            }
+            if (gh == 0) sFnext[gd] = acc;  // scratch: first-half totals
+        }
+        __syncthreads();  // the g staging has been read: GM becomes Gam
+        {
+            const float off = gh ? sFnext[gd] : 0.f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) sGam[gidx(32 * gh + r, gd)] = gv[r] + off;
+        }
+        __syncthreads();
+        if (tid < KD) {
+            const int d = tid;
+            const float g0 = sGam[gidx(0, d)], gm = sGam[gidx(mr, d)], gend = sGam[gidx(nn - 1, d)];
+            if (!(fmaxf(g0 - gm, gm - gend) <= SPAN_LIMIT)) atomicOr(sFlag, 1u);
+            sRho[d] = gm;
+            sSig[d] = gend;
+        }
+        __syncthreads();
+        const bool slow_c = (*reinterpret_cast<volatile uint32_t*>(sFlag)) != 0;
+        if (tid < KD) {
+            const int d = tid;
+            float rho = sRho[d], sig = sSig[d];
+            if (slow_c) rho = 0.f;  // sig stays Gam_end: Kchk becomes Kend
+            else sig = rho;
+            sRho[d] = rho;
+            sSig[d] = sig;
+            sERho[d] = sFpend[d] * __expf(rho);  // D4 rescale: the pending factor and e^rho
+            sESig[d] = __expf(sig);
+            sFnext[d] = __expf(sGam[gidx(CH - 1, d)] - sig);  // pending per-key factor of D4 after this chunk
+        }
+        __syncthreads();
+        if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
+        return slow_c;
+    };
+    load_inputs(0);
+    bool slow = stage_gate(0);
 
     for (int t0 = 0; t0 < T && !aborted; t0 += CH) {
         const int n = min(CH, T - t0);
-        const int m_ref = (n - 1) >> 1;
         const size_t tok0 = (size_t)b * T + t0;
+        const bool has_next = t0 + CH < T;
 
-        // ---- P2: the chunk's g and v tiles arrived in GM by cp.async; V^T -> VE, beta ----------
-        cp_async_wait_all();
-        __syncthreads();
+        // ---- P2: V^T -> VE from the VS staging (VE is free: the previous chain is done) ----------
         {
-            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::GM + 16384);
-            const int vc = tid & (VD - 1), jq0 = tid >> 7;  // one value column, token quads jq0 + 2 x
+            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::VS);
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
                 const int j = 4 * (jq0 + 2 * x);
@@ -339,51 +391,6 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                                to_tf32(bf16_bits_to_f32(sVs[(j + 3) * VD + vc])));
             }
         }
-        if (tid < CH) sBeta[tid] = bload;
-        const int gd = tid & (KD - 1), gh = tid >> 7;  // gate channel, token half
-        float gv[32];
-        {
-            const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
-            float acc = 0.f;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int i = 32 * gh + r;
-                const float x = (i < n) ? gate_value_fast(__bfloat162float(sG[i * KD + gd]), bias, rate, gate_mode,
-                                                          lower_bound)
-                                        : 0.f;
-                acc += x;
-                gv[r] = acc;
-            }
-            if (gh == 0) sFnext[gd] = acc;  // scratch: first-half totals
-        }
-        __syncthreads();
-        {
-            const float off = gh ? sFnext[gd] : 0.f;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) sGam[gidx(32 * gh + r, gd)] = gv[r] + off;
-        }
-        __syncthreads();
-        if (tid < KD) {
-            const int d = tid;
-            const float g0 = sGam[gidx(0, d)], gm = sGam[gidx(m_ref, d)], gend = sGam[gidx(n - 1, d)];
-            if (!(fmaxf(g0 - gm, gm - gend) <= SPAN_LIMIT)) atomicOr(sFlag, 1u);
-            sRho[d] = gm;
-            sSig[d] = gend;
-        }
-        __syncthreads();
-        const bool slow = (*reinterpret_cast<volatile uint32_t*>(sFlag)) != 0;
-        if (tid < KD) {
-            const int d = tid;
-            float rho = sRho[d], sig = sSig[d];
-            if (slow) rho = 0.f;  // sig stays Gam_end: Kchk becomes Kend
-            else sig = rho;
-            sRho[d] = rho;
-            sSig[d] = sig;
-            sERho[d] = sFpend[d] * __expf(rho);  // D4 rescale: previous chunk's pending factor and e^rho
-            sESig[d] = __expf(sig);
-            sFnext[d] = __expf(sGam[gidx(CH - 1, d)] - sig);  // pending per-key factor of D4 after this chunk
-        }
-        __syncthreads();
 
         // ---- P3: [Qhat; -Khat] -> X1, Kchk -> AT (B of M1), Kchk^T -> X2 (B of M6);
         //          D4 <- S_c^T diag(e^rho) (applies the previous chunk's pending factor too) ----------
@@ -528,8 +535,6 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         fence_proxy_async();
         cta_sync_tc();
-        if (t0 + CH < T) prefetch_gv(t0 + CH);  // GM (R/T) is no longer needed by this chunk
-
         // ---- state chain: M3, M2, M4, M5, M6 back to back (fast path) --------------------------
         if (tid == 0) {
             gemm_tf32_ts(tmem + L::D3, tmem + L::D4, s_base + L::X1, KD / 4 * 128, idesc_tf32(128, 128), KD / 8, false);
@@ -542,6 +547,15 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                 gemm_tf32_ts(tmem + L::D4, tmem + L::D2, s_base + L::X2, CH / 4 * 128, idesc_tf32(128, 128), CH / 8,
                              true);
             mma_commit(mbar);
+        }
+        // Next chunk's inputs: GM (R/T) and VS are no longer needed by this chunk.  VS must not be
+        // overwritten before this chunk's V^T was built (it was, in P2, before several barriers).
+        if (has_next) load_inputs(t0 + CH);
+        // fast path: the next chunk's gate runs while the chain executes (touches GM and vectors only)
+        bool slow_next = false;
+        if (!slow) {
+            if (tid < KD) sFpend[tid] = sFnext[tid];
+            if (has_next) slow_next = stage_gate(t0 + CH);
         }
         {
             const bool ok = mbar_wait(mbar, phase, WAIT_POLLS);
@@ -574,8 +588,6 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             phase ^= 1u;
         }
 
-        if (t0 + CH < T) load_qkb(t0 + CH);
-
         // ---- outputs: O^T in D3 columns 0-63 (lane = value column) ----------------------------
         {
             TmemRow<32> row;
@@ -588,8 +600,12 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                 if (i < n) op[(size_t)i * v_row] = __float2bfloat16_rn(__uint_as_float(row.r[c]));
             }
         }
-        if (tid < KD) sFpend[tid] = sFnext[tid];
-        if (tid == 0) *sFlag = 0u;
+        if (slow) {
+            cta_sync_tc();
+            if (tid < KD) sFpend[tid] = sFnext[tid];
+            if (has_next) slow_next = stage_gate(t0 + CH);
+        }
+        slow = slow_next;
         cta_sync_tc();
     }
 
