@@ -79,9 +79,11 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
                     float* g_out, kda_stream_t stream);
 
 /*
- * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs
- * for these sizes (always >= 256: the first 256 bytes hold the on-device status
- * word read by kda_read_status).  Returns 0 for sizes kda_chunk_fwd rejects.
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace with which kda_chunk_fwd
+ * runs its fastest schedule for these sizes.  Always >= 256: the first 256 bytes hold
+ * the on-device status word read by kda_read_status.  For K = V = 128 and chunk 64 it
+ * adds the per-chunk records of the two-pass schedule (about 146 KiB per chunk of 64
+ * tokens per (sequence, value head)).  Returns 0 for sizes kda_chunk_fwd rejects.
  */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk);
 
@@ -91,6 +93,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, i
  * recurrence above token by token, computed C tokens at a time with the
  * in-chunk cumulative log-decay, the triangular solve for the in-chunk delta
  * errors and one state update per chunk.
+ * Schedules (bf16 inputs, K = V = 128, chunk 64): with a workspace of at least
+ * kda_chunk_fwd_workspace_size bytes, two passes -- every chunk's local work in
+ * parallel, then the state recurrence over chunks; with a smaller workspace (>= 256
+ * bytes), one pass with one CTA per (sequence, value head).  Both compute the same
+ * quantities to the same tolerance.  Other shapes and float32 inputs use one pass.
  *   q, k     [B, T, H, K]   dtype
  *   v        [B, T, HV, V]  dtype
  *   g        [B, T, HV, K]  dtype   g_raw when gate_mode != NONE, else the log decay (<= 0)
@@ -103,9 +110,10 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, i
  *   o        [B, T, HV, V]  dtype, written; must not alias any input
  *   S_T      [B, HV, K, V]  float32 final state, written; or NULL.  May alias S0
  *            (in-place state update).
- *   workspace, workspace_bytes  >= kda_chunk_fwd_workspace_size(...) bytes of
- *            caller-owned device memory, 256-byte aligned; contents need no
- *            initialisation and are scratch after the call.
+ *   workspace, workspace_bytes  >= 256 bytes of caller-owned device memory,
+ *            256-byte aligned (kda_chunk_fwd_workspace_size(...) bytes select the
+ *            fastest schedule); contents need no initialisation and are scratch
+ *            after the call.
  * Constraints: HV % H == 0; K, V in {16, 32, 64, 128}; T >= 1 (a last partial
  * chunk is handled); every pointer 16-byte aligned.
  * Calls that share one workspace must be ordered on one stream.
@@ -116,6 +124,21 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
                          void* o, float* S_T, void* workspace, size_t workspace_bytes,
                          kda_stream_t stream);
+
+/* Schedules of kda_chunk_fwd. */
+typedef enum {
+    KDA_SCHEDULE_CUDA_CORE = 0,     /* one kernel on the CUDA cores (float32 inputs, other shapes)     */
+    KDA_SCHEDULE_TC_SINGLE_PASS = 1, /* one tensor-core kernel, one CTA per (sequence, value head)      */
+    KDA_SCHEDULE_TC_TWO_PASS = 2     /* two tensor-core kernels: all chunks' local work, then the state */
+} kda_schedule;
+
+/*
+ * kda_chunk_fwd_schedule -- the schedule kda_chunk_fwd runs for these sizes, input dtype and
+ * workspace size (a kda_schedule value), or -1 for arguments it rejects.  No launch, no device
+ * access.
+ */
+int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk, kda_dtype dtype,
+                           size_t workspace_bytes);
 
 /*
  * kda_read_status -- synchronises `stream`, then reads the status word a
@@ -142,8 +165,10 @@ kda_status kda_read_status(const void* workspace, kda_stream_t stream);
  *   - The first call on a device resolves the array's device address on that device
  *     (cudaGetSymbolAddress with the device current); make that first call before any stream
  *     capture.
- *   - Sizes that would need more workspace than KDA_NOALLOC_SCRATCH_BYTES return
- *     KDA_ERR_UNSUPPORTED with a message; nothing is launched.
+ *   - The array is smaller than the two-pass schedule's per-chunk records, so these calls
+ *     run the single-pass schedule (see kda_chunk_fwd).  Sizes that would need more
+ *     workspace than KDA_NOALLOC_SCRATCH_BYTES even so return KDA_ERR_UNSUPPORTED with a
+ *     message; nothing is launched.
  *   - Every call uses the same array and leaves its contents behind; each call clears the part
  *     that must start at zero (the status word).  Calls whose work overlaps on the GPU (for
  *     example on two streams at once) race on the array: order them on one stream.  The status

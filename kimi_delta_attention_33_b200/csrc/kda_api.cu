@@ -53,12 +53,26 @@ kda_status check_common(const void* q, const void* k, const void* v, const void*
     return KDA_OK;
 }
 
-constexpr size_t kStatusBytes = 256;
+constexpr size_t kStatusBytes = kda::kChunkStatusBytes;
+
+bool sizes_ok(int B, int T, int H, int HV, int K, int V, int chunk) {
+    return B >= 1 && T >= 1 && H >= 1 && HV >= 1 && HV % H == 0 && kv_dim_ok(K) && kv_dim_ok(V) &&
+           (chunk == 16 || chunk == 64);
+}
+
+// The tensor-core schedules cover K = V = 128, chunk 64 with bf16 inputs.  With float32 inputs the
+// stated tolerance (1e-4) is tighter than tf32 products allow, so those (and the other shapes) run
+// on the CUDA-core kernel in fp32.
+bool split_shape(int K, int V, int chunk) { return K == 128 && V == 128 && chunk == 64; }
 
 }  // namespace
 
 namespace kda {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+size_t chunk_min_workspace(int B, int T, int H, int HV, int K, int V, int chunk) {
+    return sizes_ok(B, T, H, HV, K, V, chunk) ? kStatusBytes : 0;
+}
 }  // namespace kda
 
 extern "C" {
@@ -84,9 +98,18 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
 }
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk) {
-    if (B < 1 || T < 1 || H < 1 || HV < 1 || HV % H != 0 || !kv_dim_ok(K) || !kv_dim_ok(V)) return 0;
-    if (chunk != 16 && chunk != 64) return 0;
+    if (!sizes_ok(B, T, H, HV, K, V, chunk)) return 0;
+    if (split_shape(K, V, chunk)) return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
     return kStatusBytes;
+}
+
+int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk, kda_dtype dtype,
+                           size_t workspace_bytes) {
+    if (!sizes_ok(B, T, H, HV, K, V, chunk) || (dtype != KDA_F32 && dtype != KDA_BF16) || workspace_bytes < kStatusBytes)
+        return -1;
+    if (dtype != KDA_BF16 || !split_shape(K, V, chunk)) return KDA_SCHEDULE_CUDA_CORE;
+    if (workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV)) return KDA_SCHEDULE_TC_TWO_PASS;
+    return KDA_SCHEDULE_TC_SINGLE_PASS;
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -102,9 +125,9 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, S0, o, S_T, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
-    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk);
-    if (!workspace || workspace_bytes < need)
-        return fail(KDA_ERR_INVALID_ARG, "workspace of at least %zu bytes is required (got %zu)", need, workspace_bytes);
+    if (!workspace || workspace_bytes < kStatusBytes)
+        return fail(KDA_ERR_INVALID_ARG, "workspace of at least %zu bytes is required (got %zu)", kStatusBytes,
+                    workspace_bytes);
     if (o == q || o == k || o == v || o == g || o == beta) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
     if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
     kda::ChunkArgs a{q, k, v, g, beta, A_log, dt_bias, S0, B, T, H, HV, K, V, chunk, (int)gate_mode, lower_bound,
@@ -113,7 +136,11 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                      (cudaStream_t)stream};
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "status word reset");
-    if (kda::chunk_tc_supported(a)) {
+    const int schedule = kda_chunk_fwd_schedule(B, T, H, HV, K, V, chunk, dtype, workspace_bytes);
+    if (schedule == KDA_SCHEDULE_TC_TWO_PASS) {
+        e = kda::launch_chunk_split(a);
+        if (e != cudaSuccess) return cuda_fail(e, "two-pass tensor-core chunk kernel launch");
+    } else if (schedule == KDA_SCHEDULE_TC_SINGLE_PASS) {
         e = kda::launch_chunk_tc(a);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel launch");
     } else {

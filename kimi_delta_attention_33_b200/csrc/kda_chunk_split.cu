@@ -1,0 +1,707 @@
+// kda_chunk_split.cu -- two-pass chunked prefill on the tensor cores (bf16 inputs, K = V = 128,
+// chunk 64) for shapes with few (sequence, head) pairs, where one CTA per pair leaves most SMs idle.
+//
+// DeltaNet-family digest, sections "Chunkwise KDA" and "Chunkwise Triton pipeline": everything of a
+// chunk that does not involve the state entering it can be computed for all chunks at once; only
+// the state update is sequential.  Notation as in the single-pass kernel (kda_chunk_tc.cu):
+//   Gam_i  in-chunk cumulative log decay, rho / sig per-channel reference points,
+//   Qhat_i = s q_i e^{Gam_i - rho},  Khat_i = k_i e^{Gam_i - rho},  Kchk_j = k_j e^{sig - Gam_j},
+//   A = masked Qhat Kchk^T,  R = masked beta Khat Kchk^T,  T = (I + R)^{-1},  Tb = T diag(beta).
+// With S~ = diag(e^rho) S_c (S_c the state entering the chunk) the chunk's results are
+//   E      = U - W S~        where U = Tb V and W = Tb Khat      (resolved delta errors)
+//   O      = Qhat S~ + A E                                        (chunk outputs)
+//   S_c+1  = diag(f) (diag(e^sig) S_c + Kchk^T E),   f = e^{Gam_end - sig}.
+//
+// Pass 1 (chunk_prep_kernel, persistent, one chunk per CTA iteration, all chunks in parallel):
+// gate, Gam, the operands, M1 = [-Khat; Qhat] Kchk^T -> R and A, the triangular inverse, and
+// M7 = [A; Tb] [Khat^T; V^T]^T -> W and U, written to a per-chunk record in the workspace:
+//   WQ  [W; Qhat]  128 x 128 tf32 in the K-major tiling of kda_tc_ptx.cuh (the A operand of M8)
+//   KA  [Kchk^T; A] 192 x 64 tf32, same tiling (A operands of M9 and M10)
+//   UT  U^T, fp32 rows of 64 (one per value column)
+//   VEC e^rho, e^sig, f (fp32, 128 each)
+// Pass 2 (chunk_state_kernel, one CTA per (pair, block of VB value columns), chunks in order):
+// the state slice S_c[:, block] lives in registers (thread d owns key row d, exact fp32);
+// per chunk, with tf32(S~)^T staged in shared memory as a B operand:
+//   M8   D1 = [W; Qhat] S~                -> W S~ (rows 0-63), Qhat S~ (rows 64-127)
+//   E    = U - W S~  on the CUDA cores, staged as a tf32 B operand
+//   M9   D1[64:] += A E                   -> O
+//   M10  D2 = Kchk^T E                    -> S_c+1 = f (e^sig S_c + D2), in registers
+// Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
+// where shared memory allows.
+#include "kda_chunk64.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+using bf16 = __nv_bfloat16;
+
+namespace {
+using namespace c64;
+
+// Per-chunk record in the workspace (bytes).
+struct Rec {
+    static constexpr uint32_t WQ = 0;        // [128][128] tf32 tiles
+    static constexpr uint32_t KA = 65536;    // [192][64] tf32 tiles
+    static constexpr uint32_t KA_BYTES = 49152;
+    static constexpr uint32_t UT = 114688;   // [128][64] fp32 rows
+    static constexpr uint32_t VEC = 147456;  // 3 x [128] fp32
+    static constexpr uint32_t BYTES = 149504;
+    static_assert(VEC + 3 * 512 <= BYTES && BYTES % 256 == 0, "record layout");
+};
+
+struct PrepLayout {
+    static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1), then [W; Qhat] (record WQ)
+    static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling scratch
+    static constexpr uint32_t XS = CK + 64 * RP * 4;
+    static constexpr uint32_t KA = 98304;    // [256][64]: Kchk^T rows 0-127, A rows 128-191, Tb rows 192-255
+    static constexpr uint32_t GM = 163840;   // g staging (bf16) -> Gam (fp32) -> Khat^T [128][64] (B rows 0-127 of M7)
+    static constexpr uint32_t VT = 196608;   // v staging (bf16, upper half) -> V^T [128][64] (B rows 128-255 of M7)
+    static constexpr uint32_t VEC = 229376;
+    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024;
+    static constexpr uint32_t MBAR = VEC + 1280, TBASE = MBAR + 8, FLAG = TBASE + 4;
+    static constexpr uint32_t BYTES = FLAG + 4;
+    static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
+    static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
+    static_assert(GM + 32768 == VT, "M7's B operand spans GM and VT");
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+template <int VB>
+struct StateLayout {
+    static constexpr int NKA = VB <= 32 ? 2 : 1;              // KA / U buffers
+    static constexpr uint32_t WQ = 0;                          // [128][128]
+    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], then U^T [VB][64]
+    static constexpr uint32_t KA_STRIDE = Rec::KA_BYTES + VB * 256;
+    static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S~^T [VB][128]   (B of M8)
+    static constexpr uint32_t EOP = SOP + VB * 128 * 4;        // tf32 E^T  [VB][64]    (B of M9, M10)
+    static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1]
+    static constexpr uint32_t TBASE = MBAR + 32;
+    static constexpr uint32_t BYTES = TBASE + 16;
+    static constexpr uint32_t TMEM_COLS = 2 * VB < 32 ? 32 : 2 * VB;
+    static constexpr int D1 = 0, D2 = VB;
+    static __device__ __forceinline__ uint32_t ka(int buf) { return KA0 + buf * KA_STRIDE; }
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+constexpr int STATE_THREADS = 128;
+
+struct Task {
+    int pair, c, b, hv, h, nn;
+    size_t tk0;  // token index (b * T + first token of the chunk)
+};
+
+__device__ __forceinline__ Task make_task(long long task, int T, int H, int HV, int NC) {
+    Task t;
+    t.pair = (int)(task / NC);
+    t.c = (int)(task - (long long)t.pair * NC);
+    t.b = t.pair / HV;
+    t.hv = t.pair - t.b * HV;
+    t.h = t.hv / (HV / H);
+    t.nn = min(CH, T - t.c * CH);
+    t.tk0 = (size_t)t.b * T + (size_t)t.c * CH;
+    return t;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// Pass 1: chunk-local work for every chunk.
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(TC_THREADS, 1)
+chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                  const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
+                  const float* __restrict__ dt_bias, int T, int H, int HV, int NC, long long ntasks, int gate_mode,
+                  float lower_bound, float scale, unsigned char* __restrict__ rec_base,
+                  unsigned int* __restrict__ status) {
+    using L = PrepLayout;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    float* sRho = reinterpret_cast<float*>(smem + L::RHO);
+    float* sSig = reinterpret_cast<float*>(smem + L::SIG);
+    float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
+    float* sGam = reinterpret_cast<float*>(smem + L::GM);
+    float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
+    float* sX = reinterpret_cast<float*>(smem + L::XS);
+    const bf16* sG = reinterpret_cast<const bf16*>(smem + L::GM);
+    uint32_t* sFlag = reinterpret_cast<uint32_t*>(smem + L::FLAG);
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t mbar = s_base + L::MBAR;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const size_t qk_row = (size_t)H * KD, v_row = (size_t)HV * VD, g_row = (size_t)HV * KD;
+
+    if (tid == 0) mbar_init(mbar, 1);
+    if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
+    if (tid == 0) *sFlag = 0u;
+    cta_sync_tc();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
+    uint32_t phase = 0;
+    bool aborted = false;
+
+    // Inputs of one chunk: g and v tiles into shared staging by cp.async (rows past T zero-filled),
+    // q, k and beta into registers.
+    uint4 qr[4], kr[4];
+    float bload;
+    auto load_inputs = [&](const Task& tk) {
+        const uint32_t gs = s_base + L::GM, vs = s_base + L::VT + 16384;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int u = tid + TC_THREADS * it;
+            const int i = u >> 4, c = u & 15;
+            const bool ok = i < tk.nn;
+            cp_async16(gs + i * 256 + c * 16, ok ? g + (tk.tk0 + i) * g_row + (size_t)tk.hv * KD + 8 * c : g,
+                       ok ? 16u : 0u);
+            cp_async16(vs + i * 256 + c * 16, ok ? v + (tk.tk0 + i) * v_row + (size_t)tk.hv * VD + 8 * c : v,
+                       ok ? 16u : 0u);
+        }
+        cp_async_commit();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int u = tid + TC_THREADS * it;
+            const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
+            qr[it] = make_uint4(0u, 0u, 0u, 0u);
+            kr[it] = qr[it];
+            if (i < tk.nn) {
+                qr[it] = __ldg(reinterpret_cast<const uint4*>(q + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD + 8 * d8));
+                kr[it] = __ldg(reinterpret_cast<const uint4*>(k + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD + 8 * d8));
+            }
+        }
+        bload = (tid < tk.nn) ? to_f32(beta[(tk.tk0 + tid) * HV + tk.hv]) : 0.f;
+    };
+
+    long long task = blockIdx.x;
+    if (task < ntasks) load_inputs(make_task(task, T, H, HV, NC));
+
+    for (; task < ntasks && !aborted; task += gridDim.x) {
+        const Task tk = make_task(task, T, H, HV, NC);
+        unsigned char* rec = rec_base + (size_t)task * Rec::BYTES;
+        const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[tk.hv]) : 0.0f;
+
+        // ---- gate and inclusive in-chunk cumulative log decay (two threads per key channel) ----
+        bool slow;
+        {
+            const int nn = tk.nn, mr = (nn - 1) >> 1;
+            cp_async_wait_all();
+            __syncthreads();
+            if (tid < CH) sBeta[tid] = bload;
+            const int gd = tid & (KD - 1), gh = tid >> 7;
+            float gv[32];
+            const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[tk.hv * KD + gd] : 0.0f;
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int i = 32 * gh + r;
+                const float x = (i < nn) ? gate_value_fast(__bfloat162float(sG[i * KD + gd]), bias, rate, gate_mode,
+                                                           lower_bound)
+                                         : 0.f;
+                acc += x;
+                gv[r] = acc;
+            }
+            if (gh == 0) sSig[gd] = acc;  // scratch: first-half totals
+            __syncthreads();              // the g staging has been read: GM becomes Gam
+            const float off = gh ? sSig[gd] : 0.f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) sGam[gidx(32 * gh + r, gd)] = gv[r] + off;
+            __syncthreads();
+            if (tid < KD) {
+                const int d = tid;
+                const float g0 = sGam[gidx(0, d)], gm = sGam[gidx(mr, d)], gend = sGam[gidx(nn - 1, d)];
+                if (!(fmaxf(g0 - gm, gm - gend) <= SPAN_LIMIT)) atomicOr(sFlag, 1u);
+                sRho[d] = gm;
+                sSig[d] = gend;
+            }
+            __syncthreads();
+            slow = (*reinterpret_cast<volatile uint32_t*>(sFlag)) != 0;
+            if (tid < KD) {
+                const int d = tid;
+                float rho = sRho[d], sig = sSig[d];
+                if (slow) rho = 0.f;  // sig stays Gam_end: Kchk becomes Kend
+                else sig = rho;
+                sRho[d] = rho;
+                sSig[d] = sig;
+                float* rv = reinterpret_cast<float*>(rec + Rec::VEC);
+                rv[d] = __expf(rho);
+                rv[KD + d] = __expf(sig);
+                rv[2 * KD + d] = __expf(sGam[gidx(CH - 1, d)] - sig);
+            }
+            __syncthreads();
+            if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
+        }
+
+        // ---- V^T into VT from the staged v tile (upper half of VT) ------------------------------
+        {
+            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::VT + 16384);
+            const int vc = tid & (VD - 1), jq0 = tid >> 7;
+            uint32_t vv[16];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const int j = 4 * (jq0 + 2 * x);
+                vv[2 * x] = (uint32_t)sVs[(j + 0) * VD + vc] | ((uint32_t)sVs[(j + 1) * VD + vc] << 16);
+                vv[2 * x + 1] = (uint32_t)sVs[(j + 2) * VD + vc] | ((uint32_t)sVs[(j + 3) * VD + vc] << 16);
+            }
+            // the previous chunk's record stores must be done reading X1 and KA before P3 rewrites them
+            if (tid == 0) bulk_wait_read();
+            __syncthreads();
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const int j = 4 * (jq0 + 2 * x);
+                *reinterpret_cast<uint4*>(smem + L::VT + cm_off(vc, j, CH)) =
+                    make_uint4(to_tf32(__uint_as_float(vv[2 * x] << 16)), to_tf32(__uint_as_float(vv[2 * x] & 0xFFFF0000u)),
+                               to_tf32(__uint_as_float(vv[2 * x + 1] << 16)),
+                               to_tf32(__uint_as_float(vv[2 * x + 1] & 0xFFFF0000u)));
+            }
+        }
+
+        // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK, Kchk^T -> KA rows 0-127 -----------------------
+        uint32_t kh[4][8];  // tf32 bits of -Khat, kept for Khat^T once Gam is no longer needed
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int u = tid + TC_THREADS * it;
+            const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
+            float qf[8], kf[8], gf[8], rf[8], sf[8];
+            bf16x8_to_f32(qr[it], qf);
+            bf16x8_to_f32(kr[it], kf);
+            *reinterpret_cast<float4*>(gf) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8));
+            *reinterpret_cast<float4*>(gf + 4) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8 + 4));
+            *reinterpret_cast<float4*>(rf) = *reinterpret_cast<const float4*>(sRho + 8 * d8);
+            *reinterpret_cast<float4*>(rf + 4) = *reinterpret_cast<const float4*>(sRho + 8 * d8 + 4);
+            *reinterpret_cast<float4*>(sf) = *reinterpret_cast<const float4*>(sSig + 8 * d8);
+            *reinterpret_cast<float4*>(sf + 4) = *reinterpret_cast<const float4*>(sSig + 8 * d8 + 4);
+            uint32_t wq_[8], wc_[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const float e1 = __expf(gf[t] - rf[t]), e2 = __expf(sf[t] - gf[t]);
+                wq_[t] = to_tf32(scale * qf[t] * e1);
+                kh[it][t] = to_tf32(-kf[t] * e1);
+                wc_[t] = to_tf32(kf[t] * e2);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int d = 8 * d8 + 4 * hh;
+                *reinterpret_cast<uint4*>(smem + L::X1 + cm_off(i, d, KD)) =
+                    make_uint4(kh[it][4 * hh], kh[it][4 * hh + 1], kh[it][4 * hh + 2], kh[it][4 * hh + 3]);
+                *reinterpret_cast<uint4*>(smem + L::X1 + cm_off(64 + i, d, KD)) =
+                    make_uint4(wq_[4 * hh], wq_[4 * hh + 1], wq_[4 * hh + 2], wq_[4 * hh + 3]);
+                *reinterpret_cast<uint4*>(smem + L::CK + cm_off(i, d, KD)) =
+                    make_uint4(wc_[4 * hh], wc_[4 * hh + 1], wc_[4 * hh + 2], wc_[4 * hh + 3]);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + t, i, CH)) = wc_[t];
+        }
+        fence_proxy_async();
+        cta_sync_tc();
+
+        // Khat^T into GM (B rows 0-127 of M7) once Gam is no longer read
+        auto write_khat_t = [&]() {
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int u = tid + TC_THREADS * it;
+                const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    *reinterpret_cast<uint32_t*>(smem + L::GM + cm_off(8 * d8 + t, i, CH)) = kh[it][t] ^ 0x80000000u;
+            }
+        };
+
+        // ---- A -> KA rows 128-191, R -> CK region (pitch RP) -------------------------------------
+        if (!slow) {
+            if (tid == 0) {
+                gemm_tf32(tmem, s_base + L::X1, KD / 4 * 128, s_base + L::CK, KD / 4 * 128, idesc_tf32(128, 64), KD / 8,
+                          false);
+                mma_commit(mbar);
+            }
+            write_khat_t();
+            const bool ok = mbar_wait(mbar, phase, WAIT_POLLS);
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) { aborted = true; break; }
+            phase ^= 1u;
+            uint32_t raw[32];
+            tmem_ld32(taddr(tmem, 32 * wq, 32 * wh), raw);
+            tmem_wait_ld();
+            if (wq < 2) {  // rows 0-63 of D1 hold -Khat Kchk^T
+                const int i = 32 * wq + lane;
+                const float bi = -sBeta[i];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * wh + jj;
+                    sRT[i * RP + j] = (j < i) ? bi * __uint_as_float(raw[jj]) : 0.f;
+                }
+            } else {  // rows 64-127 hold A (unmasked)
+                const int i = 32 * (wq - 2) + lane;
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 4) {
+                    const int j = 32 * wh + jj;
+                    uint4 w4;
+                    w4.x = to_tf32(j + 0 <= i ? __uint_as_float(raw[jj + 0]) : 0.f);
+                    w4.y = to_tf32(j + 1 <= i ? __uint_as_float(raw[jj + 1]) : 0.f);
+                    w4.z = to_tf32(j + 2 <= i ? __uint_as_float(raw[jj + 2]) : 0.f);
+                    w4.w = to_tf32(j + 3 <= i ? __uint_as_float(raw[jj + 3]) : 0.f);
+                    *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, j, CH)) = w4;
+                }
+            }
+        } else {
+            // exact decay factors: 4096 (i, j) cells, 16 per thread; Gam is still in GM
+            float av[16], rr[16];
+#pragma unroll 1
+            for (int x = 0; x < 16; ++x) {
+                const int p = tid + TC_THREADS * x;
+                const int i = p >> 6, j = p & 63;
+                float a = 0.f, r = 0.f;
+                if (j <= i && i < tk.nn) {
+                    const bf16* qi = q + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD;
+                    const bf16* ki = k + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD;
+                    const bf16* kj = k + (tk.tk0 + j) * qk_row + (size_t)tk.h * KD;
+                    for (int d = 0; d < KD; ++d) {
+                        const float e = __expf(sGam[gidx(i, d)] - sGam[gidx(j, d)]);
+                        const float kd = to_f32(kj[d]) * e;
+                        a += to_f32(qi[d]) * kd;
+                        r += to_f32(ki[d]) * kd;
+                    }
+                }
+                av[x] = (j <= i) ? scale * a : 0.f;
+                rr[x] = (j < i) ? sBeta[i] * r : 0.f;
+            }
+            __syncthreads();  // Gam fully read: GM becomes Khat^T
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const int p = tid + TC_THREADS * x;
+                const int i = p >> 6, j = p & 63;
+                *reinterpret_cast<uint32_t*>(smem + L::KA + 32768 + cm_off(i, j, CH)) = to_tf32(av[x]);
+                sRT[i * RP + j] = rr[x];
+            }
+            write_khat_t();
+        }
+        __syncthreads();
+
+        // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 192-255 ---------------------
+        tri_inverse_step<1>(sRT, sX, tid);
+        tri_inverse_step<2>(sRT, sX, tid);
+        tri_inverse_step<4>(sRT, sX, tid);
+        tri_inverse_step<8>(sRT, sX, tid);
+        tri_inverse_step16(sRT, sX, tid);
+        tri_inverse_step32(sRT, sX, tid);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int u = tid + TC_THREADS * x;
+            const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
+            uint32_t w[4];
+            const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
+            const float tr[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int j = 4 * j4 + t;
+                const float tv = (j < i) ? tr[t] : (j == i ? 1.f : 0.f);
+                w[t] = to_tf32(tv * sBeta[j]);
+            }
+            *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, 4 * j4, CH)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        cta_sync_tc();
+
+        // ---- M7: D[128][256] = [A; Tb] [Khat^T; V^T]^T; rows 64-127 hold W | U --------------------
+        if (tid == 0) {
+            gemm_tf32(tmem, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::GM, CH / 4 * 128, idesc_tf32(128, 256),
+                      CH / 8, false);
+            mma_commit(mbar);
+        }
+        {
+            const bool ok = mbar_wait(mbar, phase, WAIT_POLLS);
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) { aborted = true; break; }
+            phase ^= 1u;
+        }
+        // GM and VT are free: stage the next chunk of this CTA while the record is written out
+        if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
+        if (wq >= 2) {
+            const int i = 32 * (wq - 2) + lane;
+            if (wh == 0) {  // W -> X1 rows 0-63 (tf32)
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr(tmem, 32 * wq, 32 * blk), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        *reinterpret_cast<uint4*>(smem + L::X1 + cm_off(i, 32 * blk + 4 * c4, KD)) =
+                            make_uint4(to_tf32(__uint_as_float(r[4 * c4])), to_tf32(__uint_as_float(r[4 * c4 + 1])),
+                                       to_tf32(__uint_as_float(r[4 * c4 + 2])), to_tf32(__uint_as_float(r[4 * c4 + 3])));
+                }
+            } else {  // U -> record U^T (fp32, row = value column)
+                float* ut = reinterpret_cast<float*>(rec + Rec::UT);
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr(tmem, 32 * wq, 128 + 32 * blk), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) ut[(32 * blk + cc) * CH + i] = __uint_as_float(r[cc]);
+                }
+            }
+        }
+        fence_proxy_async();
+        cta_sync_tc();
+        if (tid == 0) {
+            bulk_store(rec + Rec::WQ, s_base + L::X1, 65536);
+            bulk_store(rec + Rec::KA, s_base + L::KA, Rec::KA_BYTES);
+            bulk_commit();
+        }
+    }
+
+    if (aborted) {
+        if (tid == 0) atomicOr(status, STATUS_TIMEOUT);
+        mbar_wait(mbar, phase, WAIT_POLLS);  // one more bounded chance for an MMA in flight to drain
+    }
+    cp_async_wait_all();
+    if (tid == 0) bulk_wait_all();
+    cta_sync_tc();
+    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Pass 2: the state recurrence over chunks for one (pair, value block).
+// ---------------------------------------------------------------------------------------------
+template <int N>
+__device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N % 32 == 0, "row width");
+    if constexpr (N == 16) {
+        tmem_ld16(a, r);
+    } else {
+#pragma unroll
+        for (int b = 0; b < N / 32; ++b) tmem_ld32(a + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * b));
+    }
+}
+
+template <int VB>
+__global__ void __launch_bounds__(STATE_THREADS, 1)
+chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __restrict__ S0, int T, int HV, int NC,
+                   bf16* __restrict__ o, float* __restrict__ S_T, unsigned int* __restrict__ status) {
+    using L = StateLayout<VB>;
+    constexpr int NVB = VD / VB;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t bar_wq = s_base + L::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16;
+    const int pair = blockIdx.x / NVB, vb0 = (blockIdx.x - pair * NVB) * VB;
+    const int b = pair / HV, hv = pair - b * HV;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const size_t v_row = (size_t)HV * VD;
+    const unsigned char* rec0 = rec_base + (size_t)pair * NC * Rec::BYTES;
+    auto rec = [&](int c) { return rec0 + (size_t)c * Rec::BYTES; };
+
+    if (tid == 0) {
+        mbar_init(bar_wq, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_ka0, 1);
+        mbar_init(bar_ka0 + 8, 1);
+    }
+    if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
+    cta_sync_tc();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
+
+    // loads in flight, for the bounded drain on abort: bit 0 wq, bit 1 + buf ka
+    uint32_t pending = 0;
+    auto load_wq = [&](int c) {
+        mbar_expect_tx(bar_wq, 65536);
+        bulk_load(s_base + L::WQ, rec(c) + Rec::WQ, 65536, bar_wq);
+        pending |= 1u;
+    };
+    auto load_ka = [&](int c, int buf) {
+        const uint32_t bar = bar_ka0 + 8 * buf;
+        mbar_expect_tx(bar, Rec::KA_BYTES + VB * 256);
+        bulk_load(s_base + L::ka(buf), rec(c) + Rec::KA, Rec::KA_BYTES, bar);
+        bulk_load(s_base + L::ka(buf) + Rec::KA_BYTES, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
+        pending |= 2u << buf;
+    };
+    if (tid == 0) {
+        load_wq(0);
+        load_ka(0, 0);
+        if (L::NKA == 2 && NC > 1) load_ka(1, 1);
+    }
+
+    // this thread's key row of the state slice, exact fp32
+    const int d = tid;
+    float s[VB];
+#pragma unroll
+    for (int j = 0; j < VB; j += 4) {
+        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * KD + d) * VD + vb0 + j)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[j] = x.x;
+        s[j + 1] = x.y;
+        s[j + 2] = x.z;
+        s[j + 3] = x.w;
+    }
+    auto write_sop = [&](float er) {
+#pragma unroll
+        for (int j = 0; j < VB; ++j) *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(j, d, KD)) = to_tf32(er * s[j]);
+    };
+    const float* vec0 = reinterpret_cast<const float*>(rec(0) + Rec::VEC);
+    float es = vec0[KD + d], ef = vec0[2 * KD + d];
+    write_sop(vec0[d]);
+    fence_proxy_async();
+    cta_sync_tc();
+
+    uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0;
+    bool aborted = false;
+    for (int c = 0; c < NC; ++c) {
+        const int buf = (L::NKA == 2) ? (c & 1) : 0;
+        const int n = min(CH, T - c * CH);
+        float er_n = 0.f, es_n = 0.f, ef_n = 0.f;  // the next chunk's vectors, consumed at the end
+        if (c + 1 < NC) {
+            const float* vn = reinterpret_cast<const float*>(rec(c + 1) + Rec::VEC);
+            er_n = __ldg(vn + d);
+            es_n = __ldg(vn + KD + d);
+            ef_n = __ldg(vn + 2 * KD + d);
+        }
+        // ---- M8: D1 = [W; Qhat] S~ ------------------------------------------------------------
+        bool ok = true;
+        if (tid == 0) {
+            ok = mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
+            if (ok) {
+                pending &= ~1u;
+                gemm_tf32(tmem + L::D1, s_base + L::WQ, KD / 4 * 128, s_base + L::SOP, KD / 4 * 128,
+                          idesc_tf32(128, VB), KD / 8, false);
+                mma_commit(bar_mma);
+            }
+        }
+        ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS) && ok;
+        ok = mbar_wait(bar_ka0 + 8 * buf, (ph_ka >> buf) & 1u, WAIT_POLLS) && ok;
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) { aborted = true; break; }
+        // phases advance only on success, so that on abort they name the operations still pending
+        ph_wq ^= 1u;
+        ph_mma ^= 1u;
+        ph_ka ^= 1u << buf;
+        if (tid == 0) {
+            pending &= ~(2u << buf);
+            if (c + 1 < NC) load_wq(c + 1);  // M8 has read WQ
+        }
+        // ---- E = U - W S~ (rows 0-63: warps 0, 1) -> E^T tf32 operand --------------------------
+        const uint32_t ka = s_base + L::ka(buf);
+        if (warp < 2) {
+            const int j = tid;
+            const float* sU = reinterpret_cast<const float*>(smem + L::ka(buf) + Rec::KA_BYTES);
+            uint32_t r[VB];
+            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D1), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int vv = 0; vv < VB; ++vv)
+                *reinterpret_cast<uint32_t*>(smem + L::EOP + cm_off(vv, j, CH)) =
+                    to_tf32(sU[vv * CH + j] - __uint_as_float(r[vv]));
+        }
+        fence_proxy_async();
+        cta_sync_tc();
+        // ---- M9: D1[64:] += A E ;  M10: D2 = Kchk^T E -------------------------------------------
+        if (tid == 0) {
+            gemm_tf32(tmem + L::D1, ka + 16384, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB),
+                      CH / 8, true);
+            gemm_tf32(tmem + L::D2, ka, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
+                      false);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) { aborted = true; break; }
+        ph_mma ^= 1u;
+        if (L::NKA == 1 && tid == 0 && c + 1 < NC) load_ka(c + 1, 0);
+        // ---- outputs (rows 64-127 of D1: warps 2, 3) ---------------------------------------------
+        if (warp >= 2) {
+            const int i = tid - 64;
+            uint32_t r[VB];
+            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D1), r);
+            tmem_wait_ld();
+            if (i < n) {
+                bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0;
+#pragma unroll
+                for (int j = 0; j < VB; j += 8) {
+                    uint4 w;
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+                    __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                    __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                    w.x = *reinterpret_cast<uint32_t*>(&p0);
+                    w.y = *reinterpret_cast<uint32_t*>(&p1);
+                    w.z = *reinterpret_cast<uint32_t*>(&p2);
+                    w.w = *reinterpret_cast<uint32_t*>(&p3);
+                    *reinterpret_cast<uint4*>(op + j) = w;
+                }
+            }
+        }
+        // ---- state: S = f (e^sig S + D2); S~ of the next chunk ----------------------------------
+        {
+            uint32_t r[VB];
+            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D2), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < VB; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
+        }
+        if (c + 1 < NC) {
+            write_sop(er_n);
+            es = es_n;
+            ef = ef_n;
+        }
+        fence_proxy_async();
+        cta_sync_tc();
+        if (L::NKA == 2 && tid == 0 && c + 2 < NC) load_ka(c + 2, buf);
+    }
+
+    if (aborted) {
+        if (tid == 0) {
+            atomicOr(status, STATUS_TIMEOUT);
+            // bounded drain of copies and MMAs still in flight before shared memory and TMEM go away
+            if (pending & 1u) mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
+            for (int bb = 0; bb < L::NKA; ++bb)
+                if (pending & (2u << bb)) mbar_wait(bar_ka0 + 8 * bb, (ph_ka >> bb) & 1u, WAIT_POLLS);
+            mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
+        }
+    } else if (S_T) {
+#pragma unroll
+        for (int j = 0; j < VB; j += 4)
+            *reinterpret_cast<float4*>(S_T + ((size_t)pair * KD + d) * VD + vb0 + j) =
+                make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+    }
+    cta_sync_tc();
+    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+size_t chunk_split_workspace(int B, int T, int HV) {
+    const size_t NC = ((size_t)T + CH - 1) / CH;
+    return (size_t)B * HV * NC * Rec::BYTES;
+}
+
+namespace {
+template <int VB>
+cudaError_t launch_state(const ChunkArgs& a, int NC) {
+    using L = StateLayout<VB>;
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::BYTES);
+    if (e != cudaSuccess) return e;
+    chunk_state_kernel<VB><<<a.B * a.HV * (VD / VB), STATE_THREADS, L::BYTES, a.stream>>>(
+        static_cast<const unsigned char*>(a.scratch), a.S0, a.T, a.HV, NC, static_cast<bf16*>(a.o), a.S_T, a.status);
+    return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_split(const ChunkArgs& a) {
+    const int NC = (a.T + CH - 1) / CH;
+    const long long ntasks = (long long)a.B * a.HV * NC;
+    int dev = 0, nsm = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepLayout::BYTES);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)(ntasks < nsm ? ntasks : nsm);
+    chunk_prep_kernel<<<grid, TC_THREADS, PrepLayout::BYTES, a.stream>>>(
+        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
+        static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
+        ntasks, a.gate_mode, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // value-block width: enough (pair, block) CTAs to cover the SMs, blocks as wide as that allows
+    const long long pairs = (long long)a.B * a.HV;
+    if (pairs * 8 <= nsm) return launch_state<16>(a, NC);
+    if (pairs * 4 <= nsm) return launch_state<32>(a, NC);
+    return launch_state<64>(a, NC);
+}
+
+}  // namespace kda

@@ -56,7 +56,15 @@ void set_last_error(const char* msg);
 cudaError_t launch_decode_step(const DecodeArgs& a);
 cudaError_t launch_gate(const GateArgs& a);
 cudaError_t launch_chunk_simt(const ChunkArgs& a);
-bool chunk_tc_supported(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a);
+// Two-pass tensor-core prefill (same shapes as the single-pass one): per-chunk records need
+// chunk_split_workspace(B, T, HV) bytes of scratch beyond the status block.
+size_t chunk_split_workspace(int B, int T, int HV);
+cudaError_t launch_chunk_split(const ChunkArgs& a);
+
+// Bytes of status block at the start of every chunk-prefill workspace.
+constexpr size_t kChunkStatusBytes = 256;
+// Smallest workspace kda_chunk_fwd accepts for these sizes (0 if it rejects the sizes).
+size_t chunk_min_workspace(int B, int T, int H, int HV, int K, int V, int chunk);
 
 }  // namespace kda

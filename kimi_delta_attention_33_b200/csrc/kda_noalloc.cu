@@ -6,7 +6,8 @@
 // path is forbidden.  Such a caller cannot provide the workspace kda_chunk_fwd asks for.  This
 // entry point supplies that workspace itself, from a fixed array in device memory that is part
 // of this library (every GPU that loads the library holds it until the process exits), and then
-// runs exactly the same prefill as kda_chunk_fwd.
+// runs kda_chunk_fwd with it.  The array is far smaller than the per-chunk records of the two-pass
+// schedule, so these calls always take the single-pass schedule: same results, one kernel.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -35,7 +36,9 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const 
                                             const float* S0, int B, int T, int H, int HV, int K, int V, int chunk,
                                             kda_gate_mode gate_mode, float lower_bound, float scale,
                                             kda_dtype dtype, void* o, float* S_T, kda_stream_t stream) {
-    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk);
+    // The smallest workspace kda_chunk_fwd accepts: with it, kda_chunk_fwd runs its single-pass
+    // schedule, which needs no scratch beyond the status word.
+    const size_t need = kda::chunk_min_workspace(B, T, H, HV, K, V, chunk);
     char msg[192];
     if (need > kScratchBytes) {
         // kda_chunk_fwd's own validation reports the sizes it rejects outright (need == 0).

@@ -12,6 +12,7 @@ Functions mirror the C entry points:
 * ``chunk_fwd(q, k, v, g, beta, ...)``                 -> (o, S_T)
 * ``recurrent_step(q, k, v, g, beta, S, ...)``         -> o  (S updated in place)
 * ``read_status(workspace)``                           -> synchronise and check the device status word
+* ``schedule(B, T, H, HV, K, V, chunk, dtype, ws)``     -> which kernels ``chunk_fwd`` runs
 """
 from __future__ import annotations
 
@@ -32,7 +33,11 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Every symbol include/kda.h declares, in declaration order.
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
-           "kda_read_status", "kda_chunk_fwd_noalloc", "kda_recurrent_step")
+           "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc", "kda_recurrent_step")
+SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS = 0, 1, 2
+SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass"}
+# kernels one kda_chunk_fwd call launches, per schedule
+SCHEDULE_LAUNCHES = {0: 1, 1: 1, 2: 2}
 
 
 class KdaError(RuntimeError):
@@ -58,6 +63,8 @@ lib.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
 lib.kda_chunk_fwd.restype = _i
 lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, _vp, _fp, _vp,
                                                                                   _sz, _vp]
+lib.kda_chunk_fwd_schedule.restype = _i
+lib.kda_chunk_fwd_schedule.argtypes = [_i] * 7 + [_i, _sz]
 lib.kda_read_status.restype = _i
 lib.kda_read_status.argtypes = [_vp, _vp]
 lib.kda_chunk_fwd_noalloc.restype = _i
@@ -203,9 +210,21 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
     return o
 
 
+def schedule(B, T, H, HV, K, V, chunk, dtype: torch.dtype = torch.bfloat16, workspace_bytes: int | None = None) -> int:
+    """The schedule kda_chunk_fwd runs for these sizes (SCHEDULE_* value); ``workspace_bytes`` defaults
+    to ``workspace_size(...)``, the size ``chunk_fwd`` allocates when given no workspace."""
+    if workspace_bytes is None:
+        workspace_bytes = max(workspace_size(B, T, H, HV, K, V, chunk), 256)
+    code = F32 if dtype == torch.float32 else BF16
+    s = int(lib.kda_chunk_fwd_schedule(B, T, H, HV, K, V, chunk, code, workspace_bytes))
+    if s < 0:
+        raise KdaError(ERR_INVALID_ARG, "kda_chunk_fwd rejects these sizes")
+    return s
+
+
 def uses_tensor_cores(K: int, V: int, chunk: int, dtype: torch.dtype = torch.bfloat16) -> bool:
-    """Whether kda_chunk_fwd runs these sizes on the tensor-core kernel (else the CUDA-core kernel)."""
-    return dtype == torch.bfloat16 and K == 128 and chunk == 64 and V == 128
+    """Whether kda_chunk_fwd runs these sizes on a tensor-core schedule (else the CUDA-core kernel)."""
+    return schedule(1, 1, 1, 1, K, V, chunk, dtype, 256) != SCHEDULE_CUDA_CORE
 
 
 def default_scale(K: int) -> float:

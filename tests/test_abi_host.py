@@ -110,3 +110,28 @@ def test_workspace_size():
 
 def test_read_status_rejects_null():
     assert kda.lib.kda_read_status(None, None) == kda.ERR_INVALID_ARG
+
+
+def test_workspace_size_two_pass_records():
+    # K = V = 128, chunk 64: the status block plus one 149504-byte record per chunk per (b, hv)
+    B, T, HV = 2, 1000, 8
+    nc = (T + 63) // 64
+    assert kda.workspace_size(B, T, 4, HV, 128, 128, 64) == 256 + B * HV * nc * 149504
+    assert kda.workspace_size(B, T, 4, HV, 128, 64, 64) == 256
+    assert kda.workspace_size(B, T, 4, HV, 128, 128, 16) == 256
+
+
+def test_schedule_choice():
+    L = kda.lib
+    full = kda.workspace_size(2, 1000, 4, 8, 128, 128, 64)
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, kda.BF16, full) == kda.SCHEDULE_TC_TWO_PASS
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, kda.BF16, full - 1) == kda.SCHEDULE_TC_SINGLE_PASS
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, kda.BF16, 256) == kda.SCHEDULE_TC_SINGLE_PASS
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, kda.F32, full) == kda.SCHEDULE_CUDA_CORE
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 64, 128, 64, kda.BF16, full) == kda.SCHEDULE_CUDA_CORE
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 16, kda.BF16, full) == kda.SCHEDULE_CUDA_CORE
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, kda.BF16, 255) == -1
+    assert L.kda_chunk_fwd_schedule(2, 1000, 3, 8, 128, 128, 64, kda.BF16, full) == -1
+    assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, 9, full) == -1
+    assert kda.schedule(2, 1000, 4, 8, 128, 128, 64) == kda.SCHEDULE_TC_TWO_PASS
+    assert kda.uses_tensor_cores(128, 128, 64) and not kda.uses_tensor_cores(64, 64, 64)
