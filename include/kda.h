@@ -81,9 +81,10 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
 /*
  * kda_chunk_fwd_workspace_size -- bytes of device workspace with which kda_chunk_fwd
  * runs its fastest schedule for these sizes.  Always >= 256: the first 256 bytes hold
- * the on-device status word read by kda_read_status.  For K = V = 128 and chunk 64 it
- * adds the per-chunk records of the two-pass schedule (about 146 KiB per chunk of 64
- * tokens per (sequence, value head)).  Returns 0 for sizes kda_chunk_fwd rejects.
+ * the on-device status word read by kda_read_status.  For K = V = 128, chunk 64 and at
+ * most 96 (sequence, value head) pairs (B * HV) it adds the per-chunk records of the
+ * two-pass schedule (146 KiB per chunk of 64 tokens per pair).  Returns 0 for sizes
+ * kda_chunk_fwd rejects.
  */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk);
 
@@ -93,11 +94,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, i
  * recurrence above token by token, computed C tokens at a time with the
  * in-chunk cumulative log-decay, the triangular solve for the in-chunk delta
  * errors and one state update per chunk.
- * Schedules (bf16 inputs, K = V = 128, chunk 64): with a workspace of at least
- * kda_chunk_fwd_workspace_size bytes, two passes -- every chunk's local work in
- * parallel, then the state recurrence over chunks; with a smaller workspace (>= 256
- * bytes), one pass with one CTA per (sequence, value head).  Both compute the same
- * quantities to the same tolerance.  Other shapes and float32 inputs use one pass.
+ * Schedules (bf16 inputs, K = V = 128, chunk 64): for at most 96 (sequence, value head)
+ * pairs and a workspace of at least kda_chunk_fwd_workspace_size bytes, two passes --
+ * every chunk's local work in parallel, then the state recurrence over chunks; otherwise
+ * one pass with one CTA per pair.  Both compute the same quantities to the same
+ * tolerance.  Other shapes and float32 inputs use one pass on the CUDA cores.
  *   q, k     [B, T, H, K]   dtype
  *   v        [B, T, HV, V]  dtype
  *   g        [B, T, HV, K]  dtype   g_raw when gate_mode != NONE, else the log decay (<= 0)

@@ -60,6 +60,11 @@ bool sizes_ok(int B, int T, int H, int HV, int K, int V, int chunk) {
            (chunk == 16 || chunk == 64);
 }
 
+// Up to this many (sequence, value head) pairs the two-pass schedule is the faster one on a
+// 148-SM B200: with more, one CTA per pair already keeps most SMs busy in the single pass, while
+// the two-pass schedule adds the round trip of the per-chunk records through memory.
+constexpr long long kTwoPassMaxPairs = 96;
+
 // The tensor-core schedules cover K = V = 128, chunk 64 with bf16 inputs.  With float32 inputs the
 // stated tolerance (1e-4) is tighter than tf32 products allow, so those (and the other shapes) run
 // on the CUDA-core kernel in fp32.
@@ -99,7 +104,8 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk) {
     if (!sizes_ok(B, T, H, HV, K, V, chunk)) return 0;
-    if (split_shape(K, V, chunk)) return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
+    if (split_shape(K, V, chunk) && (long long)B * HV <= kTwoPassMaxPairs)
+        return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
     return kStatusBytes;
 }
 
@@ -108,7 +114,8 @@ int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk,
     if (!sizes_ok(B, T, H, HV, K, V, chunk) || (dtype != KDA_F32 && dtype != KDA_BF16) || workspace_bytes < kStatusBytes)
         return -1;
     if (dtype != KDA_BF16 || !split_shape(K, V, chunk)) return KDA_SCHEDULE_CUDA_CORE;
-    if (workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV)) return KDA_SCHEDULE_TC_TWO_PASS;
+    if ((long long)B * HV <= kTwoPassMaxPairs && workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
+        return KDA_SCHEDULE_TC_TWO_PASS;
     return KDA_SCHEDULE_TC_SINGLE_PASS;
 }
 

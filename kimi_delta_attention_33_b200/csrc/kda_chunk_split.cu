@@ -50,7 +50,8 @@ struct Rec {
 
 struct PrepLayout {
     static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1), then [W; Qhat] (record WQ)
-    static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling scratch
+    static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling
+                                             //   scratch; then U^T [128][64] fp32 (record UT)
     static constexpr uint32_t XS = CK + 64 * RP * 4;
     static constexpr uint32_t KA = 98304;    // [256][64]: Kchk^T rows 0-127, A rows 128-191, Tb rows 192-255
     static constexpr uint32_t GM = 163840;   // g staging (bf16) -> Gam (fp32) -> Khat^T [128][64] (B rows 0-127 of M7)
@@ -82,7 +83,7 @@ struct StateLayout {
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
-constexpr int STATE_THREADS = 128;
+constexpr int STATE_THREADS = 256;
 
 struct Task {
     int pair, c, b, hv, h, nn;
@@ -176,6 +177,20 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         unsigned char* rec = rec_base + (size_t)task * Rec::BYTES;
         const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[tk.hv]) : 0.0f;
 
+        // the next chunk of this CTA: bring its q, k, v and g rows into L2 (one 256-byte row per thread)
+        if (task + gridDim.x < ntasks) {
+            const Task nx = make_task(task + gridDim.x, T, H, HV, NC);
+            const int i = tid & (CH - 1), which = tid >> 6;
+            if (i < nx.nn) {
+                const size_t tok = nx.tk0 + i;
+                const bf16* src = which == 0   ? q + tok * qk_row + (size_t)nx.h * KD
+                                  : which == 1 ? k + tok * qk_row + (size_t)nx.h * KD
+                                  : which == 2 ? v + tok * v_row + (size_t)nx.hv * VD
+                                               : g + tok * g_row + (size_t)nx.hv * KD;
+                bulk_prefetch_l2(src, 256);
+            }
+        }
+
         // ---- gate and inclusive in-chunk cumulative log decay (two threads per key channel) ----
         bool slow;
         {
@@ -238,7 +253,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 vv[2 * x] = (uint32_t)sVs[(j + 0) * VD + vc] | ((uint32_t)sVs[(j + 1) * VD + vc] << 16);
                 vv[2 * x + 1] = (uint32_t)sVs[(j + 2) * VD + vc] | ((uint32_t)sVs[(j + 3) * VD + vc] << 16);
             }
-            // the previous chunk's record stores must be done reading X1 and KA before P3 rewrites them
+            // the previous chunk's record stores must be done reading X1, KA and CK before P3 rewrites them
             if (tid == 0) bulk_wait_read();
             __syncthreads();
 #pragma unroll
@@ -284,8 +299,13 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 *reinterpret_cast<uint4*>(smem + L::CK + cm_off(i, d, KD)) =
                     make_uint4(wc_[4 * hh], wc_[4 * hh + 1], wc_[4 * hh + 2], wc_[4 * hh + 3]);
             }
+            // Kchk^T: lanes that share a bank (same i & 3) take different d of their group of 8
+            const int rot = lane >> 2;
+            rotate_groups8(wc_, rot);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + t, i, CH)) = wc_[t];
+            for (int t = 0; t < 8; ++t)
+                *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) = wc_[t];
+            rotate_groups8(kh[it], rot);  // stored transposed the same way below
         }
         fence_proxy_async();
         cta_sync_tc();
@@ -296,9 +316,11 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             for (int it = 0; it < 4; ++it) {
                 const int u = tid + TC_THREADS * it;
                 const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
+                const int rot = lane >> 2;  // kh[it] holds its group of 8 rotated by rot
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
-                    *reinterpret_cast<uint32_t*>(smem + L::GM + cm_off(8 * d8 + t, i, CH)) = kh[it][t] ^ 0x80000000u;
+                    *reinterpret_cast<uint32_t*>(smem + L::GM + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) =
+                        kh[it][t] ^ 0x80000000u;
             }
         };
 
@@ -425,8 +447,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                             make_uint4(to_tf32(__uint_as_float(r[4 * c4])), to_tf32(__uint_as_float(r[4 * c4 + 1])),
                                        to_tf32(__uint_as_float(r[4 * c4 + 2])), to_tf32(__uint_as_float(r[4 * c4 + 3])));
                 }
-            } else {  // U -> record U^T (fp32, row = value column)
-                float* ut = reinterpret_cast<float*>(rec + Rec::UT);
+            } else {  // U^T (fp32, row = value column) -> CK region, free once Tb was built
+                float* ut = reinterpret_cast<float*>(smem + L::CK);
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
                     uint32_t r[32];
@@ -442,6 +464,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         if (tid == 0) {
             bulk_store(rec + Rec::WQ, s_base + L::X1, 65536);
             bulk_store(rec + Rec::KA, s_base + L::KA, Rec::KA_BYTES);
+            bulk_store(rec + Rec::UT, s_base + L::CK, 32768);
             bulk_commit();
         }
     }
@@ -461,8 +484,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
 // ---------------------------------------------------------------------------------------------
 template <int N>
 __device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
-    static_assert(N == 16 || N % 32 == 0, "row width");
-    if constexpr (N == 16) {
+    static_assert(N == 8 || N == 16 || N % 32 == 0, "row width");
+    if constexpr (N == 8) {
+        tmem_ld8(a, r);
+    } else if constexpr (N == 16) {
         tmem_ld16(a, r);
     } else {
 #pragma unroll
@@ -470,18 +495,23 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
     }
 }
 
+// Thread layout: warp w serves TMEM lane quarter w % 4 (rows 32 (w % 4) + lane of every
+// accumulator) and column half w / 4 of the value block (HALF = VB / 2 columns).
 template <int VB>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __restrict__ S0, int T, int HV, int NC,
                    bf16* __restrict__ o, float* __restrict__ S_T, unsigned int* __restrict__ status) {
     using L = StateLayout<VB>;
     constexpr int NVB = VD / VB;
+    constexpr int HALF = VB / 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     const uint32_t s_base = smem_u32(smem);
     const uint32_t bar_wq = s_base + L::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16;
     const int pair = blockIdx.x / NVB, vb0 = (blockIdx.x - pair * NVB) * VB;
     const int b = pair / HV, hv = pair - b * HV;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, c0 = (warp >> 2) * HALF;  // lane quarter, first column of this half
+    const int rot = lane >> 2;                          // store rotation (see rotate_groups8)
     const size_t v_row = (size_t)HV * VD;
     const unsigned char* rec0 = rec_base + (size_t)pair * NC * Rec::BYTES;
     auto rec = [&](int c) { return rec0 + (size_t)c * Rec::BYTES; };
@@ -516,21 +546,27 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         if (L::NKA == 2 && NC > 1) load_ka(1, 1);
     }
 
-    // this thread's key row of the state slice, exact fp32
-    const int d = tid;
-    float s[VB];
+    // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32
+    const int d = 32 * wq + lane;
+    float s[HALF];
 #pragma unroll
-    for (int j = 0; j < VB; j += 4) {
-        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * KD + d) * VD + vb0 + j)
+    for (int j = 0; j < HALF; j += 4) {
+        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * KD + d) * VD + vb0 + c0 + j)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         s[j] = x.x;
         s[j + 1] = x.y;
         s[j + 2] = x.z;
         s[j + 3] = x.w;
     }
+    // tf32(e^rho S)^T into the B operand of M8; lanes sharing a bank store different columns
     auto write_sop = [&](float er) {
+        uint32_t w[HALF];
 #pragma unroll
-        for (int j = 0; j < VB; ++j) *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(j, d, KD)) = to_tf32(er * s[j]);
+        for (int j = 0; j < HALF; ++j) w[j] = to_tf32(er * s[j]);
+        rotate_groups8(w, rot);
+#pragma unroll
+        for (int j = 0; j < HALF; ++j)
+            *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
     };
     const float* vec0 = reinterpret_cast<const float*>(rec(0) + Rec::VEC);
     float es = vec0[KD + d], ef = vec0[2 * KD + d];
@@ -573,18 +609,20 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             pending &= ~(2u << buf);
             if (c + 1 < NC) load_wq(c + 1);  // M8 has read WQ
         }
-        // ---- E = U - W S~ (rows 0-63: warps 0, 1) -> E^T tf32 operand --------------------------
+        // ---- E = U - W S~ (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
         const uint32_t ka = s_base + L::ka(buf);
-        if (warp < 2) {
-            const int j = tid;
+        if (wq < 2) {
+            const int j = d;
             const float* sU = reinterpret_cast<const float*>(smem + L::ka(buf) + Rec::KA_BYTES);
-            uint32_t r[VB];
-            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D1), r);
+            uint32_t r[HALF];
+            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
             tmem_wait_ld();
 #pragma unroll
-            for (int vv = 0; vv < VB; ++vv)
-                *reinterpret_cast<uint32_t*>(smem + L::EOP + cm_off(vv, j, CH)) =
-                    to_tf32(sU[vv * CH + j] - __uint_as_float(r[vv]));
+            for (int vv = 0; vv < HALF; ++vv) r[vv] = to_tf32(sU[(c0 + vv) * CH + j] - __uint_as_float(r[vv]));
+            rotate_groups8(r, rot);
+#pragma unroll
+            for (int vv = 0; vv < HALF; ++vv)
+                *reinterpret_cast<uint32_t*>(smem + L::EOP + cm_off(c0 + (vv & ~7) + ((vv + rot) & 7), j, CH)) = r[vv];
         }
         fence_proxy_async();
         cta_sync_tc();
@@ -601,16 +639,16 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         if (!__syncthreads_and(ok)) { aborted = true; break; }
         ph_mma ^= 1u;
         if (L::NKA == 1 && tid == 0 && c + 1 < NC) load_ka(c + 1, 0);
-        // ---- outputs (rows 64-127 of D1: warps 2, 3) ---------------------------------------------
-        if (warp >= 2) {
-            const int i = tid - 64;
-            uint32_t r[VB];
-            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D1), r);
+        // ---- outputs (rows 64-127 of D1: lane quarters 2, 3) -------------------------------------
+        if (wq >= 2) {
+            const int i = d - 64;
+            uint32_t r[HALF];
+            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
             tmem_wait_ld();
             if (i < n) {
-                bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0;
+                bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0 + c0;
 #pragma unroll
-                for (int j = 0; j < VB; j += 8) {
+                for (int j = 0; j < HALF; j += 8) {
                     uint4 w;
                     __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
                     __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
@@ -626,11 +664,11 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         }
         // ---- state: S = f (e^sig S + D2); S~ of the next chunk ----------------------------------
         {
-            uint32_t r[VB];
-            tmem_ld_row<VB>(taddr(tmem, 32 * warp, L::D2), r);
+            uint32_t r[HALF];
+            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D2 + c0), r);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < VB; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
+            for (int j = 0; j < HALF; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
         }
         if (c + 1 < NC) {
             write_sop(er_n);
@@ -653,8 +691,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         }
     } else if (S_T) {
 #pragma unroll
-        for (int j = 0; j < VB; j += 4)
-            *reinterpret_cast<float4*>(S_T + ((size_t)pair * KD + d) * VD + vb0 + j) =
+        for (int j = 0; j < HALF; j += 4)
+            *reinterpret_cast<float4*>(S_T + ((size_t)pair * KD + d) * VD + vb0 + c0 + j) =
                 make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
     }
     cta_sync_tc();

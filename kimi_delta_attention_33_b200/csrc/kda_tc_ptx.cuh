@@ -119,6 +119,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t a, uint32_t (&r)[16]) {
           "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(a));
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t a, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(a));
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t a, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -169,17 +174,41 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
                  : "memory");
 }
+// Bulk prefetch of global memory into L2 (no destination in this CTA).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the committed bulk stores of this thread have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until the committed bulk stores of this thread are complete.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Round-to-nearest fp32 -> tf32 (low 13 mantissa bits cleared); the tensor core reads the rest.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+// fp32 -> operand word for a kind::tf32 MMA.  The tensor core reads the top 19 bits of each word
+// (sign, exponent, 10 mantissa bits) and ignores the low 13; adding half a unit of the 10th
+// mantissa bit to the magnitude first makes that truncation a round to nearest (ties away from
+// zero; a carry into the exponent gives the correctly rounded next binade).  One integer add.
+__device__ __forceinline__ uint32_t to_tf32(float x) { return __float_as_uint(x) + 0x1000u; }
+
+// Rotation inside aligned groups of 8: a[g + k] <- a[g + ((k + r) & 7)] for r in 0..7, by three
+// conditional rotations (no dynamic register indexing).  Used to give the 8 lanes that would store
+// to the same shared-memory bank 8 different words of their group, so that transposed stores into
+// the operand tiling are free of bank conflicts.
+template <int N>
+__device__ __forceinline__ void rotate_groups8(uint32_t (&a)[N], int r) {
+    static_assert(N % 8 == 0, "groups of 8");
+#pragma unroll
+    for (int sh = 1; sh < 8; sh <<= 1) {
+        const bool on = (r & sh) != 0;
+#pragma unroll
+        for (int g = 0; g < N; g += 8) {
+            uint32_t t[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = a[g + ((k + sh) & 7)];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a[g + k] = on ? t[k] : a[g + k];
+        }
+    }
 }
 
 // Row-of-TMEM loader: N columns (16 or 32) starting at `col` for this warp's 32 lanes.

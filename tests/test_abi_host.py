@@ -119,6 +119,8 @@ def test_workspace_size_two_pass_records():
     assert kda.workspace_size(B, T, 4, HV, 128, 128, 64) == 256 + B * HV * nc * 149504
     assert kda.workspace_size(B, T, 4, HV, 128, 64, 64) == 256
     assert kda.workspace_size(B, T, 4, HV, 128, 128, 16) == 256
+    assert kda.workspace_size(12, T, 8, 8, 128, 128, 64) == 256 + 12 * 8 * nc * 149504  # 96 pairs
+    assert kda.workspace_size(13, T, 8, 8, 128, 128, 64) == 256                          # 104 pairs
 
 
 def test_schedule_choice():
@@ -134,4 +136,5 @@ def test_schedule_choice():
     assert L.kda_chunk_fwd_schedule(2, 1000, 3, 8, 128, 128, 64, kda.BF16, full) == -1
     assert L.kda_chunk_fwd_schedule(2, 1000, 4, 8, 128, 128, 64, 9, full) == -1
     assert kda.schedule(2, 1000, 4, 8, 128, 128, 64) == kda.SCHEDULE_TC_TWO_PASS
+    assert L.kda_chunk_fwd_schedule(8, 1000, 16, 16, 128, 128, 64, kda.BF16, 1 << 40) == kda.SCHEDULE_TC_SINGLE_PASS
     assert kda.uses_tensor_cores(128, 128, 64) and not kda.uses_tensor_cores(64, 64, 64)

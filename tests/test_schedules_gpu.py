@@ -5,7 +5,8 @@ when it is given ``kda_chunk_fwd_workspace_size`` bytes of workspace, and the si
 (one CTA per (sequence, value head)) when it is given only the 256-byte status block.  Each case
 here runs both and checks each against the float64 oracle on the same seeded inputs, with the bar
 of the other parity tests: max|x - x_ref| / max|x_ref| <= 5e-3 for o and the final state.
-The (B, HV) sizes reach every value-block width of the state pass (16, 32 and 64 columns).
+The (B, HV) sizes reach every value-block width of the state pass (16, 32 and 64 columns); above
+96 pairs only the single pass is offered.
 """
 import numpy as np
 import pytest
@@ -25,8 +26,13 @@ def _workspace(w, schedule):
     if schedule == "single_pass":
         return torch.empty(256, dtype=torch.uint8, device="cuda")
     need = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
+    if w.B * w.HV > 96:  # the two-pass schedule is not offered for this many pairs
+        assert need == 256
+        pytest.skip("more (sequence, head) pairs than the two-pass schedule takes")
     assert need > 256
-    return torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    assert kda.schedule(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, need) == kda.SCHEDULE_TC_TWO_PASS
+    return ws
 
 
 def _run(w, xd, schedule, **kw):
@@ -60,7 +66,7 @@ def test_ragged_lengths_both_schedules(schedule, T):
 
 # (B, HV) reaching value blocks of 16 (<= 18 pairs), 32 (<= 37 pairs) and 64 columns
 @pytest.mark.parametrize("schedule", SCHEDULES)
-@pytest.mark.parametrize("B,H,HV", [(1, 1, 1), (2, 4, 8), (3, 5, 10), (1, 8, 32), (5, 8, 8), (2, 16, 48)])
+@pytest.mark.parametrize("B,H,HV", [(1, 1, 1), (2, 4, 8), (3, 5, 10), (1, 8, 32), (5, 8, 8), (2, 16, 48), (4, 8, 24)])
 def test_pair_counts_both_schedules(schedule, B, H, HV):
     w = _wl(B=B, T=130, H=H, HV=HV)
     x = make_inputs(w)
@@ -120,7 +126,7 @@ def test_schedules_agree_with_each_other():
     assert rel_err(S1, S2.cpu().numpy().astype(np.float64)) <= TOL[w.dtype]
 
 
-@pytest.mark.parametrize("wid", [2, 3, 4])
+@pytest.mark.parametrize("wid", [2, 4])
 def test_benchmark_workloads_single_pass_sampled(wid):
     # the benchmark runs these with the two-pass schedule (test_parity_gpu); here the other one
     w = WORKLOADS[wid]
