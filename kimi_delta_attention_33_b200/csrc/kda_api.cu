@@ -104,7 +104,8 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk) {
     if (!sizes_ok(B, T, H, HV, K, V, chunk)) return 0;
-    if (split_shape(K, V, chunk) && (long long)B * HV <= kTwoPassMaxPairs)
+    if (split_shape(K, V, chunk) && (long long)B * HV <= kTwoPassMaxPairs &&
+        (long long)B * HV * ((T + 63) / 64) < (1ll << 30))
         return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
     return kStatusBytes;
 }
@@ -114,7 +115,9 @@ int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk,
     if (!sizes_ok(B, T, H, HV, K, V, chunk) || (dtype != KDA_F32 && dtype != KDA_BF16) || workspace_bytes < kStatusBytes)
         return -1;
     if (dtype != KDA_BF16 || !split_shape(K, V, chunk)) return KDA_SCHEDULE_CUDA_CORE;
-    if ((long long)B * HV <= kTwoPassMaxPairs && workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
+    const long long chunks = (long long)B * HV * ((T + 63) / 64);  // one prep task per chunk, counted in an int
+    if ((long long)B * HV <= kTwoPassMaxPairs && chunks < (1ll << 30) &&
+        workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
         return KDA_SCHEDULE_TC_TWO_PASS;
     return KDA_SCHEDULE_TC_SINGLE_PASS;
 }

@@ -49,16 +49,19 @@ struct Rec {
 };
 
 struct PrepLayout {
-    static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1), then [W; Qhat] (record WQ)
+    static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1); Qhat is the record's WQ rows
+                                             //   64-127; once M1 is done rows 0-63 stage the next chunk's
+                                             //   g (bf16 [64][128]) and v (bf16 [64][128]) tiles
     static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling
                                              //   scratch; then U^T [128][64] fp32 (record UT)
     static constexpr uint32_t XS = CK + 64 * RP * 4;
-    static constexpr uint32_t KA = 98304;    // [256][64]: Kchk^T rows 0-127, A rows 128-191, Tb rows 192-255
-    static constexpr uint32_t GM = 163840;   // g staging (bf16) -> Gam (fp32) -> Khat^T [128][64] (B rows 0-127 of M7)
-    static constexpr uint32_t VT = 196608;   // v staging (bf16, upper half) -> V^T [128][64] (B rows 128-255 of M7)
+    static constexpr uint32_t KA = 98304;    // [256][64]: Kchk^T rows 0-127 (record KA, first part),
+                                             //   Tb twice in rows 128-255 (A of M7)
+    static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
+    static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)
     static constexpr uint32_t VEC = 229376;
     static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024;
-    static constexpr uint32_t MBAR = VEC + 1280, TBASE = MBAR + 8, FLAG = TBASE + 4;
+    static constexpr uint32_t MBAR = VEC + 1280, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8, FLAG = TBASE + 4;
     static constexpr uint32_t BYTES = FLAG + 4;
     static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
@@ -70,8 +73,9 @@ template <int VB>
 struct StateLayout {
     static constexpr int NKA = VB <= 32 ? 2 : 1;              // KA / U buffers
     static constexpr uint32_t WQ = 0;                          // [128][128]
-    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], then U^T [VB][64]
-    static constexpr uint32_t KA_STRIDE = Rec::KA_BYTES + VB * 256;
+    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], U^T [VB][64], VEC
+    static constexpr uint32_t UT_OFF = Rec::KA_BYTES, VEC_OFF = Rec::KA_BYTES + VB * 256;
+    static constexpr uint32_t KA_STRIDE = VEC_OFF + 3 * 512;
     static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S~^T [VB][128]   (B of M8)
     static constexpr uint32_t EOP = SOP + VB * 128 * 4;        // tf32 E^T  [VB][64]    (B of M9, M10)
     static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1]
@@ -90,10 +94,10 @@ struct Task {
     size_t tk0;  // token index (b * T + first token of the chunk)
 };
 
-__device__ __forceinline__ Task make_task(long long task, int T, int H, int HV, int NC) {
+__device__ __forceinline__ Task make_task(int task, int T, int H, int HV, int NC) {
     Task t;
-    t.pair = (int)(task / NC);
-    t.c = (int)(task - (long long)t.pair * NC);
+    t.pair = task / NC;
+    t.c = task - t.pair * NC;
     t.b = t.pair / HV;
     t.hv = t.pair - t.b * HV;
     t.h = t.hv / (HV / H);
@@ -107,13 +111,15 @@ __device__ __forceinline__ Task make_task(long long task, int T, int H, int HV, 
 // ---------------------------------------------------------------------------------------------
 // Pass 1: chunk-local work for every chunk.
 // ---------------------------------------------------------------------------------------------
+template <int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                   const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
-                  const float* __restrict__ dt_bias, int T, int H, int HV, int NC, long long ntasks, int gate_mode,
+                  const float* __restrict__ dt_bias, int T, int H, int HV, int NC, int ntasks,
                   float lower_bound, float scale, unsigned char* __restrict__ rec_base,
                   unsigned int* __restrict__ status) {
     using L = PrepLayout;
+    constexpr int gate_mode = MODE;
     extern __shared__ __align__(1024) unsigned char smem[];
     float* sRho = reinterpret_cast<float*>(smem + L::RHO);
     float* sSig = reinterpret_cast<float*>(smem + L::SIG);
@@ -121,40 +127,51 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
-    const bf16* sG = reinterpret_cast<const bf16*>(smem + L::GM);
+    const bf16* sG = reinterpret_cast<const bf16*>(smem + L::X1);  // staged g tile
     uint32_t* sFlag = reinterpret_cast<uint32_t*>(smem + L::FLAG);
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t mbar = s_base + L::MBAR;
+    const uint32_t mbar = s_base + L::MBAR, mbar_in = s_base + L::MBAR_IN;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
     const size_t qk_row = (size_t)H * KD, v_row = (size_t)HV * VD, g_row = (size_t)HV * KD;
 
-    if (tid == 0) mbar_init(mbar, 1);
+    // the state kernel that follows may start its set-up as SMs free up; it waits for this grid's
+    // completion before it reads any record
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_init(mbar_in, 1);
+    }
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
     if (tid == 0) *sFlag = 0u;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
-    uint32_t phase = 0;
-    bool aborted = false;
+    uint32_t phase = 0, phase_in = 0;
+    bool aborted = false, in_pending = false;
 
-    // Inputs of one chunk: g and v tiles into shared staging by cp.async (rows past T zero-filled),
-    // q, k and beta into registers.
+    // Inputs of one chunk: g and v tiles into the staging half of X1 by bulk copies, one 256-byte row
+    // per thread, completing on mbar_in (rows past T are zeroed by plain stores instead); q, k, beta,
+    // this head's A_log and this thread's dt_bias entry into registers.
     uint4 qr[4], kr[4];
-    float bload;
+    uint32_t beta_bits;  // raw bf16 bits of this thread's beta (row tid), converted where used
+    float alog_in = 0.f, bias_in = 0.f;
     auto load_inputs = [&](const Task& tk) {
-        const uint32_t gs = s_base + L::GM, vs = s_base + L::VT + 16384;
+        const int i = tid & (CH - 1), which = tid >> 6;  // which: 0 g, 1 v (threads 128-255: none)
+        if (tid == 0) mbar_expect_tx(mbar_in, 2u * 256u * (uint32_t)tk.nn);
+        if (which < 2) {
+            const uint32_t dst = s_base + L::X1 + which * 16384 + i * 256;
+            if (i < tk.nn) {
+                const bf16* src = which == 0 ? g + (tk.tk0 + i) * g_row + (size_t)tk.hv * KD
+                                             : v + (tk.tk0 + i) * v_row + (size_t)tk.hv * VD;
+                bulk_load(dst, src, 256, mbar_in);
+            } else {
+                uint4* z = reinterpret_cast<uint4*>(smem + L::X1 + which * 16384 + i * 256);
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
-            const int i = u >> 4, c = u & 15;
-            const bool ok = i < tk.nn;
-            cp_async16(gs + i * 256 + c * 16, ok ? g + (tk.tk0 + i) * g_row + (size_t)tk.hv * KD + 8 * c : g,
-                       ok ? 16u : 0u);
-            cp_async16(vs + i * 256 + c * 16, ok ? v + (tk.tk0 + i) * v_row + (size_t)tk.hv * VD + 8 * c : v,
-                       ok ? 16u : 0u);
+                for (int c = 0; c < 16; ++c) z[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
-        cp_async_commit();
+        in_pending = true;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
             const int u = tid + TC_THREADS * it;
@@ -166,16 +183,21 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 kr[it] = __ldg(reinterpret_cast<const uint4*>(k + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD + 8 * d8));
             }
         }
-        bload = (tid < tk.nn) ? to_f32(beta[(tk.tk0 + tid) * HV + tk.hv]) : 0.f;
+        beta_bits = (tid < tk.nn) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(beta) + (tk.tk0 + tid) * HV + tk.hv)
+                                  : 0u;
+        if (gate_mode != KDA_GATE_NONE) {
+            alog_in = __ldg(A_log + tk.hv);
+            bias_in = dt_bias != nullptr ? __ldg(dt_bias + tk.hv * KD + (tid & (KD - 1))) : 0.f;
+        }
     };
 
-    long long task = blockIdx.x;
+    int task = blockIdx.x;
     if (task < ntasks) load_inputs(make_task(task, T, H, HV, NC));
 
     for (; task < ntasks && !aborted; task += gridDim.x) {
         const Task tk = make_task(task, T, H, HV, NC);
         unsigned char* rec = rec_base + (size_t)task * Rec::BYTES;
-        const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[tk.hv]) : 0.0f;
+        const float rate = (gate_mode != KDA_GATE_NONE) ? expf(alog_in) : 0.0f;
 
         // the next chunk of this CTA: bring its q, k, v and g rows into L2 (one 256-byte row per thread)
         if (task + gridDim.x < ntasks) {
@@ -195,27 +217,21 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         bool slow;
         {
             const int nn = tk.nn, mr = (nn - 1) >> 1;
-            cp_async_wait_all();
-            __syncthreads();
-            if (tid < CH) sBeta[tid] = bload;
+            const bool ok_in = mbar_wait(mbar_in, phase_in, WAIT_POLLS);
+            if (!__syncthreads_and(ok_in)) { aborted = true; break; }
+            phase_in ^= 1u;
+            in_pending = false;
+            if (tid < CH) sBeta[tid] = __uint_as_float(beta_bits << 16);
             const int gd = tid & (KD - 1), gh = tid >> 7;
-            float gv[32];
-            const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[tk.hv * KD + gd] : 0.0f;
-            float acc = 0.f;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int i = 32 * gh + r;
-                const float x = (i < nn) ? gate_value_fast(__bfloat162float(sG[i * KD + gd]), bias, rate, gate_mode,
-                                                           lower_bound)
-                                         : 0.f;
-                acc += x;
-                gv[r] = acc;
-            }
+            const float acc = gate_rows32_to<MODE>(sG + 32 * gh * KD + gd, KD, nn - 32 * gh, bias_in, rate, lower_bound,
+                                                   sGam, [&](int r) { return gidx(32 * gh + r, gd); });
             if (gh == 0) sSig[gd] = acc;  // scratch: first-half totals
-            __syncthreads();              // the g staging has been read: GM becomes Gam
-            const float off = gh ? sSig[gd] : 0.f;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) sGam[gidx(32 * gh + r, gd)] = gv[r] + off;
+            __syncthreads();
+            if (gh == 1) {  // second half: add the first half's total
+                const float off = sSig[gd];
+#pragma unroll 4
+                for (int r = 32; r < 64; ++r) sGam[gidx(r, gd)] += off;
+            }
             __syncthreads();
             if (tid < KD) {
                 const int d = tid;
@@ -242,9 +258,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
         }
 
-        // ---- V^T into VT from the staged v tile (upper half of VT) ------------------------------
+        // ---- V^T into VT from the staged v tile ----------------------------------------------------
         {
-            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::VT + 16384);
+            const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::X1 + 16384);
             const int vc = tid & (VD - 1), jq0 = tid >> 7;
             uint32_t vv[16];
 #pragma unroll
@@ -253,7 +269,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 vv[2 * x] = (uint32_t)sVs[(j + 0) * VD + vc] | ((uint32_t)sVs[(j + 1) * VD + vc] << 16);
                 vv[2 * x + 1] = (uint32_t)sVs[(j + 2) * VD + vc] | ((uint32_t)sVs[(j + 3) * VD + vc] << 16);
             }
-            // the previous chunk's record stores must be done reading X1, KA and CK before P3 rewrites them
+            // the previous chunk's record stores must be done reading X1, KA and CK before P3 rewrites
+            // them (and the staged tiles in X1 must all be read)
             if (tid == 0) bulk_wait_read();
             __syncthreads();
 #pragma unroll
@@ -336,6 +353,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             fence_after_sync();
             if (!__syncthreads_and(ok)) { aborted = true; break; }
             phase ^= 1u;
+            // X1 rows 0-63 are free: stage the next chunk of this CTA during the rest of this one
+            if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
             uint32_t raw[32];
             tmem_ld32(taddr(tmem, 32 * wq, 32 * wh), raw);
             tmem_wait_ld();
@@ -347,8 +366,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                     const int j = 32 * wh + jj;
                     sRT[i * RP + j] = (j < i) ? bi * __uint_as_float(raw[jj]) : 0.f;
                 }
-            } else {  // rows 64-127 hold A (unmasked)
+            } else {  // rows 64-127 hold A (unmasked): masked, tf32, straight into the record
                 const int i = 32 * (wq - 2) + lane;
+                unsigned char* ra = rec + Rec::KA + 32768;
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 4) {
                     const int j = 32 * wh + jj;
@@ -357,10 +377,11 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                     w4.y = to_tf32(j + 1 <= i ? __uint_as_float(raw[jj + 1]) : 0.f);
                     w4.z = to_tf32(j + 2 <= i ? __uint_as_float(raw[jj + 2]) : 0.f);
                     w4.w = to_tf32(j + 3 <= i ? __uint_as_float(raw[jj + 3]) : 0.f);
-                    *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, j, CH)) = w4;
+                    *reinterpret_cast<uint4*>(ra + cm_off(i, j, CH)) = w4;
                 }
             }
         } else {
+            if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
             // exact decay factors: 4096 (i, j) cells, 16 per thread; Gam is still in GM
             float av[16], rr[16];
 #pragma unroll 1
@@ -387,14 +408,14 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             for (int x = 0; x < 16; ++x) {
                 const int p = tid + TC_THREADS * x;
                 const int i = p >> 6, j = p & 63;
-                *reinterpret_cast<uint32_t*>(smem + L::KA + 32768 + cm_off(i, j, CH)) = to_tf32(av[x]);
+                *reinterpret_cast<uint32_t*>(rec + Rec::KA + 32768 + cm_off(i, j, CH)) = to_tf32(av[x]);
                 sRT[i * RP + j] = rr[x];
             }
             write_khat_t();
         }
         __syncthreads();
 
-        // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 192-255 ---------------------
+        // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 and 192-255 ----------
         tri_inverse_step<1>(sRT, sX, tid);
         tri_inverse_step<2>(sRT, sX, tid);
         tri_inverse_step<4>(sRT, sX, tid);
@@ -414,12 +435,14 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 const float tv = (j < i) ? tr[t] : (j == i ? 1.f : 0.f);
                 w[t] = to_tf32(tv * sBeta[j]);
             }
-            *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, 4 * j4, CH)) = make_uint4(w[0], w[1], w[2], w[3]);
+            const uint4 w4 = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, 4 * j4, CH)) = w4;
+            *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, 4 * j4, CH)) = w4;
         }
         fence_proxy_async();
         cta_sync_tc();
 
-        // ---- M7: D[128][256] = [A; Tb] [Khat^T; V^T]^T; rows 64-127 hold W | U --------------------
+        // ---- M7: D[128][256] = [Tb; Tb] [Khat^T; V^T]^T; rows 0-63 and 64-127 both hold W | U ------
         if (tid == 0) {
             gemm_tf32(tmem, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::GM, CH / 4 * 128, idesc_tf32(128, 256),
                       CH / 8, false);
@@ -431,39 +454,39 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (!__syncthreads_and(ok)) { aborted = true; break; }
             phase ^= 1u;
         }
-        // GM and VT are free: stage the next chunk of this CTA while the record is written out
-        if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
-        if (wq >= 2) {
-            const int i = 32 * (wq - 2) + lane;
-            if (wh == 0) {  // W -> X1 rows 0-63 (tf32)
+        {
+            // lane quarters 0-1 read W (rows 0-63), quarters 2-3 read U (rows 64-127); wh picks 64 columns
+            const int i = 32 * (wq & 1) + lane;
+            const int col = (wq < 2 ? 0 : 128) + 64 * wh;
+            uint32_t r0[32], r1[32];
+            tmem_ld32(taddr(tmem, 32 * wq, col), r0);
+            tmem_ld32(taddr(tmem, 32 * wq, col + 32), r1);
+            tmem_wait_ld();
+            if (wq < 2) {  // W -> record WQ rows 0-63 (tf32, operand tiling)
+                unsigned char* rw = rec + Rec::WQ;
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr(tmem, 32 * wq, 32 * blk), r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4)
-                        *reinterpret_cast<uint4*>(smem + L::X1 + cm_off(i, 32 * blk + 4 * c4, KD)) =
-                            make_uint4(to_tf32(__uint_as_float(r[4 * c4])), to_tf32(__uint_as_float(r[4 * c4 + 1])),
-                                       to_tf32(__uint_as_float(r[4 * c4 + 2])), to_tf32(__uint_as_float(r[4 * c4 + 3])));
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    *reinterpret_cast<uint4*>(rw + cm_off(i, 64 * wh + 4 * c4, KD)) =
+                        make_uint4(to_tf32(__uint_as_float(r0[4 * c4])), to_tf32(__uint_as_float(r0[4 * c4 + 1])),
+                                   to_tf32(__uint_as_float(r0[4 * c4 + 2])), to_tf32(__uint_as_float(r0[4 * c4 + 3])));
+                    *reinterpret_cast<uint4*>(rw + cm_off(i, 64 * wh + 32 + 4 * c4, KD)) =
+                        make_uint4(to_tf32(__uint_as_float(r1[4 * c4])), to_tf32(__uint_as_float(r1[4 * c4 + 1])),
+                                   to_tf32(__uint_as_float(r1[4 * c4 + 2])), to_tf32(__uint_as_float(r1[4 * c4 + 3])));
                 }
             } else {  // U^T (fp32, row = value column) -> CK region, free once Tb was built
                 float* ut = reinterpret_cast<float*>(smem + L::CK);
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr(tmem, 32 * wq, 128 + 32 * blk), r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int cc = 0; cc < 32; ++cc) ut[(32 * blk + cc) * CH + i] = __uint_as_float(r[cc]);
+                for (int cc = 0; cc < 32; ++cc) {
+                    ut[(64 * wh + cc) * CH + i] = __uint_as_float(r0[cc]);
+                    ut[(64 * wh + 32 + cc) * CH + i] = __uint_as_float(r1[cc]);
                 }
             }
         }
         fence_proxy_async();
         cta_sync_tc();
         if (tid == 0) {
-            bulk_store(rec + Rec::WQ, s_base + L::X1, 65536);
-            bulk_store(rec + Rec::KA, s_base + L::KA, Rec::KA_BYTES);
+            bulk_store(rec + Rec::WQ + 32768, s_base + L::X1 + 32768, 32768);  // Qhat; W went straight out
+            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);  // Kchk^T; A went straight to the record
             bulk_store(rec + Rec::UT, s_base + L::CK, 32768);
             bulk_commit();
         }
@@ -472,8 +495,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     if (aborted) {
         if (tid == 0) atomicOr(status, STATUS_TIMEOUT);
         mbar_wait(mbar, phase, WAIT_POLLS);  // one more bounded chance for an MMA in flight to drain
+        if (in_pending) mbar_wait(mbar_in, phase_in, WAIT_POLLS);  // and for staged copies in flight
     }
-    cp_async_wait_all();
     if (tid == 0) bulk_wait_all();
     cta_sync_tc();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
@@ -535,17 +558,12 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     };
     auto load_ka = [&](int c, int buf) {
         const uint32_t bar = bar_ka0 + 8 * buf;
-        mbar_expect_tx(bar, Rec::KA_BYTES + VB * 256);
+        mbar_expect_tx(bar, L::KA_STRIDE);
         bulk_load(s_base + L::ka(buf), rec(c) + Rec::KA, Rec::KA_BYTES, bar);
-        bulk_load(s_base + L::ka(buf) + Rec::KA_BYTES, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
+        bulk_load(s_base + L::ka(buf) + L::UT_OFF, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
+        bulk_load(s_base + L::ka(buf) + L::VEC_OFF, rec(c) + Rec::VEC, 3 * 512, bar);
         pending |= 2u << buf;
     };
-    if (tid == 0) {
-        load_wq(0);
-        load_ka(0, 0);
-        if (L::NKA == 2 && NC > 1) load_ka(1, 1);
-    }
-
     // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32
     const int d = 32 * wq + lane;
     float s[HALF];
@@ -558,6 +576,18 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         s[j + 2] = x.z;
         s[j + 3] = x.w;
     }
+    // per-key vectors of the chunk held in KA buffer `buf`: e^rho, e^sig, f
+    auto vec = [&](int buf, int which) {
+        return reinterpret_cast<const float*>(smem + L::ka(buf) + L::VEC_OFF)[which * KD + d];
+    };
+    // the chunk records are written by the preceding prep kernel: wait for it (a no-op unless this
+    // grid was launched as its programmatic dependent, whose set-up above then overlapped its tail)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) {
+        load_wq(0);
+        load_ka(0, 0);
+        if (L::NKA == 2 && NC > 1) load_ka(1, 1);
+    }
     // tf32(e^rho S)^T into the B operand of M8; lanes sharing a bank store different columns
     auto write_sop = [&](float er) {
         uint32_t w[HALF];
@@ -568,24 +598,20 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         for (int j = 0; j < HALF; ++j)
             *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
     };
-    const float* vec0 = reinterpret_cast<const float*>(rec(0) + Rec::VEC);
-    float es = vec0[KD + d], ef = vec0[2 * KD + d];
-    write_sop(vec0[d]);
-    fence_proxy_async();
-    cta_sync_tc();
-
     uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0;
     bool aborted = false;
-    for (int c = 0; c < NC; ++c) {
+    {
+        const bool ok = mbar_wait(bar_ka0, 0, WAIT_POLLS);  // chunk 0's KA group holds its vectors
+        if (!__syncthreads_and(ok)) aborted = true;
+    }
+    if (!aborted) write_sop(vec(0, 0));
+    fence_proxy_async();
+    cta_sync_tc();
+    for (int c = 0; c < NC && !aborted; ++c) {
         const int buf = (L::NKA == 2) ? (c & 1) : 0;
         const int n = min(CH, T - c * CH);
-        float er_n = 0.f, es_n = 0.f, ef_n = 0.f;  // the next chunk's vectors, consumed at the end
-        if (c + 1 < NC) {
-            const float* vn = reinterpret_cast<const float*>(rec(c + 1) + Rec::VEC);
-            er_n = __ldg(vn + d);
-            es_n = __ldg(vn + KD + d);
-            ef_n = __ldg(vn + 2 * KD + d);
-        }
+        float er_n = 0.f;  // with one KA buffer the next chunk's e^rho comes from the record directly
+        if (L::NKA == 1 && c + 1 < NC) er_n = __ldg(reinterpret_cast<const float*>(rec(c + 1) + Rec::VEC) + d);
         // ---- M8: D1 = [W; Qhat] S~ ------------------------------------------------------------
         bool ok = true;
         if (tid == 0) {
@@ -605,6 +631,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         ph_wq ^= 1u;
         ph_mma ^= 1u;
         ph_ka ^= 1u << buf;
+        // this chunk's e^sig and f, read before a single KA buffer is refilled below
+        const float es = vec(buf, 1), ef = vec(buf, 2);
         if (tid == 0) {
             pending &= ~(2u << buf);
             if (c + 1 < NC) load_wq(c + 1);  // M8 has read WQ
@@ -613,7 +641,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         const uint32_t ka = s_base + L::ka(buf);
         if (wq < 2) {
             const int j = d;
-            const float* sU = reinterpret_cast<const float*>(smem + L::ka(buf) + Rec::KA_BYTES);
+            const float* sU = reinterpret_cast<const float*>(smem + L::ka(buf) + L::UT_OFF);
             uint32_t r[HALF];
             tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
             tmem_wait_ld();
@@ -671,9 +699,13 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             for (int j = 0; j < HALF; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
         }
         if (c + 1 < NC) {
+            if (L::NKA == 2) {  // the next chunk's KA group (loaded a chunk ago) holds its e^rho
+                const int nb = buf ^ 1;
+                const bool okn = mbar_wait(bar_ka0 + 8 * nb, (ph_ka >> nb) & 1u, WAIT_POLLS);
+                if (!__syncthreads_and(okn)) { aborted = true; break; }
+                er_n = vec(nb, 0);
+            }
             write_sop(er_n);
-            es = es_n;
-            ef = ef_n;
         }
         fence_proxy_async();
         cta_sync_tc();
@@ -706,34 +738,53 @@ size_t chunk_split_workspace(int B, int T, int HV) {
 }
 
 namespace {
+template <int MODE>
+cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PrepLayout::BYTES);
+    if (e != cudaSuccess) return e;
+    chunk_prep_kernel<MODE><<<grid, TC_THREADS, PrepLayout::BYTES, a.stream>>>(
+        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
+        static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
+        ntasks, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status);
+    return cudaGetLastError();
+}
+
 template <int VB>
 cudaError_t launch_state(const ChunkArgs& a, int NC) {
     using L = StateLayout<VB>;
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_state_kernel<VB><<<a.B * a.HV * (VD / VB), STATE_THREADS, L::BYTES, a.stream>>>(
-        static_cast<const unsigned char*>(a.scratch), a.S0, a.T, a.HV, NC, static_cast<bf16*>(a.o), a.S_T, a.status);
-    return cudaGetLastError();
+    // programmatic dependent launch: the state kernel's set-up may overlap the prep kernel's tail;
+    // it waits (griddepcontrol.wait) for the prep grid's completion before reading any record
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.HV * (VD / VB));
+    cfg.blockDim = dim3(STATE_THREADS);
+    cfg.dynamicSmemBytes = L::BYTES;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk_state_kernel<VB>, static_cast<const unsigned char*>(a.scratch), a.S0, a.T,
+                              a.HV, NC, static_cast<bf16*>(a.o), a.S_T, a.status);
 }
 }  // namespace
 
 cudaError_t launch_chunk_split(const ChunkArgs& a) {
     const int NC = (a.T + CH - 1) / CH;
-    const long long ntasks = (long long)a.B * a.HV * NC;
+    const int ntasks = a.B * a.HV * NC;  // < 2^30: checked by kda_chunk_fwd_schedule
     int dev = 0, nsm = 148;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepLayout::BYTES);
-    if (e != cudaSuccess) return e;
-    const int grid = (int)(ntasks < nsm ? ntasks : nsm);
-    chunk_prep_kernel<<<grid, TC_THREADS, PrepLayout::BYTES, a.stream>>>(
-        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
-        static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
-        ntasks, a.gate_mode, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status);
-    e = cudaGetLastError();
+    const int grid = ntasks < nsm ? ntasks : nsm;
+    e = a.gate_mode == KDA_GATE_SAFE       ? launch_prep<KDA_GATE_SAFE>(a, NC, ntasks, grid)
+        : a.gate_mode == KDA_GATE_STANDARD ? launch_prep<KDA_GATE_STANDARD>(a, NC, ntasks, grid)
+                                           : launch_prep<KDA_GATE_NONE>(a, NC, ntasks, grid);
     if (e != cudaSuccess) return e;
     // value-block width: enough (pair, block) CTAs to cover the SMs, blocks as wide as that allows
     const long long pairs = (long long)a.B * a.HV;

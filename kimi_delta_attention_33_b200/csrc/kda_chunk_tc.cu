@@ -173,16 +173,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         float gv[32];
         {
             const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
-            float acc = 0.f;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int i = 32 * gh + r;
-                const float x = (i < nn) ? gate_value_fast(__bfloat162float(sG[i * KD + gd]), bias, rate, gate_mode,
-                                                           lower_bound)
-                                         : 0.f;
-                acc += x;
-                gv[r] = acc;
-            }
+            const float acc = gate_rows32(gate_mode, sG + 32 * gh * KD + gd, KD, nn - 32 * gh, bias, rate, lower_bound, gv);
             if (gh == 0) sFnext[gd] = acc;  // scratch: first-half totals
         }
         __syncthreads();  // the g staging has been read: GM becomes Gam
