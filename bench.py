@@ -157,18 +157,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ distributed ---
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU from the torch.distributed.run environment.  The bench uses NCCL; the
+    CPU tests of this plumbing pass backend="gloo" (no device is touched then)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return ws, rank, local
 
 
@@ -179,12 +180,27 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """MAX of a per-rank scalar over all ranks (every rank gets the result)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of a rank's input shard: rank 0 draws the workload's own inputs (seed 1000 + id, as the
+    parity tests do), every other rank an independent shard of the same shape."""
+    return 1000 + w.wid + 7919 * rank
+
+
+def aggregate(units_per_step: int, steps: int, local_total_ms: float, ws: int):
+    """Whole-job throughput under weak scaling: every rank processed units_per_step per step on its
+    own shard; the job took as long as its slowest rank.  Returns (value per second, ms per step)."""
+    total_ms = max_over_ranks(local_total_ms, ws)
+    return ws * units_per_step * steps / (total_ms / 1e3), total_ms / steps
 
 
 # ----------------------------------------------------------------------------- our arm -------
@@ -201,7 +217,7 @@ def run_ours(args, ws, rank, local):
     if args.B is not None:
         w = w.scaled(B=args.B)
     torch.manual_seed(0)
-    x = make_inputs(w, seed=1000 + w.wid + 7919 * rank, device=str(dev))
+    x = make_inputs(w, seed=rank_seed(w, rank), device=str(dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm_peak, _, peak_kind = measured_peaks()
     stream = torch.cuda.current_stream(dev)
@@ -257,9 +273,7 @@ def run_ours(args, ws, rank, local):
         torch.cuda.synchronize(dev)
         barrier(ws)
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(sum(step_ms), ws)
-    ms_per_step = total_ms / args.steps
-    value = ws * units_per_step * args.steps / (total_ms / 1e3)
+    value, ms_per_step = aggregate(units_per_step, args.steps, sum(step_ms), ws)
     # one library call per step: its kernels (one, or the two of the two-pass schedule) are timed
     # together, since the algorithmic bytes belong to the pass as a whole
     kern_s = (sum(step_ms) / args.steps) / 1e3
