@@ -81,6 +81,28 @@ __device__ __forceinline__ float gate_rows32_to(const __nv_bfloat16* col, int st
     return acc;
 }
 
+// The same for 16 rows (CTAs with four threads per key channel).
+template <int MODE, typename Idx>
+__device__ __forceinline__ float gate_rows16_to(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
+                                                float lower_bound, float* dst, Idx idx) {
+    float acc = 0.f;
+#pragma unroll
+    for (int r0 = 0; r0 < 16; r0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const float gr = __bfloat162float(col[(r0 + r) * stride]);
+            x[r] = (r0 + r < nn) ? gate_value_fast(gr, bias, rate, MODE, lower_bound) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            acc += x[r];
+            dst[idx(r0 + r)] = acc;
+        }
+    }
+    return acc;
+}
+
 __device__ __forceinline__ float gate_rows32(int mode, const __nv_bfloat16* col, int stride, int nn, float bias,
                                              float rate, float lower_bound, float (&gv)[32]) {
     if (mode == KDA_GATE_SAFE) return gate_rows32<KDA_GATE_SAFE>(col, stride, nn, bias, rate, lower_bound, gv);
@@ -94,14 +116,14 @@ __device__ __forceinline__ float bf16_bits_to_f32(unsigned short u) { return __u
 // stored with row pitch RP: every diagonal block of size 2 HS, [[Ta, 0], [C, Td]], whose diagonal
 // sub-blocks already hold their inverses, gets its lower-left block -Td C Ta (Ta, Td with implicit
 // unit diagonals).  X = C Ta goes through the scratch sX.
-template <int HS>
+template <int HS, int NT = TC_THREADS>
 __device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid) {
     constexpr int CNT = (CH / (2 * HS)) * HS * HS;
-    constexpr int ITERS = (CNT + TC_THREADS - 1) / TC_THREADS;
+    constexpr int ITERS = (CNT + NT - 1) / NT;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-        const int e = tid + TC_THREADS * it;
-        if (CNT % TC_THREADS == 0 || e < CNT) {
+        const int e = tid + NT * it;
+        if (CNT % NT == 0 || e < CNT) {
             const int c = e % HS, r = (e / HS) % HS, base = (e / (HS * HS)) * 2 * HS;
             const float* Crow = sRT + (base + HS + r) * RP + base;
             float acc = Crow[c];
@@ -114,8 +136,8 @@ __device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid)
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-        const int e = tid + TC_THREADS * it;
-        if (CNT % TC_THREADS == 0 || e < CNT) {
+        const int e = tid + NT * it;
+        if (CNT % NT == 0 || e < CNT) {
             const int c = e % HS, r = (e / HS) % HS, blk = e / (HS * HS), base = blk * 2 * HS;
             const float* Drow = sRT + (base + HS + r) * RP + base + HS;
             const float* Xb = sX + blk * HS * HS;
@@ -134,7 +156,8 @@ __device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid)
 // Step 16 -> 32 (two blocks, at 0 and 32): warp w serves block w / 4 and rows 4 (w % 4) .. + 3 of its
 // 16 x 16 lower-left block; lane = column (lane % 16) and row pair (lane / 16).
 __device__ __forceinline__ void tri_inverse_step16(float* sRT, float* sX, int tid) {
-    const int w = tid >> 5, lane = tid & 31;
+    const bool active = tid < TC_THREADS;  // larger CTAs: threads past the first 256 only join the barriers
+    const int w = (tid >> 5) & 7, lane = tid & 31;
     const int base = 32 * (w >> 2), c = lane & 15;
     const int r0 = 4 * (w & 3) + 2 * (lane >> 4);  // rows r0, r0 + 1 of the 16 x 16 lower-left block
     float acc[2];
@@ -151,8 +174,10 @@ __device__ __forceinline__ void tri_inverse_step16(float* sRT, float* sX, int ti
             acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
         }
     }
+    if (active) {
 #pragma unroll
-    for (int x = 0; x < 2; ++x) sX[(w >> 2) * 256 + (r0 + x) * 16 + c] = acc[x];
+        for (int x = 0; x < 2; ++x) sX[(w >> 2) * 256 + (r0 + x) * 16 + c] = acc[x];
+    }
     __syncthreads();
     const float* Xb = sX + (w >> 2) * 256;
 #pragma unroll
@@ -170,14 +195,17 @@ __device__ __forceinline__ void tri_inverse_step16(float* sRT, float* sX, int ti
                       (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
         }
     }
+    if (active) {
 #pragma unroll
-    for (int x = 0; x < 2; ++x) sRT[(base + 16 + r0 + x) * RP + base + c] = -acc[x];
+        for (int x = 0; x < 2; ++x) sRT[(base + 16 + r0 + x) * RP + base + c] = -acc[x];
+    }
     __syncthreads();
 }
 
 // Step 32 -> 64 (one block): warp w serves rows 4 w + {0..3}, lane = column.
 __device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int tid) {
-    const int w = tid >> 5, c = tid & 31, r0 = 4 * w;
+    const bool active = tid < TC_THREADS;  // larger CTAs: threads past the first 256 only join the barriers
+    const int w = (tid >> 5) & 7, c = tid & 31, r0 = 4 * w;
     float acc[4];
 #pragma unroll
     for (int x = 0; x < 4; ++x) acc[x] = sRT[(32 + r0 + x) * RP + c];
@@ -192,8 +220,10 @@ __device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int ti
             acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
         }
     }
+    if (active) {
 #pragma unroll
-    for (int x = 0; x < 4; ++x) sX[(r0 + x) * 32 + c] = acc[x];
+        for (int x = 0; x < 4; ++x) sX[(r0 + x) * 32 + c] = acc[x];
+    }
     __syncthreads();
 #pragma unroll
     for (int x = 0; x < 4; ++x) acc[x] = sX[(r0 + x) * 32 + c];
@@ -211,8 +241,10 @@ __device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int ti
                       (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
         }
     }
+    if (active) {
 #pragma unroll
-    for (int x = 0; x < 4; ++x) sRT[(32 + r0 + x) * RP + c] = -acc[x];
+        for (int x = 0; x < 4; ++x) sRT[(32 + r0 + x) * RP + c] = -acc[x];
+    }
     __syncthreads();
 }
 

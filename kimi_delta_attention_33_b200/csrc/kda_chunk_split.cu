@@ -60,8 +60,8 @@ struct PrepLayout {
     static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
     static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)
     static constexpr uint32_t VEC = 229376;
-    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024;
-    static constexpr uint32_t MBAR = VEC + 1280, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8, FLAG = TBASE + 4;
+    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, SC2 = VEC + 1024, BETA = VEC + 1536;
+    static constexpr uint32_t MBAR = VEC + 1792, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8, FLAG = TBASE + 4;
     static constexpr uint32_t BYTES = FLAG + 4;
     static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
@@ -88,6 +88,7 @@ struct StateLayout {
 };
 
 constexpr int STATE_THREADS = 256;
+constexpr int PREP_THREADS = 512;
 
 struct Task {
     int pair, c, b, hv, h, nn;
@@ -112,17 +113,18 @@ __device__ __forceinline__ Task make_task(int task, int T, int H, int HV, int NC
 // Pass 1: chunk-local work for every chunk.
 // ---------------------------------------------------------------------------------------------
 template <int MODE>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(PREP_THREADS, 1)
 chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                   const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, int T, int H, int HV, int NC, int ntasks,
                   float lower_bound, float scale, unsigned char* __restrict__ rec_base,
                   unsigned int* __restrict__ status) {
     using L = PrepLayout;
-    constexpr int gate_mode = MODE;
+    constexpr int NT = PREP_THREADS;
     extern __shared__ __align__(1024) unsigned char smem[];
     float* sRho = reinterpret_cast<float*>(smem + L::RHO);
     float* sSig = reinterpret_cast<float*>(smem + L::SIG);
+    float* sSc2 = reinterpret_cast<float*>(smem + L::SC2);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
@@ -133,7 +135,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     const uint32_t mbar = s_base + L::MBAR, mbar_in = s_base + L::MBAR_IN;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column quarter
+    const int rot = lane >> 2;                // store rotation (see rotate_groups8)
     const size_t qk_row = (size_t)H * KD, v_row = (size_t)HV * VD, g_row = (size_t)HV * KD;
 
     // the state kernel that follows may start its set-up as SMs free up; it waits for this grid's
@@ -151,15 +154,16 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     bool aborted = false, in_pending = false;
 
     // Inputs of one chunk: g and v tiles into the staging half of X1 by bulk copies, one 256-byte row
-    // per thread, completing on mbar_in (rows past T are zeroed by plain stores instead); q, k, beta,
-    // this head's A_log and this thread's dt_bias entry into registers.
-    uint4 qr[4], kr[4];
-    uint32_t beta_bits;  // raw bf16 bits of this thread's beta (row tid), converted where used
+    // per thread of the first 128, completing on mbar_in (rows past T are zeroed by plain stores
+    // instead); q, k, beta, this head's A_log and this thread's dt_bias entry into registers.
+    // q / k units: u = tid + NT * it covers row i = 8 (u / 128) + u % 8 and key group d8 = (u / 8) % 16.
+    uint4 qr[2], kr[2];
+    uint32_t beta_bits = 0;  // raw bf16 bits of beta for row tid (tid < 64), converted where used
     float alog_in = 0.f, bias_in = 0.f;
     auto load_inputs = [&](const Task& tk) {
-        const int i = tid & (CH - 1), which = tid >> 6;  // which: 0 g, 1 v (threads 128-255: none)
-        if (tid == 0) mbar_expect_tx(mbar_in, 2u * 256u * (uint32_t)tk.nn);
-        if (which < 2) {
+        if (tid < 2 * CH) {
+            const int i = tid & (CH - 1), which = tid >> 6;  // which: 0 g, 1 v
+            if (tid == 0) mbar_expect_tx(mbar_in, 2u * 256u * (uint32_t)tk.nn);
             const uint32_t dst = s_base + L::X1 + which * 16384 + i * 256;
             if (i < tk.nn) {
                 const bf16* src = which == 0 ? g + (tk.tk0 + i) * g_row + (size_t)tk.hv * KD
@@ -173,8 +177,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
         in_pending = true;
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
+        for (int it = 0; it < 2; ++it) {
+            const int u = tid + NT * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
             qr[it] = make_uint4(0u, 0u, 0u, 0u);
             kr[it] = qr[it];
@@ -185,7 +189,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
         beta_bits = (tid < tk.nn) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(beta) + (tk.tk0 + tid) * HV + tk.hv)
                                   : 0u;
-        if (gate_mode != KDA_GATE_NONE) {
+        if (MODE != KDA_GATE_NONE) {
             alog_in = __ldg(A_log + tk.hv);
             bias_in = dt_bias != nullptr ? __ldg(dt_bias + tk.hv * KD + (tid & (KD - 1))) : 0.f;
         }
@@ -197,23 +201,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     for (; task < ntasks && !aborted; task += gridDim.x) {
         const Task tk = make_task(task, T, H, HV, NC);
         unsigned char* rec = rec_base + (size_t)task * Rec::BYTES;
-        const float rate = (gate_mode != KDA_GATE_NONE) ? expf(alog_in) : 0.0f;
+        const float rate = (MODE != KDA_GATE_NONE) ? expf(alog_in) : 0.0f;
 
-        // the next chunk of this CTA: bring its q, k, v and g rows into L2 (one 256-byte row per thread)
-        if (task + gridDim.x < ntasks) {
-            const Task nx = make_task(task + gridDim.x, T, H, HV, NC);
-            const int i = tid & (CH - 1), which = tid >> 6;
-            if (i < nx.nn) {
-                const size_t tok = nx.tk0 + i;
-                const bf16* src = which == 0   ? q + tok * qk_row + (size_t)nx.h * KD
-                                  : which == 1 ? k + tok * qk_row + (size_t)nx.h * KD
-                                  : which == 2 ? v + tok * v_row + (size_t)nx.hv * VD
-                                               : g + tok * g_row + (size_t)nx.hv * KD;
-                bulk_prefetch_l2(src, 256);
-            }
-        }
-
-        // ---- gate and inclusive in-chunk cumulative log decay (two threads per key channel) ----
+        // ---- gate and inclusive in-chunk cumulative log decay (four threads per key channel) ----
         bool slow;
         {
             const int nn = tk.nn, mr = (nn - 1) >> 1;
@@ -222,15 +212,19 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             phase_in ^= 1u;
             in_pending = false;
             if (tid < CH) sBeta[tid] = __uint_as_float(beta_bits << 16);
-            const int gd = tid & (KD - 1), gh = tid >> 7;
-            const float acc = gate_rows32_to<MODE>(sG + 32 * gh * KD + gd, KD, nn - 32 * gh, bias_in, rate, lower_bound,
-                                                   sGam, [&](int r) { return gidx(32 * gh + r, gd); });
-            if (gh == 0) sSig[gd] = acc;  // scratch: first-half totals
+            const int gd = tid & (KD - 1), gq = tid >> 7;  // channel, quarter of the rows (16 each)
+            const float acc = gate_rows16_to<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias_in, rate, lower_bound,
+                                                   sGam, [&](int r) { return gidx(16 * gq + r, gd); });
+            // totals of quarters 0-2 go to scratch; later quarters add the ones before them
+            float* part = gq == 0 ? sRho : gq == 1 ? sSig : sSc2;
+            if (gq < 3) part[gd] = acc;
             __syncthreads();
-            if (gh == 1) {  // second half: add the first half's total
-                const float off = sSig[gd];
+            if (gq > 0) {
+                float off = sRho[gd];
+                if (gq > 1) off += sSig[gd];
+                if (gq > 2) off += sSc2[gd];
 #pragma unroll 4
-                for (int r = 32; r < 64; ++r) sGam[gidx(r, gd)] += off;
+                for (int r = 0; r < 16; ++r) sGam[gidx(16 * gq + r, gd)] += off;
             }
             __syncthreads();
             if (tid < KD) {
@@ -258,14 +252,14 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
         }
 
-        // ---- V^T into VT from the staged v tile ----------------------------------------------------
+        // ---- V^T into VT from the staged v tile (value column vc, token quads q0 + 4 x) ---------------
         {
             const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::X1 + 16384);
-            const int vc = tid & (VD - 1), jq0 = tid >> 7;
-            uint32_t vv[16];
+            const int vc = tid & (VD - 1), q0 = tid >> 7;
+            uint32_t vv[8];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const int j = 4 * (jq0 + 2 * x);
+            for (int x = 0; x < 4; ++x) {
+                const int j = 4 * (q0 + 4 * x);
                 vv[2 * x] = (uint32_t)sVs[(j + 0) * VD + vc] | ((uint32_t)sVs[(j + 1) * VD + vc] << 16);
                 vv[2 * x + 1] = (uint32_t)sVs[(j + 2) * VD + vc] | ((uint32_t)sVs[(j + 3) * VD + vc] << 16);
             }
@@ -274,8 +268,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (tid == 0) bulk_wait_read();
             __syncthreads();
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const int j = 4 * (jq0 + 2 * x);
+            for (int x = 0; x < 4; ++x) {
+                const int j = 4 * (q0 + 4 * x);
                 *reinterpret_cast<uint4*>(smem + L::VT + cm_off(vc, j, CH)) =
                     make_uint4(to_tf32(__uint_as_float(vv[2 * x] << 16)), to_tf32(__uint_as_float(vv[2 * x] & 0xFFFF0000u)),
                                to_tf32(__uint_as_float(vv[2 * x + 1] << 16)),
@@ -284,10 +278,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
 
         // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK, Kchk^T -> KA rows 0-127 -----------------------
-        uint32_t kh[4][8];  // tf32 bits of -Khat, kept for Khat^T once Gam is no longer needed
+        uint32_t kh[2][8];  // tf32 bits of -Khat (rotated), kept for Khat^T once Gam is no longer needed
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
+        for (int it = 0; it < 2; ++it) {
+            const int u = tid + NT * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
             float qf[8], kf[8], gf[8], rf[8], sf[8];
             bf16x8_to_f32(qr[it], qf);
@@ -317,7 +311,6 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                     make_uint4(wc_[4 * hh], wc_[4 * hh + 1], wc_[4 * hh + 2], wc_[4 * hh + 3]);
             }
             // Kchk^T: lanes that share a bank (same i & 3) take different d of their group of 8
-            const int rot = lane >> 2;
             rotate_groups8(wc_, rot);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
@@ -330,10 +323,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         // Khat^T into GM (B rows 0-127 of M7) once Gam is no longer read
         auto write_khat_t = [&]() {
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int u = tid + TC_THREADS * it;
+            for (int it = 0; it < 2; ++it) {
+                const int u = tid + NT * it;
                 const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
-                const int rot = lane >> 2;  // kh[it] holds its group of 8 rotated by rot
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
                     *reinterpret_cast<uint32_t*>(smem + L::GM + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) =
@@ -341,7 +333,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
         };
 
-        // ---- A -> KA rows 128-191, R -> CK region (pitch RP) -------------------------------------
+        // ---- A -> record (KA rows 128-191), R -> CK region (pitch RP) ----------------------------
         if (!slow) {
             if (tid == 0) {
                 gemm_tf32(tmem, s_base + L::X1, KD / 4 * 128, s_base + L::CK, KD / 4 * 128, idesc_tf32(128, 64), KD / 8,
@@ -355,23 +347,27 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             phase ^= 1u;
             // X1 rows 0-63 are free: stage the next chunk of this CTA during the rest of this one
             if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
-            uint32_t raw[32];
-            tmem_ld32(taddr(tmem, 32 * wq, 32 * wh), raw);
+            uint32_t raw[16];
+            tmem_ld16(taddr(tmem, 32 * wq, 16 * wc), raw);
             tmem_wait_ld();
             if (wq < 2) {  // rows 0-63 of D1 hold -Khat Kchk^T
                 const int i = 32 * wq + lane;
                 const float bi = -sBeta[i];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = 32 * wh + jj;
-                    sRT[i * RP + j] = (j < i) ? bi * __uint_as_float(raw[jj]) : 0.f;
+                for (int jj = 0; jj < 16; jj += 4) {
+                    const int j = 16 * wc + jj;
+                    *reinterpret_cast<float4*>(sRT + i * RP + j) =
+                        make_float4(j + 0 < i ? bi * __uint_as_float(raw[jj + 0]) : 0.f,
+                                    j + 1 < i ? bi * __uint_as_float(raw[jj + 1]) : 0.f,
+                                    j + 2 < i ? bi * __uint_as_float(raw[jj + 2]) : 0.f,
+                                    j + 3 < i ? bi * __uint_as_float(raw[jj + 3]) : 0.f);
                 }
             } else {  // rows 64-127 hold A (unmasked): masked, tf32, straight into the record
                 const int i = 32 * (wq - 2) + lane;
                 unsigned char* ra = rec + Rec::KA + 32768;
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 4) {
-                    const int j = 32 * wh + jj;
+                for (int jj = 0; jj < 16; jj += 4) {
+                    const int j = 16 * wc + jj;
                     uint4 w4;
                     w4.x = to_tf32(j + 0 <= i ? __uint_as_float(raw[jj + 0]) : 0.f);
                     w4.y = to_tf32(j + 1 <= i ? __uint_as_float(raw[jj + 1]) : 0.f);
@@ -382,11 +378,11 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
         } else {
             if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
-            // exact decay factors: 4096 (i, j) cells, 16 per thread; Gam is still in GM
-            float av[16], rr[16];
+            // exact decay factors: 4096 (i, j) cells, 8 per thread; Gam is still in GM
+            float av[8], rr[8];
 #pragma unroll 1
-            for (int x = 0; x < 16; ++x) {
-                const int p = tid + TC_THREADS * x;
+            for (int x = 0; x < 8; ++x) {
+                const int p = tid + NT * x;
                 const int i = p >> 6, j = p & 63;
                 float a = 0.f, r = 0.f;
                 if (j <= i && i < tk.nn) {
@@ -405,8 +401,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
             __syncthreads();  // Gam fully read: GM becomes Khat^T
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                const int p = tid + TC_THREADS * x;
+            for (int x = 0; x < 8; ++x) {
+                const int p = tid + NT * x;
                 const int i = p >> 6, j = p & 63;
                 *reinterpret_cast<uint32_t*>(rec + Rec::KA + 32768 + cm_off(i, j, CH)) = to_tf32(av[x]);
                 sRT[i * RP + j] = rr[x];
@@ -416,15 +412,15 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         __syncthreads();
 
         // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 and 192-255 ----------
-        tri_inverse_step<1>(sRT, sX, tid);
-        tri_inverse_step<2>(sRT, sX, tid);
-        tri_inverse_step<4>(sRT, sX, tid);
-        tri_inverse_step<8>(sRT, sX, tid);
+        tri_inverse_step<1, NT>(sRT, sX, tid);
+        tri_inverse_step<2, NT>(sRT, sX, tid);
+        tri_inverse_step<4, NT>(sRT, sX, tid);
+        tri_inverse_step<8, NT>(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
         tri_inverse_step32(sRT, sX, tid);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int u = tid + TC_THREADS * x;
+        for (int x = 0; x < 2; ++x) {
+            const int u = tid + NT * x;
             const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
             uint32_t w[4];
             const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
@@ -455,31 +451,22 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             phase ^= 1u;
         }
         {
-            // lane quarters 0-1 read W (rows 0-63), quarters 2-3 read U (rows 64-127); wh picks 64 columns
+            // lane quarters 0-1 read W (rows 0-63), quarters 2-3 read U (rows 64-127); wc picks 32 columns
             const int i = 32 * (wq & 1) + lane;
-            const int col = (wq < 2 ? 0 : 128) + 64 * wh;
-            uint32_t r0[32], r1[32];
-            tmem_ld32(taddr(tmem, 32 * wq, col), r0);
-            tmem_ld32(taddr(tmem, 32 * wq, col + 32), r1);
+            uint32_t r0[32];
+            tmem_ld32(taddr(tmem, 32 * wq, (wq < 2 ? 0 : 128) + 32 * wc), r0);
             tmem_wait_ld();
             if (wq < 2) {  // W -> record WQ rows 0-63 (tf32, operand tiling)
                 unsigned char* rw = rec + Rec::WQ;
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    *reinterpret_cast<uint4*>(rw + cm_off(i, 64 * wh + 4 * c4, KD)) =
+                for (int c4 = 0; c4 < 8; ++c4)
+                    *reinterpret_cast<uint4*>(rw + cm_off(i, 32 * wc + 4 * c4, KD)) =
                         make_uint4(to_tf32(__uint_as_float(r0[4 * c4])), to_tf32(__uint_as_float(r0[4 * c4 + 1])),
                                    to_tf32(__uint_as_float(r0[4 * c4 + 2])), to_tf32(__uint_as_float(r0[4 * c4 + 3])));
-                    *reinterpret_cast<uint4*>(rw + cm_off(i, 64 * wh + 32 + 4 * c4, KD)) =
-                        make_uint4(to_tf32(__uint_as_float(r1[4 * c4])), to_tf32(__uint_as_float(r1[4 * c4 + 1])),
-                                   to_tf32(__uint_as_float(r1[4 * c4 + 2])), to_tf32(__uint_as_float(r1[4 * c4 + 3])));
-                }
             } else {  // U^T (fp32, row = value column) -> CK region, free once Tb was built
                 float* ut = reinterpret_cast<float*>(smem + L::CK);
 #pragma unroll
-                for (int cc = 0; cc < 32; ++cc) {
-                    ut[(64 * wh + cc) * CH + i] = __uint_as_float(r0[cc]);
-                    ut[(64 * wh + 32 + cc) * CH + i] = __uint_as_float(r1[cc]);
-                }
+                for (int cc = 0; cc < 32; ++cc) ut[(32 * wc + cc) * CH + i] = __uint_as_float(r0[cc]);
             }
         }
         fence_proxy_async();
@@ -743,7 +730,7 @@ cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepLayout::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_prep_kernel<MODE><<<grid, TC_THREADS, PrepLayout::BYTES, a.stream>>>(
+    chunk_prep_kernel<MODE><<<grid, PREP_THREADS, PrepLayout::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
         ntasks, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status);
