@@ -151,6 +151,49 @@ __device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid)
     __syncthreads();
 }
 
+// The doubling steps with blocks of 2, 4, 8 and 16 rows never cross a 16 x 16 diagonal block, so
+// one warp can take one such block through all four with warp-level syncs only: warp w < 4 inverts
+// the diagonal block at rows / columns 16 w .. 16 w + 15 (scratch: 64 floats of sX per warp).
+template <int HS>
+__device__ __forceinline__ void tri_inverse_diag16_step(float* sRT, float* sXw, int b16, int lane) {
+    constexpr int CNT = 8 * HS;  // entries of the HS x HS lower-left blocks inside one 16 x 16 block
+#pragma unroll
+    for (int e = lane; e < CNT; e += 32) {  // X = C Ta
+        const int c = e % HS, r = (e / HS) % HS, base = b16 + (e / (HS * HS)) * 2 * HS;
+        const float* Crow = sRT + (base + HS + r) * RP + base;
+        float acc = Crow[c];
+#pragma unroll
+        for (int m = 1; m < HS; ++m)
+            if (m > c) acc += Crow[m] * sRT[(base + m) * RP + base + c];
+        sXw[e] = acc;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = lane; e < CNT; e += 32) {  // C <- -Td X
+        const int c = e % HS, r = (e / HS) % HS, blk = e / (HS * HS), base = b16 + blk * 2 * HS;
+        const float* Drow = sRT + (base + HS + r) * RP + base + HS;
+        const float* Xb = sXw + blk * HS * HS;
+        float acc = Xb[r * HS + c];
+#pragma unroll
+        for (int m = 0; m < HS - 1; ++m)
+            if (m < r) acc += Drow[m] * Xb[m * HS + c];
+        sRT[(base + HS + r) * RP + base + c] = -acc;
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ void tri_inverse_diag16(float* sRT, float* sX, int tid) {
+    const int w = tid >> 5, lane = tid & 31;
+    if (w < 4) {
+        float* sXw = sX + 64 * w;
+        tri_inverse_diag16_step<1>(sRT, sXw, 16 * w, lane);
+        tri_inverse_diag16_step<2>(sRT, sXw, 16 * w, lane);
+        tri_inverse_diag16_step<4>(sRT, sXw, 16 * w, lane);
+        tri_inverse_diag16_step<8>(sRT, sXw, 16 * w, lane);
+    }
+    __syncthreads();
+}
+
 // The last two doubling steps with one column per lane and four rows per thread: X = C Ta and the
 // new block -Td X, accumulating over m with loads of four consecutive row entries at a time.
 // Step 16 -> 32 (two blocks, at 0 and 32): warp w serves block w / 4 and rows 4 (w % 4) .. + 3 of its

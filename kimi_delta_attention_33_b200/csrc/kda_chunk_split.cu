@@ -412,10 +412,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         __syncthreads();
 
         // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 and 192-255 ----------
-        tri_inverse_step<1, NT>(sRT, sX, tid);
-        tri_inverse_step<2, NT>(sRT, sX, tid);
-        tri_inverse_step<4, NT>(sRT, sX, tid);
-        tri_inverse_step<8, NT>(sRT, sX, tid);
+        tri_inverse_diag16(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
         tri_inverse_step32(sRT, sX, tid);
 #pragma unroll

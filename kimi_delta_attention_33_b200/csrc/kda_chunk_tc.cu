@@ -348,10 +348,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         __syncthreads();
 
         // ---- P6: T = (I + R)^{-1}, in place over R, by six doubling steps (block sizes 2 .. 64) --
-        tri_inverse_step<1>(sRT, sX, tid);
-        tri_inverse_step<2>(sRT, sX, tid);
-        tri_inverse_step<4>(sRT, sX, tid);
-        tri_inverse_step<8>(sRT, sX, tid);
+        tri_inverse_diag16(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
         tri_inverse_step32(sRT, sX, tid);
         // Tb = T diag(beta) as tf32 into AT rows 64-127

@@ -153,3 +153,36 @@ def test_in_place_state_two_pass():
     o_ref, S_ref = _ref(w, x)
     assert rel_err(o, o_ref) <= TOL[w.dtype]
     assert rel_err(S, S_ref) <= TOL[w.dtype]
+
+
+# Shapes at the edges of the two-pass schedule's choices: many chunk records per pair (value blocks
+# of 32 columns), many pairs (blocks of 64), and a ragged last chunk across several sequences.
+@pytest.mark.parametrize("B,H,HV,T", [(1, 2, 4, 16384),
+                                      (1, 37, 37, 448),
+                                      (1, 38, 38, 64),
+                                      (3, 2, 6, 700)])
+def test_two_pass_edge_shapes(B, H, HV, T):
+    w = _wl(B=B, T=T, H=H, HV=HV)
+    x = make_inputs(w)
+    o, S = _run(w, to_dev(x), "two_pass")
+    pairs = sample_pairs(B, HV, 3)
+    refs = oracle_pairs(x, w, pairs)
+    o_gpu = torch.stack([o[b, :, hv] for b, hv in pairs]).cpu()
+    S_gpu = torch.stack([S[b, hv] for b, hv in pairs]).cpu()
+    assert rel_err(o_gpu, np.stack([r[0] for r in refs])) <= TOL[w.dtype]
+    assert rel_err(S_gpu, np.stack([r[1] for r in refs])) <= TOL[w.dtype]
+
+
+def test_two_pass_repeated_calls_reuse_workspace():
+    # records left in the workspace by one call must not leak into the next call's results
+    w = _wl(B=2, T=300, H=2, HV=4)
+    ws = _workspace(w, "two_pass")
+    outs = []
+    for seed in (11, 12, 11):
+        xd = to_dev(make_inputs(w, seed=seed))
+        o, S = kda.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"], xd["S0"],
+                             chunk=64, gate_mode=w.gate_mode, lower_bound=w.lower_bound, workspace=ws)
+        kda.read_status(ws)
+        outs.append((o.clone(), S.clone()))
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    assert not torch.equal(outs[0][0], outs[1][0])
