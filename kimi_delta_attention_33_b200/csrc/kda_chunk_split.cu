@@ -24,8 +24,9 @@
 // per chunk, with tf32(S~)^T staged in shared memory as a B operand:
 //   M8   D1 = [W; Qhat] S~                -> W S~ (rows 0-63), Qhat S~ (rows 64-127)
 //   E    = U - W S~  on the CUDA cores, staged as a tf32 B operand
-//   M9   D1[64:] += A E                   -> O
 //   M10  D2 = Kchk^T E                    -> S_c+1 = f (e^sig S_c + D2), in registers
+//   M9   D1[64:] += A E                   -> O  (issued after M10 with its own commit: off the
+//                                             chunk-to-chunk path)
 // Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
 // where shared memory allows.
 #include "kda_chunk64.cuh"
@@ -78,8 +79,8 @@ struct StateLayout {
     static constexpr uint32_t KA_STRIDE = VEC_OFF + 3 * 512;
     static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S~^T [VB][128]   (B of M8)
     static constexpr uint32_t EOP = SOP + VB * 128 * 4;        // tf32 E^T  [VB][64]    (B of M9, M10)
-    static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1]
-    static constexpr uint32_t TBASE = MBAR + 32;
+    static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1], out
+    static constexpr uint32_t TBASE = MBAR + 40;
     static constexpr uint32_t BYTES = TBASE + 16;
     static constexpr uint32_t TMEM_COLS = 2 * VB < 32 ? 32 : 2 * VB;
     static constexpr int D1 = 0, D2 = VB;
@@ -513,7 +514,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     constexpr int HALF = VB / 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t bar_wq = s_base + L::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16;
+    const uint32_t bar_wq = s_base + L::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16, bar_out = bar_wq + 32;
     const int pair = blockIdx.x / NVB, vb0 = (blockIdx.x - pair * NVB) * VB;
     const int b = pair / HV, hv = pair - b * HV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -528,6 +529,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         mbar_init(bar_mma, 1);
         mbar_init(bar_ka0, 1);
         mbar_init(bar_ka0 + 8, 1);
+        mbar_init(bar_out, 1);
     }
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
     cta_sync_tc();
@@ -582,7 +584,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         for (int j = 0; j < HALF; ++j)
             *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
     };
-    uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0;
+    uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0, ph_out = 0;
     bool aborted = false;
     {
         const bool ok = mbar_wait(bar_ka0, 0, WAIT_POLLS);  // chunk 0's KA group holds its vectors
@@ -638,21 +640,36 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         }
         fence_proxy_async();
         cta_sync_tc();
-        // ---- M9: D1[64:] += A E ;  M10: D2 = Kchk^T E -------------------------------------------
+        // ---- M10: D2 = Kchk^T E (the state side), then M9: D1[64:] += A E (the outputs), each with its
+        //      own commit, so that the state update starts after M10 while M9 still runs -------------
         if (tid == 0) {
-            gemm_tf32(tmem + L::D1, ka + 16384, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB),
-                      CH / 8, true);
             gemm_tf32(tmem + L::D2, ka, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
                       false);
             mma_commit(bar_mma);
+            gemm_tf32(tmem + L::D1, ka + 16384, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB),
+                      CH / 8, true);
+            mma_commit(bar_out);
         }
         ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
         fence_after_sync();
         if (!__syncthreads_and(ok)) { aborted = true; break; }
         ph_mma ^= 1u;
-        if (L::NKA == 1 && tid == 0 && c + 1 < NC) load_ka(c + 1, 0);
-        // ---- outputs (rows 64-127 of D1: lane quarters 2, 3) -------------------------------------
-        if (wq >= 2) {
+        // ---- state: S = f (e^sig S + D2) --------------------------------------------------------
+        {
+            uint32_t r[HALF];
+            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D2 + c0), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < HALF; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
+        }
+        // ---- outputs (rows 64-127 of D1: lane quarters 2, 3), once M9 is done; thread 0 waits for it
+        //      too before a KA buffer M9 reads is refilled -----------------------------------------
+        bool ok_out = true;
+        if (wq >= 2 || tid == 0) {
+            ok_out = mbar_wait(bar_out, ph_out, WAIT_POLLS);
+            fence_after_sync();
+        }
+        if (wq >= 2 && ok_out) {
             const int i = d - 64;
             uint32_t r[HALF];
             tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
@@ -674,25 +691,22 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
                 }
             }
         }
-        // ---- state: S = f (e^sig S + D2); S~ of the next chunk ----------------------------------
-        {
-            uint32_t r[HALF];
-            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D2 + c0), r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < HALF; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
-        }
+        if (L::NKA == 1 && tid == 0 && ok_out && c + 1 < NC) load_ka(c + 1, 0);
+        // ---- S~ of the next chunk ---------------------------------------------------------------
         if (c + 1 < NC) {
             if (L::NKA == 2) {  // the next chunk's KA group (loaded a chunk ago) holds its e^rho
                 const int nb = buf ^ 1;
-                const bool okn = mbar_wait(bar_ka0 + 8 * nb, (ph_ka >> nb) & 1u, WAIT_POLLS);
+                const bool okn = mbar_wait(bar_ka0 + 8 * nb, (ph_ka >> nb) & 1u, WAIT_POLLS) && ok_out;
                 if (!__syncthreads_and(okn)) { aborted = true; break; }
                 er_n = vec(nb, 0);
             }
             write_sop(er_n);
         }
         fence_proxy_async();
-        cta_sync_tc();
+        fence_before_sync();
+        if (!__syncthreads_and(ok_out)) { aborted = true; break; }
+        fence_after_sync();
+        ph_out ^= 1u;
         if (L::NKA == 2 && tid == 0 && c + 2 < NC) load_ka(c + 2, buf);
     }
 
@@ -704,6 +718,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             for (int bb = 0; bb < L::NKA; ++bb)
                 if (pending & (2u << bb)) mbar_wait(bar_ka0 + 8 * bb, (ph_ka >> bb) & 1u, WAIT_POLLS);
             mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
+            mbar_wait(bar_out, ph_out, WAIT_POLLS);
         }
     } else if (S_T) {
 #pragma unroll

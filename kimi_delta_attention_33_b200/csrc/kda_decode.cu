@@ -6,6 +6,9 @@
 // S in R^{K x V} (fp32, key-major, 64 KiB at K = V = 128) and moves it through registers
 // exactly once: every thread loads its rows of S with 128-bit streaming loads, and both
 // reductions over K (p = k . S_dec and u = q . S_dec) come out of that single read.
+// Value columns are independent in every step, so a state may be split into NSPLIT column
+// blocks owned by separate CTAs (smaller CTAs, more of them resident per SM); each recomputes
+// the per-token vectors and q . k it needs.
 // The read-out uses q . S_t = q . S_dec + beta (q . k) r, which follows from steps 3-4 of
 // the recurrence (KDA notes, "KDA 递归核心", §逐步公式), so S_t never has to be re-read.
 #include "kda_common.cuh"
@@ -13,34 +16,36 @@
 
 namespace kda {
 
-template <int K, int V>
+template <int K, int V, int NSPLIT = 1>
 struct DecodeShape {
-    static constexpr int NT = (K * V / 4 < 256) ? K * V / 4 : 256;  // threads per CTA
-    static constexpr int TPR = V / 4;                                  // threads per state row
+    static constexpr int VC = V / NSPLIT;                              // value columns per CTA
+    static constexpr int NT = (K * VC / 4 < 256) ? K * VC / 4 : 256;  // threads per CTA
+    static constexpr int TPR = VC / 4;                                 // threads per state row
     static constexpr int RPP = NT / TPR;                               // rows per pass
     static constexpr int R = K / RPP;                                  // rows per thread
-    static_assert(R >= 1 && RPP * R == K, "decode shape");
+    static_assert(R >= 1 && RPP * R == K && VC * NSPLIT == V, "decode shape");
 };
 
-template <typename T, int K, int V>
-__global__ void __launch_bounds__(DecodeShape<K, V>::NT)
+template <typename T, int K, int V, int NSPLIT = 1>
+__global__ void __launch_bounds__(DecodeShape<K, V, NSPLIT>::NT)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const T* __restrict__ g, const T* __restrict__ beta, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, int H, int HV, int gate_mode, float lower_bound,
                    float scale, float* __restrict__ S, T* __restrict__ o) {
-    using Sh = DecodeShape<K, V>;
-    constexpr int NT = Sh::NT, TPR = Sh::TPR, RPP = Sh::RPP, R = Sh::R;
+    using Sh = DecodeShape<K, V, NSPLIT>;
+    constexpr int NT = Sh::NT, TPR = Sh::TPR, RPP = Sh::RPP, R = Sh::R, VC = Sh::VC;
     __shared__ float s_q[K], s_k[K], s_a[K];
-    __shared__ float s_p[RPP][V], s_u[RPP][V];
-    __shared__ float s_r[V];
+    __shared__ float s_p[RPP][VC], s_u[RPP][VC];
+    __shared__ float s_r[VC];
     __shared__ float s_qk;
 
-    const int pair = blockIdx.x;  // b * HV + hv
+    const int pair = blockIdx.x / NSPLIT;  // b * HV + hv
+    const int v0 = (blockIdx.x - pair * NSPLIT) * VC;
     const int b = pair / HV, hv = pair - b * HV;
     const int h = hv / (HV / H);
     const int tid = threadIdx.x;
     const int cg = tid % TPR, rg = tid / TPR;
-    float* Sp = S + (size_t)pair * K * V;
+    float* Sp = S + (size_t)pair * K * V + v0;
 
     // 1. stream this thread's rows of S in first, so the loads are all in flight together
     float4 st[R];
@@ -80,13 +85,13 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 
     // 4. finish the reductions per value column: residual r (step 2) and the read-out (step 4)
     const float bt = to_f32(beta[pair]);
-    if (tid < V) {
+    if (tid < VC) {
         float pp = 0.0f, uu = 0.0f;
 #pragma unroll
         for (int j = 0; j < RPP; ++j) { pp += s_p[j][tid]; uu += s_u[j][tid]; }
-        const float r = to_f32(v[(size_t)pair * V + tid]) - pp;
+        const float r = to_f32(v[(size_t)pair * V + v0 + tid]) - pp;
         s_r[tid] = r;
-        o[(size_t)pair * V + tid] = from_f32<T>(scale * (uu + bt * s_qk * r));
+        o[(size_t)pair * V + v0 + tid] = from_f32<T>(scale * (uu + bt * s_qk * r));
     }
     __syncthreads();
 
@@ -101,10 +106,10 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     }
 }
 
-template <typename T, int K, int V>
+template <typename T, int K, int V, int NSPLIT = 1>
 static cudaError_t launch_decode(const DecodeArgs& a) {
-    using Sh = DecodeShape<K, V>;
-    decode_step_kernel<T, K, V><<<a.B * a.HV, Sh::NT, 0, a.stream>>>(
+    using Sh = DecodeShape<K, V, NSPLIT>;
+    decode_step_kernel<T, K, V, NSPLIT><<<a.B * a.HV * NSPLIT, Sh::NT, 0, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
         static_cast<const T*>(a.g), static_cast<const T*>(a.beta), a.A_log, a.dt_bias, a.H, a.HV, a.gate_mode,
         a.lower_bound, a.scale, a.S, static_cast<T*>(a.o));
@@ -117,7 +122,9 @@ static cudaError_t dispatch_v(const DecodeArgs& a) {
         case 16: return launch_decode<T, K, 16>(a);
         case 32: return launch_decode<T, K, 32>(a);
         case 64: return launch_decode<T, K, 64>(a);
-        case 128: return launch_decode<T, K, 128>(a);
+        // 128 value columns: two CTAs per state (32 KiB each) -- about 7 % more bandwidth than one
+        // 64 KiB CTA per state on B256 H32 K=V=128, since more of the smaller CTAs stay resident
+        case 128: return launch_decode<T, K, 128, 2>(a);
     }
     return cudaErrorInvalidValue;
 }
