@@ -103,6 +103,32 @@ __device__ __forceinline__ float gate_rows16_to(const __nv_bfloat16* col, int st
     return acc;
 }
 
+// Gate values of one key channel for 16 consecutive rows as their running sum in registers.
+template <int MODE>
+__device__ __forceinline__ float gate_rows16_regs(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
+                                                  float lower_bound, float (&gv)[16]) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const float gr = __bfloat162float(col[r * stride]);
+        gv[r] = (r < nn) ? gate_value_fast(gr, bias, rate, MODE, lower_bound) : 0.f;
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        acc += gv[r];
+        gv[r] = acc;
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float gate_rows16_regs(int mode, const __nv_bfloat16* col, int stride, int nn, float bias,
+                                                  float rate, float lower_bound, float (&gv)[16]) {
+    if (mode == KDA_GATE_SAFE) return gate_rows16_regs<KDA_GATE_SAFE>(col, stride, nn, bias, rate, lower_bound, gv);
+    if (mode == KDA_GATE_STANDARD)
+        return gate_rows16_regs<KDA_GATE_STANDARD>(col, stride, nn, bias, rate, lower_bound, gv);
+    return gate_rows16_regs<KDA_GATE_NONE>(col, stride, nn, bias, rate, lower_bound, gv);
+}
+
 __device__ __forceinline__ float gate_rows32(int mode, const __nv_bfloat16* col, int stride, int nn, float bias,
                                              float rate, float lower_bound, float (&gv)[32]) {
     if (mode == KDA_GATE_SAFE) return gate_rows32<KDA_GATE_SAFE>(col, stride, nn, bias, rate, lower_bound, gv);

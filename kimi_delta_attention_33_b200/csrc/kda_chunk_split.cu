@@ -140,9 +140,6 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     const int rot = lane >> 2;                // store rotation (see rotate_groups8)
     const size_t qk_row = (size_t)H * KD, v_row = (size_t)HV * VD, g_row = (size_t)HV * KD;
 
-    // the state kernel that follows may start its set-up as SMs free up; it waits for this grid's
-    // completion before it reads any record
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         mbar_init(mbar, 1);
         mbar_init(mbar_in, 1);
@@ -484,6 +481,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     }
     if (tid == 0) bulk_wait_all();
     cta_sync_tc();
+    // Only now may the state kernel that follows be released: every record store of this CTA is
+    // complete.  (Triggering earlier is not safe: in a captured graph the dependent's wait returns
+    // once every CTA has triggered, and it sees only the memory written before the trigger.)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
 }
 
@@ -567,7 +568,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         return reinterpret_cast<const float*>(smem + L::ka(buf) + L::VEC_OFF)[which * KD + d];
     };
     // the chunk records are written by the preceding prep kernel: wait for it (a no-op unless this
-    // grid was launched as its programmatic dependent, whose set-up above then overlapped its tail)
+    // grid was launched as its programmatic dependent; the prep CTAs release it once their records
+    // are complete, so only the launch itself overlaps their tail)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {
         load_wq(0);

@@ -44,6 +44,8 @@ using bf16 = __nv_bfloat16;
 namespace {
 using namespace c64;
 
+constexpr int SP_THREADS = 512;  // 16 warps: TMEM lane quarter x column quarter
+
 struct TcLayout {
     // shared memory regions (bytes)
     static constexpr uint32_t X1 = 0;          // [128][128] [Qhat; -Khat]   A of M1, B of M3
@@ -74,7 +76,7 @@ struct TcLayout {
 
 }  // namespace
 
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(SP_THREADS, 1)
 chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                 const float* __restrict__ dt_bias, const float* __restrict__ S0, int T, int H, int HV,
@@ -101,7 +103,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     const int b = pair / HV, hv = pair - b * HV;
     const int h = hv / (HV / H);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    constexpr int NT = SP_THREADS;
+    const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column quarter
     const int vrow = 32 * wq + lane;          // value column held by this thread's TMEM lane
     const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[hv]) : 0.0f;
     const size_t qk_row = (size_t)H * KD;     // elements between consecutive tokens of q / k
@@ -114,10 +117,9 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (tid == 0) *sFlag = 0u;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    {
         TmemRow<32> row;
-        const int d0 = 64 * wh + 32 * half;
+        const int d0 = 32 * wc;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
             row.r[c] = __float_as_uint(S0 ? S0[((size_t)pair * KD + d0 + c) * VD + vrow] : 0.f);
@@ -132,15 +134,15 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     // registers, bring its g tile into GM by cp.async, and run its gate and in-chunk cumulative decay
     // into GM.  Rows past T are zero-filled.
     const uint32_t gm_addr = s_base + L::GM;
-    uint4 qr[4], kr[4];
+    uint4 qr[2], kr[2];
     float bload;
-    const int vc = tid & (VD - 1), jq0 = tid >> 7;  // value column, first token quad (quads jq0 + 2 x)
+    const int vc = tid & (VD - 1), q0 = tid >> 7;  // value column, first token quad (quads q0 + 4 x)
     auto load_inputs = [&](int tc0) {
         const int nn = min(CH, T - tc0);
         const size_t tk0 = (size_t)b * T + tc0;
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {  // g tile -> GM staging, v tile -> VS staging, bf16 [64][128]
-            const int u = tid + TC_THREADS * it;
+        for (int it = 0; it < 2; ++it) {  // g tile -> GM staging, v tile -> VS staging, bf16 [64][128]
+            const int u = tid + NT * it;
             const int i = u >> 4, c = u & 15;
             const bool ok = i < nn;
             cp_async16(gm_addr + i * 256 + c * 16, ok ? g + (tk0 + i) * g_row + (size_t)hv * KD + 8 * c : g, ok ? 16u : 0u);
@@ -149,8 +151,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         cp_async_commit();
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
+        for (int it = 0; it < 2; ++it) {
+            const int u = tid + NT * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
             qr[it] = make_uint4(0u, 0u, 0u, 0u);
             kr[it] = qr[it];
@@ -161,7 +163,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         bload = (tid < nn) ? to_f32(beta[(tk0 + tid) * HV + hv]) : 0.f;  // tid < nn <= 64
     };
-    // Gate + inclusive in-chunk cumulative log decay of the chunk at tc0 (two threads per key channel),
+    // Gate + inclusive in-chunk cumulative log decay of the chunk at tc0 (four threads per key channel),
     // its beta, the fast/exact decision and the per-channel vectors.  Uses sFpend, the pending state
     // factor the chunk starts from.  Returns whether the chunk takes the exact path.
     auto stage_gate = [&](int tc0) -> bool {
@@ -169,18 +171,24 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         cp_async_wait_all();
         __syncthreads();
         if (tid < CH) sBeta[tid] = bload;
-        const int gd = tid & (KD - 1), gh = tid >> 7;
-        float gv[32];
+        const int gd = tid & (KD - 1), gq = tid >> 7;  // channel, quarter of the rows (16 each)
+        float gv[16];
         {
             const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
-            const float acc = gate_rows32(gate_mode, sG + 32 * gh * KD + gd, KD, nn - 32 * gh, bias, rate, lower_bound, gv);
-            if (gh == 0) sFnext[gd] = acc;  // scratch: first-half totals
+            const float acc =
+                gate_rows16_regs(gate_mode, sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias, rate, lower_bound, gv);
+            // totals of quarters 0-2 to scratch (all three are rewritten below)
+            float* part = gq == 0 ? sFnext : gq == 1 ? sRho : sSig;
+            if (gq < 3) part[gd] = acc;
         }
         __syncthreads();  // the g staging has been read: GM becomes Gam
         {
-            const float off = gh ? sFnext[gd] : 0.f;
+            float off = 0.f;
+            if (gq > 0) off += sFnext[gd];
+            if (gq > 1) off += sRho[gd];
+            if (gq > 2) off += sSig[gd];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) sGam[gidx(32 * gh + r, gd)] = gv[r] + off;
+            for (int r = 0; r < 16; ++r) sGam[gidx(16 * gq + r, gd)] = gv[r] + off;
         }
         __syncthreads();
         if (tid < KD) {
@@ -219,8 +227,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         {
             const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::VS);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const int j = 4 * (jq0 + 2 * x);
+            for (int x = 0; x < 4; ++x) {
+                const int j = 4 * (q0 + 4 * x);
                 *reinterpret_cast<uint4*>(smem + L::VE + cm_off(vc, j, CH)) =
                     make_uint4(to_tf32(bf16_bits_to_f32(sVs[(j + 0) * VD + vc])),
                                to_tf32(bf16_bits_to_f32(sVs[(j + 1) * VD + vc])),
@@ -232,8 +240,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         // ---- P3: [Qhat; -Khat] -> X1, Kchk -> AT (B of M1), Kchk^T -> X2 (B of M6);
         //          D4 <- S_c^T diag(e^rho) (applies the previous chunk's pending factor too) ----------
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int u = tid + TC_THREADS * it;
+        for (int it = 0; it < 2; ++it) {
+            const int u = tid + NT * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
             float qf[8], kf[8], gf[8], rf[8], sf[8];
             bf16x8_to_f32(qr[it], qf);
@@ -262,12 +270,15 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                 *reinterpret_cast<uint4*>(smem + L::AT + cm_off(i, d, KD)) =
                     make_uint4(wc_[4 * hh], wc_[4 * hh + 1], wc_[4 * hh + 2], wc_[4 * hh + 3]);
             }
+            // Kchk^T: lanes that share a bank (same i & 3) take different d of their group of 8
+            const int rot = lane >> 2;
+            rotate_groups8(wc_, rot);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) *reinterpret_cast<uint32_t*>(smem + L::X2 + cm_off(8 * d8 + t, i, CH)) = wc_[t];
+            for (int t = 0; t < 8; ++t)
+                *reinterpret_cast<uint32_t*>(smem + L::X2 + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) = wc_[t];
         }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int d0 = 64 * wh + 32 * half;
+        {
+            const int d0 = 32 * wc;
             TmemRow<32> row;
             row.load(taddr(tmem, 32 * wq, L::D4 + d0));
             tmem_wait_ld();
@@ -291,14 +302,14 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             fence_after_sync();
             if (!__syncthreads_and(ok)) { aborted = true; break; }
             phase ^= 1u;
-            uint32_t raw[32];
-            tmem_ld32(taddr(tmem, 32 * wq, L::D2 + 32 * wh), raw);
+            uint32_t raw[16];
+            tmem_ld16(taddr(tmem, 32 * wq, L::D2 + 16 * wc), raw);
             tmem_wait_ld();
             const int i = 32 * (wq & 1) + lane;
             if (wq < 2) {
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 4) {
-                    const int j = 32 * wh + jj;
+                for (int jj = 0; jj < 16; jj += 4) {
+                    const int j = 16 * wc + jj;
                     uint4 w4;
                     w4.x = to_tf32(j + 0 <= i ? __uint_as_float(raw[jj + 0]) : 0.f);
                     w4.y = to_tf32(j + 1 <= i ? __uint_as_float(raw[jj + 1]) : 0.f);
@@ -309,17 +320,21 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             } else {
                 const float bi = -sBeta[i];  // rows 64-127 of D1 hold -Khat Kchk^T
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = 32 * wh + jj;
-                    sRT[i * RP + j] = (j < i) ? bi * __uint_as_float(raw[jj]) : 0.f;
+                for (int jj = 0; jj < 16; jj += 4) {
+                    const int j = 16 * wc + jj;
+                    *reinterpret_cast<float4*>(sRT + i * RP + j) =
+                        make_float4(j + 0 < i ? bi * __uint_as_float(raw[jj + 0]) : 0.f,
+                                    j + 1 < i ? bi * __uint_as_float(raw[jj + 1]) : 0.f,
+                                    j + 2 < i ? bi * __uint_as_float(raw[jj + 2]) : 0.f,
+                                    j + 3 < i ? bi * __uint_as_float(raw[jj + 3]) : 0.f);
                 }
             }
         } else {
-            // exact decay factors: 4096 (i, j) cells, 16 per thread; Gam is still in GM
-            float av[16], rr[16];
+            // exact decay factors: 4096 (i, j) cells, 8 per thread; Gam is still in GM
+            float av[8], rr[8];
 #pragma unroll 1
-            for (int x = 0; x < 16; ++x) {
-                const int p = tid + TC_THREADS * x;
+            for (int x = 0; x < 8; ++x) {
+                const int p = tid + NT * x;
                 const int i = p >> 6, j = p & 63;
                 float a = 0.f, r = 0.f;
                 if (j <= i && i < n) {
@@ -338,8 +353,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             }
             __syncthreads();  // Gam fully read: GM becomes R
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                const int p = tid + TC_THREADS * x;
+            for (int x = 0; x < 8; ++x) {
+                const int p = tid + NT * x;
                 const int i = p >> 6, j = p & 63;
                 *reinterpret_cast<uint32_t*>(smem + L::AT + cm_off(i, j, CH)) = to_tf32(av[x]);
                 sRT[i * RP + j] = rr[x];
@@ -353,8 +368,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         tri_inverse_step32(sRT, sX, tid);
         // Tb = T diag(beta) as tf32 into AT rows 64-127
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int u = tid + TC_THREADS * x;
+        for (int x = 0; x < 2; ++x) {
+            const int u = tid + NT * x;
             const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
             uint32_t w[4];
             const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
@@ -399,9 +414,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
         if (slow) {
             // exact path: M3 read S_c (rho = 0); M6 needs e^{Gam_end} S_c, i.e. e^sig per key column
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int d0 = 64 * wh + 32 * half;
+            {
+                const int d0 = 32 * wc;
                 TmemRow<32> row;
                 row.load(taddr(tmem, 32 * wq, L::D4 + d0));
                 tmem_wait_ld();
@@ -424,13 +438,13 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 
         // ---- outputs: O^T in D3 columns 0-63 (lane = value column) ----------------------------
         {
-            TmemRow<32> row;
-            row.load(taddr(tmem, 32 * wq, L::D3 + 32 * wh));
+            TmemRow<16> row;
+            row.load(taddr(tmem, 32 * wq, L::D3 + 16 * wc));
             tmem_wait_ld();
             bf16* op = o + tok0 * v_row + (size_t)hv * VD + vrow;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int i = 32 * wh + c;
+            for (int c = 0; c < 16; ++c) {
+                const int i = 16 * wc + c;
                 if (i < n) op[(size_t)i * v_row] = __float2bfloat16_rn(__uint_as_float(row.r[c]));
             }
         }
@@ -448,9 +462,8 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         // give any MMA still in flight one more bounded chance to drain before TMEM is released
         mbar_wait(mbar, phase, WAIT_POLLS);
     } else if (S_T) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int d0 = 64 * wh + 32 * half;
+        {
+            const int d0 = 32 * wc;
             TmemRow<32> row;
             row.load(taddr(tmem, 32 * wq, L::D4 + d0));
             tmem_wait_ld();
@@ -467,7 +480,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a) {
     using L = TcLayout;
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<<<a.B * a.HV, TC_THREADS, L::BYTES, a.stream>>>(
+    chunk_tc_kernel<<<a.B * a.HV, SP_THREADS, L::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.S0, a.T, a.H, a.HV,
         a.gate_mode, a.lower_bound, a.scale, static_cast<bf16*>(a.o), a.S_T, a.status);
