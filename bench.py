@@ -316,61 +316,85 @@ def workload_config(w, ws, flushed):
 
 
 def run_e2e(args, w, x, dev, kda):
-    """Same metric through the public API with host buffers: pinned H2D of the step's inputs, the call,
-    D2H of the step's result, all inside the timed region."""
-    stream = torch.cuda.current_stream(dev)
+    """Same metric through the public API with host buffers: every step copies its inputs from pinned
+    host memory to the device, makes the call, and copies its result back, all inside the timed
+    region.  Two buffer sets and three streams overlap step i's call with step i+1's input copies and
+    step i-1's result copies, as a serving loop would."""
     names = ("q", "k", "v", "g", "beta")
+    h2d_s, comp_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nbuf = 2
     if w.is_decode:
-        host = {n: x[n][:, 0].contiguous().cpu().pin_memory() for n in names}
-        devb = {n: torch.empty_like(host[n], device=dev) for n in names}
+        inputs = names
+        host = [{n: x[n][:, 0].contiguous().cpu().pin_memory() for n in inputs} for _ in range(nbuf)]
         S = x["S0"].clone()
-        o_dev = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
-        o_host = torch.empty(o_dev.shape, dtype=w.dtype).pin_memory()
+        outs = [torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev) for _ in range(nbuf)]
+        out_host = [torch.empty(w.B, w.HV, w.V, dtype=w.dtype).pin_memory() for _ in range(nbuf)]
         units = w.B
 
-        def call():
-            for n in names:
-                devb[n].copy_(host[n], non_blocking=True)
+        def launch(devb, j):
             kda.recurrent_step(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"], S, x["A_log"], x["dt_bias"],
-                               gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o_dev)
-            o_host.copy_(o_dev, non_blocking=True)
-        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-        d2h = o_host.numel() * o_host.element_size()
+                               gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=outs[j])
+            return (outs[j],)
+        results_host = [(out_host[j],) for j in range(nbuf)]
     else:
         inputs = names + (("S0",) if x["S0"] is not None else ())
-        host = {n: x[n].cpu().pin_memory() for n in inputs}
-        devb = {n: torch.empty_like(host[n], device=dev) for n in inputs}
+        host = [{n: x[n].cpu().pin_memory() for n in inputs} for _ in range(nbuf)]
         ws_bytes = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
-        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
-        o_dev = torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev)
-        S_dev = torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev)
-        o_host = torch.empty(o_dev.shape, dtype=w.dtype).pin_memory()
-        S_host = torch.empty(S_dev.shape, dtype=torch.float32).pin_memory()
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)  # calls are ordered on comp_s
+        o_dev = [torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev) for _ in range(nbuf)]
+        S_dev = [torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev) for _ in range(nbuf)]
+        results_host = [(torch.empty(o_dev[0].shape, dtype=w.dtype).pin_memory(),
+                         torch.empty(S_dev[0].shape, dtype=torch.float32).pin_memory()) for _ in range(nbuf)]
         units = w.B * w.T
 
-        def call():
-            for n in inputs:
-                devb[n].copy_(host[n], non_blocking=True)
+        def launch(devb, j):
             kda.chunk_fwd(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"], x["A_log"], x["dt_bias"],
-                          devb.get("S0"), chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o_dev,
-                          S_T=S_dev, workspace=workspace)
-            o_host.copy_(o_dev, non_blocking=True)
-            S_host.copy_(S_dev, non_blocking=True)
-        h2d = sum(host[n].numel() * host[n].element_size() for n in inputs)
-        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
-    for _ in range(max(args.warmup, 1)):
-        call()
+                          devb.get("S0"), chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o_dev[j],
+                          S_T=S_dev[j], workspace=workspace)
+            return (o_dev[j], S_dev[j])
+    devbufs = [{n: torch.empty_like(host[j][n], device=dev) for n in inputs} for j in range(nbuf)]
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def step(i):
+        j = i % nbuf
+        with torch.cuda.stream(h2d_s):  # inputs of step i, once step i - nbuf's call released the buffer
+            if i >= nbuf:
+                h2d_s.wait_event(ev_done[j])
+            for n in inputs:
+                devbufs[j][n].copy_(host[j][n], non_blocking=True)
+            ev_in[j].record(h2d_s)
+        with torch.cuda.stream(comp_s):  # the call, once its inputs landed and its outputs were read back
+            comp_s.wait_event(ev_in[j])
+            if i >= nbuf:
+                comp_s.wait_event(ev_out[j])
+            res = launch(devbufs[j], j)
+            ev_done[j].record(comp_s)
+        with torch.cuda.stream(d2h_s):  # the step's result back to the host
+            d2h_s.wait_event(ev_done[j])
+            for dst, src in zip(results_host[j], res):
+                dst.copy_(src, non_blocking=True)
+            ev_out[j].record(d2h_s)
+
+    for i in range(max(args.warmup, 1)):
+        step(i)
     torch.cuda.synchronize(dev)
     n = max(3, min(args.steps, 50))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n):
-        call()
-    b.record(stream)
+    a.record(h2d_s)
+    for i in range(n):
+        step(i)
+    d2h_s.wait_stream(h2d_s)
+    d2h_s.wait_stream(comp_s)
+    b.record(d2h_s)
     torch.cuda.synchronize(dev)
     sec = a.elapsed_time(b) / 1e3 / n
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in inputs)
+    d2h = sum(t.numel() * t.element_size() for t in results_host[0])
     return {"value": round(units / sec, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": n}
+            "d2h_bytes_per_step": int(d2h), "steps": n, "overlap": "inputs of step i+1 and results of step i-1 "
+            "copy while step i runs (two buffer sets, three streams)"}
 
 
 def run_decode_extra(args, dev, kda, hbm_peak):

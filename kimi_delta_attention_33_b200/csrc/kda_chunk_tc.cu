@@ -76,13 +76,15 @@ struct TcLayout {
 
 }  // namespace
 
+template <int MODE>
 __global__ void __launch_bounds__(SP_THREADS, 1)
 chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                 const float* __restrict__ dt_bias, const float* __restrict__ S0, int T, int H, int HV,
-                int gate_mode, float lower_bound, float scale, bf16* __restrict__ o, float* __restrict__ S_T,
+                float lower_bound, float scale, bf16* __restrict__ o, float* __restrict__ S_T,
                 unsigned int* __restrict__ status) {
     using L = TcLayout;
+    constexpr int gate_mode = MODE;
     extern __shared__ __align__(1024) unsigned char smem[];
     float* sRho = reinterpret_cast<float*>(smem + L::RHO);
     float* sSig = reinterpret_cast<float*>(smem + L::SIG);
@@ -176,7 +178,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         {
             const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
             const float acc =
-                gate_rows16_regs(gate_mode, sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias, rate, lower_bound, gv);
+                gate_rows16_regs<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias, rate, lower_bound, gv);
             // totals of quarters 0-2 to scratch (all three are rewritten below)
             float* part = gq == 0 ? sFnext : gq == 1 ? sRho : sSig;
             if (gq < 3) part[gd] = acc;
@@ -476,15 +478,26 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
 }
 
-cudaError_t launch_chunk_tc(const ChunkArgs& a) {
+namespace {
+template <int MODE>
+cudaError_t launch_tc(const ChunkArgs& a) {
     using L = TcLayout;
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<<<a.B * a.HV, SP_THREADS, L::BYTES, a.stream>>>(
+    chunk_tc_kernel<MODE><<<a.B * a.HV, SP_THREADS, L::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.S0, a.T, a.H, a.HV,
-        a.gate_mode, a.lower_bound, a.scale, static_cast<bf16*>(a.o), a.S_T, a.status);
+        a.lower_bound, a.scale, static_cast<bf16*>(a.o), a.S_T, a.status);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_tc(const ChunkArgs& a) {
+    // one kernel per gate mode: the gate's 16-row loop is straight-line code in each
+    return a.gate_mode == KDA_GATE_SAFE       ? launch_tc<KDA_GATE_SAFE>(a)
+           : a.gate_mode == KDA_GATE_STANDARD ? launch_tc<KDA_GATE_STANDARD>(a)
+                                              : launch_tc<KDA_GATE_NONE>(a);
 }
 
 }  // namespace kda
