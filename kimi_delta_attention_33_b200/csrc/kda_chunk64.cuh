@@ -36,51 +36,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
     }
 }
 
-// Gate values (KDA notes, "Gate 激活") of one key channel for 32 consecutive rows of a staged bf16
-// g tile (col points at the first row's element, rows `stride` elements apart; rows >= nn are
-// padding and give 0), written to gv as their running sum; returns the sum.  The mode is a template
-// parameter so that the 32 independent evaluations interleave before the dependent prefix sum.
-template <int MODE>
-__device__ __forceinline__ float gate_rows32(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
-                                             float lower_bound, float (&gv)[32]) {
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-        const float x = __bfloat162float(col[r * stride]);
-        gv[r] = (r < nn) ? gate_value_fast(x, bias, rate, MODE, lower_bound) : 0.f;
-    }
-    float acc = 0.f;
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-        acc += gv[r];
-        gv[r] = acc;
-    }
-    return acc;
-}
-
-// Gate values of one key channel for 32 consecutive rows, as their running sum written to an fp32
-// column (dst[r * dst_stride] through the index function idx(r)), eight rows at a time so that the
-// code stays small; returns the sum.
-template <int MODE, typename Idx>
-__device__ __forceinline__ float gate_rows32_to(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
-                                                float lower_bound, float* dst, Idx idx) {
-    float acc = 0.f;
-#pragma unroll 1
-    for (int r0 = 0; r0 < 32; r0 += 8) {
-        float x[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float gr = __bfloat162float(col[(r0 + r) * stride]);
-            x[r] = (r0 + r < nn) ? gate_value_fast(gr, bias, rate, MODE, lower_bound) : 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            acc += x[r];
-            dst[idx(r0 + r)] = acc;
-        }
-    }
-    return acc;
-}
-
 // The same for 16 rows (CTAs with four threads per key channel).
 template <int MODE, typename Idx>
 __device__ __forceinline__ float gate_rows16_to(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
@@ -129,53 +84,7 @@ __device__ __forceinline__ float gate_rows16_regs(int mode, const __nv_bfloat16*
     return gate_rows16_regs<KDA_GATE_NONE>(col, stride, nn, bias, rate, lower_bound, gv);
 }
 
-__device__ __forceinline__ float gate_rows32(int mode, const __nv_bfloat16* col, int stride, int nn, float bias,
-                                             float rate, float lower_bound, float (&gv)[32]) {
-    if (mode == KDA_GATE_SAFE) return gate_rows32<KDA_GATE_SAFE>(col, stride, nn, bias, rate, lower_bound, gv);
-    if (mode == KDA_GATE_STANDARD) return gate_rows32<KDA_GATE_STANDARD>(col, stride, nn, bias, rate, lower_bound, gv);
-    return gate_rows32<KDA_GATE_NONE>(col, stride, nn, bias, rate, lower_bound, gv);
-}
-
 __device__ __forceinline__ float bf16_bits_to_f32(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
-
-// One doubling step of the unit-lower-triangular inverse, in place over the strictly-lower part
-// stored with row pitch RP: every diagonal block of size 2 HS, [[Ta, 0], [C, Td]], whose diagonal
-// sub-blocks already hold their inverses, gets its lower-left block -Td C Ta (Ta, Td with implicit
-// unit diagonals).  X = C Ta goes through the scratch sX.
-template <int HS, int NT = TC_THREADS>
-__device__ __forceinline__ void tri_inverse_step(float* sRT, float* sX, int tid) {
-    constexpr int CNT = (CH / (2 * HS)) * HS * HS;
-    constexpr int ITERS = (CNT + NT - 1) / NT;
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const int e = tid + NT * it;
-        if (CNT % NT == 0 || e < CNT) {
-            const int c = e % HS, r = (e / HS) % HS, base = (e / (HS * HS)) * 2 * HS;
-            const float* Crow = sRT + (base + HS + r) * RP + base;
-            float acc = Crow[c];
-#pragma unroll
-            for (int m = 1; m < HS; ++m)
-                if (m > c) acc += Crow[m] * sRT[(base + m) * RP + base + c];
-            sX[e] = acc;
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const int e = tid + NT * it;
-        if (CNT % NT == 0 || e < CNT) {
-            const int c = e % HS, r = (e / HS) % HS, blk = e / (HS * HS), base = blk * 2 * HS;
-            const float* Drow = sRT + (base + HS + r) * RP + base + HS;
-            const float* Xb = sX + blk * HS * HS;
-            float acc = Xb[r * HS + c];
-#pragma unroll
-            for (int m = 0; m < HS - 1; ++m)
-                if (m < r) acc += Drow[m] * Xb[m * HS + c];
-            sRT[(base + HS + r) * RP + base + c] = -acc;
-        }
-    }
-    __syncthreads();
-}
 
 // The doubling steps with blocks of 2, 4, 8 and 16 rows never cross a 16 x 16 diagonal block, so
 // one warp can take one such block through all four with warp-level syncs only: warp w < 4 inverts
