@@ -10,7 +10,7 @@ namespace kda {
 namespace c64 {
 using namespace tc;
 
-constexpr int TC_THREADS = 256;  // threads of the kernels that run the triangular inverse
+constexpr int INV_THREADS = 512;  // threads of the kernels that run the triangular inverse
 constexpr int KD = 128;          // key dimension
 constexpr int VD = 128;          // value dimension
 constexpr int CH = 64;           // chunk length
@@ -129,100 +129,82 @@ __device__ __forceinline__ void tri_inverse_diag16(float* sRT, float* sX, int ti
     __syncthreads();
 }
 
-// The last two doubling steps with one column per lane and four rows per thread: X = C Ta and the
-// new block -Td X, accumulating over m with loads of four consecutive row entries at a time.
-// Step 16 -> 32 (two blocks, at 0 and 32): warp w serves block w / 4 and rows 4 (w % 4) .. + 3 of its
-// 16 x 16 lower-left block; lane = column (lane % 16) and row pair (lane / 16).
+// The last two doubling steps, for CTAs of INV_THREADS = 512 threads.  With T's strictly-lower
+// part stored in place and its unit diagonal implicit, a block [[Ta, 0], [C, Td]] of the matrix being
+// inverted, whose diagonal blocks Ta, Td are already inverted, becomes [[Ta, 0], [-Td C Ta, Td]]:
+// first X = C Ta (the m = c term of Ta is the unit diagonal), then C <- -(X + Td' X) with Td' the
+// strictly-lower part of Td.
+// Step 16 -> 32 (two 32 x 32 blocks, at 0 and 32): thread (blk, r, c) = (tid / 256, (tid / 16) % 16,
+// tid % 16) owns entry (r, c) of its block's 16 x 16 lower-left part.
 __device__ __forceinline__ void tri_inverse_step16(float* sRT, float* sX, int tid) {
-    const bool active = tid < TC_THREADS;  // larger CTAs: threads past the first 256 only join the barriers
-    const int w = (tid >> 5) & 7, lane = tid & 31;
-    const int base = 32 * (w >> 2), c = lane & 15;
-    const int r0 = 4 * (w & 3) + 2 * (lane >> 4);  // rows r0, r0 + 1 of the 16 x 16 lower-left block
-    float acc[2];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) acc[x] = sRT[(base + 16 + r0 + x) * RP + base + c];
+    const int blk = tid >> 8, r = (tid >> 4) & 15, c = tid & 15, base = 32 * blk;
+    const float* Crow = sRT + (base + 16 + r) * RP + base;
+    float acc = Crow[c];
 #pragma unroll
     for (int m4 = 0; m4 < 16; m4 += 4) {
-        float a[4];
+        const float4 cr = *reinterpret_cast<const float4*>(Crow + m4);
+        const float cm[4] = {cr.x, cr.y, cr.z, cr.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) a[t] = (m4 + t > c) ? sRT[(base + m4 + t) * RP + base + c] : 0.f;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const float4 cr = *reinterpret_cast<const float4*>(sRT + (base + 16 + r0 + x) * RP + base + m4);
-            acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
-        }
+        for (int t = 0; t < 4; ++t)
+            if (m4 + t > c) acc += cm[t] * sRT[(base + m4 + t) * RP + base + c];
     }
-    if (active) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) sX[(w >> 2) * 256 + (r0 + x) * 16 + c] = acc[x];
-    }
+    float* Xb = sX + blk * 256;
+    Xb[r * 16 + c] = acc;
     __syncthreads();
-    const float* Xb = sX + (w >> 2) * 256;
-#pragma unroll
-    for (int x = 0; x < 2; ++x) acc[x] = Xb[(r0 + x) * 16 + c];
+    const float* Drow = sRT + (base + 16 + r) * RP + base + 16;
+    acc = Xb[r * 16 + c];
 #pragma unroll
     for (int m4 = 0; m4 < 16; m4 += 4) {
-        float xm[4];
+        const float4 dr = *reinterpret_cast<const float4*>(Drow + m4);
+        const float dm[4] = {dr.x, dr.y, dr.z, dr.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) xm[t] = Xb[(m4 + t) * 16 + c];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const float4 dr = *reinterpret_cast<const float4*>(sRT + (base + 16 + r0 + x) * RP + base + 16 + m4);
-            const int r = r0 + x;
-            acc[x] += (m4 + 0 < r ? dr.x * xm[0] : 0.f) + (m4 + 1 < r ? dr.y * xm[1] : 0.f) +
-                      (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
-        }
+        for (int t = 0; t < 4; ++t)
+            if (m4 + t < r) acc += dm[t] * Xb[(m4 + t) * 16 + c];
     }
-    if (active) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) sRT[(base + 16 + r0 + x) * RP + base + c] = -acc[x];
-    }
+    sRT[(base + 16 + r) * RP + base + c] = -acc;
     __syncthreads();
 }
 
-// Step 32 -> 64 (one block): warp w serves rows 4 w + {0..3}, lane = column.
+// Step 32 -> 64 (one 64 x 64 block): thread (r, c) = (tid / 16, tid % 16) owns entries (r, c) and
+// (r, c + 16) of the 32 x 32 lower-left part.
 __device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int tid) {
-    const bool active = tid < TC_THREADS;  // larger CTAs: threads past the first 256 only join the barriers
-    const int w = (tid >> 5) & 7, c = tid & 31, r0 = 4 * w;
-    float acc[4];
-#pragma unroll
-    for (int x = 0; x < 4; ++x) acc[x] = sRT[(32 + r0 + x) * RP + c];
+    const int r = tid >> 4, c = tid & 15;
+    const float* Crow = sRT + (32 + r) * RP;
+    float acc0 = Crow[c], acc1 = Crow[c + 16];
 #pragma unroll
     for (int m4 = 0; m4 < 32; m4 += 4) {
-        float a[4];
+        const float4 cr = *reinterpret_cast<const float4*>(Crow + m4);
+        const float cm[4] = {cr.x, cr.y, cr.z, cr.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) a[t] = (m4 + t > c) ? sRT[(m4 + t) * RP + c] : 0.f;
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float4 cr = *reinterpret_cast<const float4*>(sRT + (32 + r0 + x) * RP + m4);
-            acc[x] += cr.x * a[0] + cr.y * a[1] + cr.z * a[2] + cr.w * a[3];
+        for (int t = 0; t < 4; ++t) {
+            const int m = m4 + t;
+            if (m > c) acc0 += cm[t] * sRT[m * RP + c];
+            if (m4 >= 16 && m > c + 16) acc1 += cm[t] * sRT[m * RP + c + 16];
         }
     }
-    if (active) {
-#pragma unroll
-        for (int x = 0; x < 4; ++x) sX[(r0 + x) * 32 + c] = acc[x];
-    }
+    sX[r * 32 + c] = acc0;
+    sX[r * 32 + c + 16] = acc1;
     __syncthreads();
-#pragma unroll
-    for (int x = 0; x < 4; ++x) acc[x] = sX[(r0 + x) * 32 + c];
+    const float* Drow = sRT + (32 + r) * RP + 32;
+    acc0 = sX[r * 32 + c];
+    acc1 = sX[r * 32 + c + 16];
+    const int rmax = 2 * (tid >> 5) + 1;  // largest row of this warp: rows m < r <= rmax contribute
 #pragma unroll
     for (int m4 = 0; m4 < 32; m4 += 4) {
-        if (m4 >= r0 + 3) break;  // warp-uniform: no row of this warp reaches these m
-        float xm[4];
+        if (m4 >= rmax) break;  // warp-uniform
+        const float4 dr = *reinterpret_cast<const float4*>(Drow + m4);
+        const float dm[4] = {dr.x, dr.y, dr.z, dr.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) xm[t] = sX[(m4 + t) * 32 + c];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float4 dr = *reinterpret_cast<const float4*>(sRT + (32 + r0 + x) * RP + 32 + m4);
-            const int r = r0 + x;
-            acc[x] += (m4 + 0 < r ? dr.x * xm[0] : 0.f) + (m4 + 1 < r ? dr.y * xm[1] : 0.f) +
-                      (m4 + 2 < r ? dr.z * xm[2] : 0.f) + (m4 + 3 < r ? dr.w * xm[3] : 0.f);
+        for (int t = 0; t < 4; ++t) {
+            const int m = m4 + t;
+            if (m < r) {
+                acc0 += dm[t] * sX[m * 32 + c];
+                acc1 += dm[t] * sX[m * 32 + c + 16];
+            }
         }
     }
-    if (active) {
-#pragma unroll
-        for (int x = 0; x < 4; ++x) sRT[(32 + r0 + x) * RP + c] = -acc[x];
-    }
+    sRT[(32 + r) * RP + c] = -acc0;
+    sRT[(32 + r) * RP + c + 16] = -acc1;
     __syncthreads();
 }
 

@@ -29,6 +29,9 @@
 //                                             chunk-to-chunk path)
 // Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
 // where shared memory allows.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kda_chunk64.cuh"
 #include "kda_internal.h"
 
@@ -51,8 +54,10 @@ struct Rec {
 
 struct PrepLayout {
     static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1); Qhat is the record's WQ rows
-                                             //   64-127; once M1 is done rows 0-63 stage the next chunk's
-                                             //   g (bf16 [64][128]) and v (bf16 [64][128]) tiles
+                                             //   64-127; once M1 is done (and Qhat's record store has read
+                                             //   it) X1 stages the next chunk's input tiles, bf16 [64][128]
+                                             //   each: g, v (plain rows), q, k (two 64-column halves each,
+                                             //   rows of 128 bytes with the 128-byte swizzle)
     static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling
                                              //   scratch; then U^T [128][64] fp32 (record UT)
     static constexpr uint32_t XS = CK + 64 * RP * 4;
@@ -63,6 +68,7 @@ struct PrepLayout {
     static constexpr uint32_t VEC = 229376;
     static constexpr uint32_t RHO = VEC, SIG = VEC + 512, SC2 = VEC + 1024, BETA = VEC + 1536;
     static constexpr uint32_t MBAR = VEC + 1792, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8, FLAG = TBASE + 4;
+    static constexpr uint32_t STG_G = X1, STG_V = X1 + 16384, STG_Q = X1 + 32768, STG_K = X1 + 49152;
     static constexpr uint32_t BYTES = FLAG + 4;
     static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
@@ -90,6 +96,7 @@ struct StateLayout {
 
 constexpr int STATE_THREADS = 256;
 constexpr int PREP_THREADS = 512;
+static_assert(PREP_THREADS == INV_THREADS, "the triangular inverse assumes 512 threads");
 
 struct Task {
     int pair, c, b, hv, h, nn;
@@ -119,7 +126,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                   const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, int T, int H, int HV, int NC, int ntasks,
                   float lower_bound, float scale, unsigned char* __restrict__ rec_base,
-                  unsigned int* __restrict__ status) {
+                  unsigned int* __restrict__ status, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_g) {
     using L = PrepLayout;
     constexpr int NT = PREP_THREADS;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -138,7 +147,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column quarter
     const int rot = lane >> 2;                // store rotation (see rotate_groups8)
-    const size_t qk_row = (size_t)H * KD, v_row = (size_t)HV * VD, g_row = (size_t)HV * KD;
+    const size_t qk_row = (size_t)H * KD;  // elements between consecutive tokens of q / k (exact path)
 
     if (tid == 0) {
         mbar_init(mbar, 1);
@@ -151,40 +160,26 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     uint32_t phase = 0, phase_in = 0;
     bool aborted = false, in_pending = false;
 
-    // Inputs of one chunk: g and v tiles into the staging half of X1 by bulk copies, one 256-byte row
-    // per thread of the first 128, completing on mbar_in (rows past T are zeroed by plain stores
-    // instead); q, k, beta, this head's A_log and this thread's dt_bias entry into registers.
-    // q / k units: u = tid + NT * it covers row i = 8 (u / 128) + u % 8 and key group d8 = (u / 8) % 16.
-    uint4 qr[2], kr[2];
+    // Inputs of one chunk: the q, k, g and v tiles into X1 by six tensor-map copies issued by thread 32
+    // (rows past T read as zero), completing on mbar_in; beta, this head's A_log and this thread's
+    // dt_bias entry into registers.  Thread 32 first lets the record stores it issued finish reading
+    // X1.  q / k are read back in the operand pass as units u = tid + NT * it: row
+    // i = 8 (u / 128) + u % 8, key group d8 = (u / 8) % 16.
     uint32_t beta_bits = 0;  // raw bf16 bits of beta for row tid (tid < 64), converted where used
     float alog_in = 0.f, bias_in = 0.f;
     auto load_inputs = [&](const Task& tk) {
-        if (tid < 2 * CH) {
-            const int i = tid & (CH - 1), which = tid >> 6;  // which: 0 g, 1 v
-            if (tid == 0) mbar_expect_tx(mbar_in, 2u * 256u * (uint32_t)tk.nn);
-            const uint32_t dst = s_base + L::X1 + which * 16384 + i * 256;
-            if (i < tk.nn) {
-                const bf16* src = which == 0 ? g + (tk.tk0 + i) * g_row + (size_t)tk.hv * KD
-                                             : v + (tk.tk0 + i) * v_row + (size_t)tk.hv * VD;
-                bulk_load(dst, src, 256, mbar_in);
-            } else {
-                uint4* z = reinterpret_cast<uint4*>(smem + L::X1 + which * 16384 + i * 256);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) z[c] = make_uint4(0u, 0u, 0u, 0u);
-            }
+        if (tid == 32) {
+            bulk_wait_read();
+            mbar_expect_tx(mbar_in, 4u * 16384u);
+            const int t0 = tk.c * CH;
+            tma_load_4d(s_base + L::STG_G, &tm_g, 0, tk.hv, t0, tk.b, mbar_in);
+            tma_load_4d(s_base + L::STG_V, &tm_v, 0, tk.hv, t0, tk.b, mbar_in);
+            tma_load_4d(s_base + L::STG_Q, &tm_q, 0, tk.h, t0, tk.b, mbar_in);
+            tma_load_4d(s_base + L::STG_Q + 8192, &tm_q, 64, tk.h, t0, tk.b, mbar_in);
+            tma_load_4d(s_base + L::STG_K, &tm_k, 0, tk.h, t0, tk.b, mbar_in);
+            tma_load_4d(s_base + L::STG_K + 8192, &tm_k, 64, tk.h, t0, tk.b, mbar_in);
         }
         in_pending = true;
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int u = tid + NT * it;
-            const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
-            qr[it] = make_uint4(0u, 0u, 0u, 0u);
-            kr[it] = qr[it];
-            if (i < tk.nn) {
-                qr[it] = __ldg(reinterpret_cast<const uint4*>(q + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD + 8 * d8));
-                kr[it] = __ldg(reinterpret_cast<const uint4*>(k + (tk.tk0 + i) * qk_row + (size_t)tk.h * KD + 8 * d8));
-            }
-        }
         beta_bits = (tid < tk.nn) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(beta) + (tk.tk0 + tid) * HV + tk.hv)
                                   : 0u;
         if (MODE != KDA_GATE_NONE) {
@@ -251,6 +246,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
 
         // ---- V^T into VT from the staged v tile (value column vc, token quads q0 + 4 x) ---------------
+        uint4 qr[2], kr[2];  // bf16 q / k of this thread's two operand units
         {
             const unsigned short* sVs = reinterpret_cast<const unsigned short*>(smem + L::X1 + 16384);
             const int vc = tid & (VD - 1), q0 = tid >> 7;
@@ -261,9 +257,19 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 vv[2 * x] = (uint32_t)sVs[(j + 0) * VD + vc] | ((uint32_t)sVs[(j + 1) * VD + vc] << 16);
                 vv[2 * x + 1] = (uint32_t)sVs[(j + 2) * VD + vc] | ((uint32_t)sVs[(j + 3) * VD + vc] << 16);
             }
-            // the previous chunk's record stores must be done reading X1, KA and CK before P3 rewrites
-            // them (and the staged tiles in X1 must all be read)
-            if (tid == 0) bulk_wait_read();
+            // this thread's q / k units from the swizzled staging (16-byte chunk c of row i sits at chunk
+            // c ^ (i % 8) of its 128-byte row)
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int u = tid + NT * it;
+                const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
+                const uint32_t off = (uint32_t)(d8 >> 3) * 8192u + (uint32_t)i * 128u + ((uint32_t)((d8 & 7) ^ (i & 7)) << 4);
+                qr[it] = *reinterpret_cast<const uint4*>(smem + L::STG_Q + off);
+                kr[it] = *reinterpret_cast<const uint4*>(smem + L::STG_K + off);
+            }
+            // the previous chunk's record stores must be done reading CK before P3 rewrites it, and
+            // the staged tiles in X1 must all be read
+            if (tid == 32) bulk_wait_read();
             __syncthreads();
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
@@ -317,6 +323,11 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
         fence_proxy_async();
         cta_sync_tc();
+        if (tid == 32) {  // Qhat and Kchk^T are final: their record stores run while M1 does
+            bulk_store(rec + Rec::WQ + 32768, s_base + L::X1 + 32768, 32768);  // W goes straight out later
+            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);  // A goes straight to the record later
+            bulk_commit();
+        }
 
         // Khat^T into GM (B rows 0-127 of M7) once Gam is no longer read
         auto write_khat_t = [&]() {
@@ -466,9 +477,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         }
         fence_proxy_async();
         cta_sync_tc();
-        if (tid == 0) {
-            bulk_store(rec + Rec::WQ + 32768, s_base + L::X1 + 32768, 32768);  // Qhat; W went straight out
-            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);  // Kchk^T; A went straight to the record
+        if (tid == 32) {
             bulk_store(rec + Rec::UT, s_base + L::CK, 32768);
             bulk_commit();
         }
@@ -479,7 +488,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         mbar_wait(mbar, phase, WAIT_POLLS);  // one more bounded chance for an MMA in flight to drain
         if (in_pending) mbar_wait(mbar_in, phase_in, WAIT_POLLS);  // and for staged copies in flight
     }
-    if (tid == 0) bulk_wait_all();
+    if (tid == 32) bulk_wait_all();
     cta_sync_tc();
     // Only now may the state kernel that follows be released: every record store of this CTA is
     // complete.  (Triggering earlier is not safe: in a captured graph the dependent's wait returns
@@ -739,15 +748,49 @@ size_t chunk_split_workspace(int B, int T, int HV) {
 }
 
 namespace {
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// Tensor map over a bf16 [B][T][heads][128] tensor whose box is 64 tokens of one head and `inner`
+// entries of the last dimension: plain rows for inner = 128, 128-byte rows with the 128-byte swizzle
+// for inner = 64.  Tokens past T read as zero.
+cudaError_t make_token_tile_map(CUtensorMap* m, const void* base, int B, int T, int heads, int inner) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {256, (cuuint64_t)heads * 256, (cuuint64_t)T * heads * 256};  // bytes
+    const cuuint32_t box[4] = {(cuuint32_t)inner, 1, (cuuint32_t)CH, 1};
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int MODE>
 cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepLayout::BYTES);
     if (e != cudaSuccess) return e;
+    CUtensorMap tq, tk, tv, tg;
+    if ((e = make_token_tile_map(&tq, a.q, a.B, a.T, a.H, 64)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&tk, a.k, a.B, a.T, a.H, 64)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&tv, a.v, a.B, a.T, a.HV, 128)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&tg, a.g, a.B, a.T, a.HV, 128)) != cudaSuccess) return e;
     chunk_prep_kernel<MODE><<<grid, PREP_THREADS, PrepLayout::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
-        ntasks, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status);
+        ntasks, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status, tq, tk, tv, tg);
     return cudaGetLastError();
 }
 

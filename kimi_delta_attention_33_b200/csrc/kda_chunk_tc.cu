@@ -45,6 +45,7 @@ namespace {
 using namespace c64;
 
 constexpr int SP_THREADS = 512;  // 16 warps: TMEM lane quarter x column quarter
+static_assert(SP_THREADS == INV_THREADS, "the triangular inverse assumes 512 threads");
 
 struct TcLayout {
     // shared memory regions (bytes)

@@ -170,6 +170,17 @@ __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, ui
                  "l"(src), "r"(bytes), "r"(mbar)
                  : "memory");
 }
+// Tiled 4-D tensor copy global -> shared through a tensor map (a __grid_constant__ kernel parameter),
+// completing on an mbarrier as transaction bytes.  Coordinates innermost first; the innermost one
+// times the element size must be a multiple of 16 bytes.  Elements outside the tensor read as zero.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst_smem, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(mbar)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
                  : "memory");
