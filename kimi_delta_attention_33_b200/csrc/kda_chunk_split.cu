@@ -66,10 +66,12 @@ struct PrepLayout {
     static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
     static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)
     static constexpr uint32_t VEC = 229376;
-    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, SC2 = VEC + 1024, BETA = VEC + 1536;
-    static constexpr uint32_t MBAR = VEC + 1792, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8, FLAG = TBASE + 4;
+    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024;
+    static constexpr uint32_t MBAR = VEC + 1280, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8;
+    static constexpr uint32_t PART = KA + 32768;  // gate: per-channel quarter totals and Gam_0 (5 x [128] fp32),
+                                                  //   in the Tb rows, which are free until the inverse
     static constexpr uint32_t STG_G = X1, STG_V = X1 + 16384, STG_Q = X1 + 32768, STG_K = X1 + 49152;
-    static constexpr uint32_t BYTES = FLAG + 4;
+    static constexpr uint32_t BYTES = TBASE + 4;
     static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
     static_assert(GM + 32768 == VT, "M7's B operand spans GM and VT");
@@ -134,13 +136,12 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     extern __shared__ __align__(1024) unsigned char smem[];
     float* sRho = reinterpret_cast<float*>(smem + L::RHO);
     float* sSig = reinterpret_cast<float*>(smem + L::SIG);
-    float* sSc2 = reinterpret_cast<float*>(smem + L::SC2);
+    float* sPart = reinterpret_cast<float*>(smem + L::PART);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
     const bf16* sG = reinterpret_cast<const bf16*>(smem + L::X1);  // staged g tile
-    uint32_t* sFlag = reinterpret_cast<uint32_t*>(smem + L::FLAG);
     const uint32_t s_base = smem_u32(smem);
     const uint32_t mbar = s_base + L::MBAR, mbar_in = s_base + L::MBAR_IN;
 
@@ -154,7 +155,6 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         mbar_init(mbar_in, 1);
     }
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
-    if (tid == 0) *sFlag = 0u;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
     uint32_t phase = 0, phase_in = 0;
@@ -197,52 +197,44 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         const float rate = (MODE != KDA_GATE_NONE) ? expf(alog_in) : 0.0f;
 
         // ---- gate and inclusive in-chunk cumulative log decay (four threads per key channel) ----
+        // Thread (gd, gq) keeps the running sums of rows 16 gq .. 16 gq + 15 of channel gd in registers;
+        // the quarter totals give every thread its offset and the channel's Gam_31 (the reference
+        // point rho) and Gam_end (rows past the chunk's end add zero), so the fast / exact decision is
+        // one barrier reduction.  Gam, rho and sig are made visible by the barrier of the V^T step.
         bool slow;
         {
-            const int nn = tk.nn, mr = (nn - 1) >> 1;
+            const int nn = tk.nn;
             const bool ok_in = mbar_wait(mbar_in, phase_in, WAIT_POLLS);
             if (!__syncthreads_and(ok_in)) { aborted = true; break; }
             phase_in ^= 1u;
             in_pending = false;
             if (tid < CH) sBeta[tid] = __uint_as_float(beta_bits << 16);
             const int gd = tid & (KD - 1), gq = tid >> 7;  // channel, quarter of the rows (16 each)
-            const float acc = gate_rows16_to<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias_in, rate, lower_bound,
-                                                   sGam, [&](int r) { return gidx(16 * gq + r, gd); });
-            // totals of quarters 0-2 go to scratch; later quarters add the ones before them
-            float* part = gq == 0 ? sRho : gq == 1 ? sSig : sSc2;
-            if (gq < 3) part[gd] = acc;
+            float gv[16];
+            const float acc = gate_rows16_regs<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias_in, rate,
+                                                     lower_bound, gv);
+            sPart[gq * KD + gd] = acc;
+            if (gq == 0) sPart[4 * KD + gd] = gv[0];
             __syncthreads();
-            if (gq > 0) {
-                float off = sRho[gd];
-                if (gq > 1) off += sSig[gd];
-                if (gq > 2) off += sSc2[gd];
-#pragma unroll 4
-                for (int r = 0; r < 16; ++r) sGam[gidx(16 * gq + r, gd)] += off;
-            }
-            __syncthreads();
-            if (tid < KD) {
-                const int d = tid;
-                const float g0 = sGam[gidx(0, d)], gm = sGam[gidx(mr, d)], gend = sGam[gidx(nn - 1, d)];
-                if (!(fmaxf(g0 - gm, gm - gend) <= SPAN_LIMIT)) atomicOr(sFlag, 1u);
-                sRho[d] = gm;
-                sSig[d] = gend;
-            }
-            __syncthreads();
-            slow = (*reinterpret_cast<volatile uint32_t*>(sFlag)) != 0;
-            if (tid < KD) {
-                const int d = tid;
-                float rho = sRho[d], sig = sSig[d];
+            const float p0 = sPart[gd], p1 = sPart[KD + gd], p2 = sPart[2 * KD + gd], p3 = sPart[3 * KD + gd];
+            const float g0 = sPart[4 * KD + gd];
+            const float s01 = p0 + p1, s012 = s01 + p2;
+            const float off = gq == 0 ? 0.f : gq == 1 ? p0 : gq == 2 ? s01 : s012;
+            const float gmid = s01, gend = s012 + p3;  // the values rows 31 and 63 receive below
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sGam[gidx(16 * gq + r, gd)] = gv[r] + off;
+            slow = __syncthreads_or(!(fmaxf(g0 - gmid, gmid - gend) <= SPAN_LIMIT)) != 0;
+            if (gq == 0) {
+                float rho = gmid, sig = gend;
                 if (slow) rho = 0.f;  // sig stays Gam_end: Kchk becomes Kend
                 else sig = rho;
-                sRho[d] = rho;
-                sSig[d] = sig;
+                sRho[gd] = rho;
+                sSig[gd] = sig;
                 float* rv = reinterpret_cast<float*>(rec + Rec::VEC);
-                rv[d] = __expf(rho);
-                rv[KD + d] = __expf(sig);
-                rv[2 * KD + d] = __expf(sGam[gidx(CH - 1, d)] - sig);
+                rv[gd] = __expf(rho);
+                rv[KD + gd] = __expf(sig);
+                rv[2 * KD + gd] = __expf(gend - sig);
             }
-            __syncthreads();
-            if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
         }
 
         // ---- V^T into VT from the staged v tile (value column vc, token quads q0 + 4 x) ---------------

@@ -62,10 +62,9 @@ struct TcLayout {
     static constexpr uint32_t BETA = VEC + 3072;  // [64]
     static constexpr uint32_t MBAR = BETA + 256;  // 8 B
     static constexpr uint32_t TBASE = MBAR + 8;   // 4 B
-    static constexpr uint32_t FLAG = TBASE + 4;   // 4 B
     static constexpr uint32_t VS = VEC + 4096;    // bf16 [64][128] staging of the next chunk's v tile
     static constexpr uint32_t BYTES = VS + 64 * VD * 2;
-    static_assert(FLAG + 4 <= VS, "vector region");
+    static_assert(TBASE + 4 <= VS, "vector region");
     // TMEM columns (all accumulators M = 128: TMEM lane = row)
     static constexpr int D4 = 0;     // state^T [v][d], 128 columns
     static constexpr int D3 = 128;   // [v][i]: 0-63 outputs, 64-127 -P
@@ -98,7 +97,6 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     float* sRT = reinterpret_cast<float*>(smem + L::GM);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
     const bf16* sG = reinterpret_cast<const bf16*>(smem + L::GM);  // g tile staging (bf16 [64][128])
-    uint32_t* sFlag = reinterpret_cast<uint32_t*>(smem + L::FLAG);
     const uint32_t s_base = smem_u32(smem);
     const uint32_t mbar = s_base + L::MBAR;
 
@@ -117,7 +115,6 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (tid == 0) mbar_init(mbar, 1);
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
     if (tid < KD) sFpend[tid] = 1.0f;
-    if (tid == 0) *sFlag = 0u;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
     {
@@ -170,7 +167,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     // its beta, the fast/exact decision and the per-channel vectors.  Uses sFpend, the pending state
     // factor the chunk starts from.  Returns whether the chunk takes the exact path.
     auto stage_gate = [&](int tc0) -> bool {
-        const int nn = min(CH, T - tc0), mr = (nn - 1) >> 1;
+        const int nn = min(CH, T - tc0);
         cp_async_wait_all();
         __syncthreads();
         if (tid < CH) sBeta[tid] = bload;
@@ -180,42 +177,38 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             const float bias = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * KD + gd] : 0.0f;
             const float acc =
                 gate_rows16_regs<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias, rate, lower_bound, gv);
-            // totals of quarters 0-2 to scratch (all three are rewritten below)
+            // quarter totals 0-2 and Gam_0 to scratch (vectors that are rewritten below)
             float* part = gq == 0 ? sFnext : gq == 1 ? sRho : sSig;
             if (gq < 3) part[gd] = acc;
+            if (gq == 0) sESig[gd] = gv[0];
         }
         __syncthreads();  // the g staging has been read: GM becomes Gam
+        // Quarter 3 knows the channel's Gam_31 (the reference point) and Gam_end (rows past the chunk's
+        // end add zero) from the totals; one barrier reduction makes the fast / exact decision.
+        bool bad = false;
+        float gmid = 0.f, gend = 0.f;
         {
-            float off = 0.f;
-            if (gq > 0) off += sFnext[gd];
-            if (gq > 1) off += sRho[gd];
-            if (gq > 2) off += sSig[gd];
+            const float p0 = sFnext[gd], p1 = sRho[gd], p2 = sSig[gd], g0 = sESig[gd];
+            const float s01 = p0 + p1, s012 = s01 + p2;
+            const float off = gq == 0 ? 0.f : gq == 1 ? p0 : gq == 2 ? s01 : s012;
 #pragma unroll
             for (int r = 0; r < 16; ++r) sGam[gidx(16 * gq + r, gd)] = gv[r] + off;
+            gmid = s01;
+            gend = s012 + gv[15];  // the value row 63 receives (quarter 3's own total is gv[15])
+            bad = gq == 3 && !(fmaxf(g0 - gmid, gmid - gend) <= SPAN_LIMIT);
         }
-        __syncthreads();
-        if (tid < KD) {
-            const int d = tid;
-            const float g0 = sGam[gidx(0, d)], gm = sGam[gidx(mr, d)], gend = sGam[gidx(nn - 1, d)];
-            if (!(fmaxf(g0 - gm, gm - gend) <= SPAN_LIMIT)) atomicOr(sFlag, 1u);
-            sRho[d] = gm;
-            sSig[d] = gend;
-        }
-        __syncthreads();
-        const bool slow_c = (*reinterpret_cast<volatile uint32_t*>(sFlag)) != 0;
-        if (tid < KD) {
-            const int d = tid;
-            float rho = sRho[d], sig = sSig[d];
+        const bool slow_c = __syncthreads_or(bad) != 0;
+        if (gq == 3) {
+            float rho = gmid, sig = gend;
             if (slow_c) rho = 0.f;  // sig stays Gam_end: Kchk becomes Kend
             else sig = rho;
-            sRho[d] = rho;
-            sSig[d] = sig;
-            sERho[d] = sFpend[d] * __expf(rho);  // D4 rescale: the pending factor and e^rho
-            sESig[d] = __expf(sig);
-            sFnext[d] = __expf(sGam[gidx(CH - 1, d)] - sig);  // pending per-key factor of D4 after this chunk
+            sRho[gd] = rho;
+            sSig[gd] = sig;
+            sERho[gd] = sFpend[gd] * __expf(rho);  // D4 rescale: the pending factor and e^rho
+            sESig[gd] = __expf(sig);
+            sFnext[gd] = __expf(gend - sig);  // pending per-key factor of D4 after this chunk
         }
         __syncthreads();
-        if (tid == 0) *sFlag = 0u;  // read by every thread above; reset for the next chunk
         return slow_c;
     };
     load_inputs(0);
