@@ -7,24 +7,27 @@
 //   Gam_i  in-chunk cumulative log decay, rho / sig per-channel reference points,
 //   Qhat_i = s q_i e^{Gam_i - rho},  Khat_i = k_i e^{Gam_i - rho},  Kchk_j = k_j e^{sig - Gam_j},
 //   A = masked Qhat Kchk^T,  R = masked beta Khat Kchk^T,  T = (I + R)^{-1},  Tb = T diag(beta).
-// With S~ = diag(e^rho) S_c (S_c the state entering the chunk) the chunk's results are
-//   E      = U - W S~        where U = Tb V and W = Tb Khat      (resolved delta errors)
-//   O      = Qhat S~ + A E                                        (chunk outputs)
-//   S_c+1  = diag(f) (diag(e^sig) S_c + Kchk^T E),   f = e^{Gam_end - sig}.
+// The factorised operands keep the in-chunk products within range; the state side needs the plain
+// ones, Wtil = W diag(e^rho) = Tb Ktil (Ktil_j = k_j e^{Gam_j}), Qtil = Qhat diag(e^rho) = s q e^{Gam}
+// and Kend = diag(f) Kchk^T = (k_j e^{Gam_end - Gam_j})^T with f = e^{Gam_end - sig}.  With S_c the
+// state entering the chunk the results are
+//   E      = U - Wtil S_c        where U = Tb V                   (resolved delta errors)
+//   O      = Qtil S_c + A E                                       (chunk outputs)
+//   S_c+1  = diag(e^{Gam_end}) S_c + Kend E.
 //
 // Pass 1 (chunk_prep_kernel, persistent, one chunk per CTA iteration, all chunks in parallel):
 // gate, Gam, the operands, M1 = [-Khat; Qhat] Kchk^T -> R and A, the triangular inverse, and
-// M7 = [A; Tb] [Khat^T; V^T]^T -> W and U, written to a per-chunk record in the workspace:
-//   WQ  [W; Qhat]  128 x 128 tf32 in the K-major tiling of kda_tc_ptx.cuh (the A operand of M8)
-//   KA  [Kchk^T; A] 192 x 64 tf32, same tiling (A operands of M9 and M10)
+// M7 = [Tb; Tb] [Khat^T; V^T]^T -> W and U, written to a per-chunk record in the workspace:
+//   WQ  [Wtil; Qtil]  128 x 128 tf32 in the K-major tiling of kda_tc_ptx.cuh (the A operand of M8)
+//   KA  [Kend; A]     192 x 64 tf32, same tiling (A operands of M9 and M10)
 //   UT  U^T, fp32 rows of 64 (one per value column)
-//   VEC e^rho, e^sig, f (fp32, 128 each)
+//   VEC e^{Gam_end} (fp32, 128)
 // Pass 2 (chunk_state_kernel, one CTA per (pair, block of VB value columns), chunks in order):
 // the state slice S_c[:, block] lives in registers (thread d owns key row d, exact fp32);
-// per chunk, with tf32(S~)^T staged in shared memory as a B operand:
-//   M8   D1 = [W; Qhat] S~                -> W S~ (rows 0-63), Qhat S~ (rows 64-127)
-//   E    = U - W S~  on the CUDA cores, staged as a tf32 B operand
-//   M10  D2 = Kchk^T E                    -> S_c+1 = f (e^sig S_c + D2), in registers
+// per chunk, with tf32(S_c)^T staged in shared memory as a B operand:
+//   M8   D1 = [Wtil; Qtil] S_c           -> Wtil S_c (rows 0-63), Qtil S_c (rows 64-127)
+//   E    = U - Wtil S_c  on the CUDA cores, staged as a tf32 B operand
+//   M10  D2 = Kend E                      -> S_c+1 = e^{Gam_end} S_c + D2, in registers
 //   M9   D1[64:] += A E                   -> O  (issued after M10 with its own commit: off the
 //                                             chunk-to-chunk path)
 // Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
@@ -47,9 +50,9 @@ struct Rec {
     static constexpr uint32_t KA = 65536;    // [192][64] tf32 tiles
     static constexpr uint32_t KA_BYTES = 49152;
     static constexpr uint32_t UT = 114688;   // [128][64] fp32 rows
-    static constexpr uint32_t VEC = 147456;  // 3 x [128] fp32
+    static constexpr uint32_t VEC = 147456;  // [128] fp32 e^{Gam_end}, then padding
     static constexpr uint32_t BYTES = 149504;
-    static_assert(VEC + 3 * 512 <= BYTES && BYTES % 256 == 0, "record layout");
+    static_assert(VEC + 512 <= BYTES && BYTES % 256 == 0, "record layout");
 };
 
 struct PrepLayout {
@@ -66,8 +69,9 @@ struct PrepLayout {
     static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
     static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)
     static constexpr uint32_t VEC = 229376;
-    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024;
-    static constexpr uint32_t MBAR = VEC + 1280, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8;
+    static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024, ERHO = VEC + 1280, FEND = VEC + 1792;
+    static constexpr uint32_t MBAR = VEC + 2304, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8;
+    static constexpr uint32_t QT = KA + 32768;    // record Qtil staging, in the Tb rows (free until the inverse)
     static constexpr uint32_t PART = KA + 32768;  // gate: per-channel quarter totals and Gam_0 (5 x [128] fp32),
                                                   //   in the Tb rows, which are free until the inverse
     static constexpr uint32_t STG_G = X1, STG_V = X1 + 16384, STG_Q = X1 + 32768, STG_K = X1 + 49152;
@@ -82,10 +86,10 @@ template <int VB>
 struct StateLayout {
     static constexpr int NKA = VB <= 32 ? 2 : 1;              // KA / U buffers
     static constexpr uint32_t WQ = 0;                          // [128][128]
-    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], U^T [VB][64], VEC
+    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], U^T [VB][64], e^{Gam_end}
     static constexpr uint32_t UT_OFF = Rec::KA_BYTES, VEC_OFF = Rec::KA_BYTES + VB * 256;
-    static constexpr uint32_t KA_STRIDE = VEC_OFF + 3 * 512;
-    static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S~^T [VB][128]   (B of M8)
+    static constexpr uint32_t KA_STRIDE = VEC_OFF + 512;
+    static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S^T [VB][128]    (B of M8)
     static constexpr uint32_t EOP = SOP + VB * 128 * 4;        // tf32 E^T  [VB][64]    (B of M9, M10)
     static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1], out
     static constexpr uint32_t TBASE = MBAR + 40;
@@ -138,6 +142,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     float* sSig = reinterpret_cast<float*>(smem + L::SIG);
     float* sPart = reinterpret_cast<float*>(smem + L::PART);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
+    float* sERho = reinterpret_cast<float*>(smem + L::ERHO);
+    float* sFend = reinterpret_cast<float*>(smem + L::FEND);
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
@@ -230,10 +236,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 else sig = rho;
                 sRho[gd] = rho;
                 sSig[gd] = sig;
-                float* rv = reinterpret_cast<float*>(rec + Rec::VEC);
-                rv[gd] = __expf(rho);
-                rv[KD + gd] = __expf(sig);
-                rv[2 * KD + gd] = __expf(gend - sig);
+                sERho[gd] = __expf(rho);
+                sFend[gd] = __expf(gend - sig);
+                reinterpret_cast<float*>(rec + Rec::VEC)[gd] = __expf(gend);
             }
         }
 
@@ -273,13 +278,13 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
         }
 
-        // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK, Kchk^T -> KA rows 0-127 -----------------------
+        // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK; record parts Kend -> KA rows 0-127, Qtil -> QT -----
         uint32_t kh[2][8];  // tf32 bits of -Khat (rotated), kept for Khat^T once Gam is no longer needed
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
             const int u = tid + NT * it;
             const int i = ((u >> 7) << 3) + (u & 7), d8 = (u >> 3) & 15;
-            float qf[8], kf[8], gf[8], rf[8], sf[8];
+            float qf[8], kf[8], gf[8], rf[8], sf[8], ef[8], ff[8];
             bf16x8_to_f32(qr[it], qf);
             bf16x8_to_f32(kr[it], kf);
             *reinterpret_cast<float4*>(gf) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8));
@@ -288,13 +293,20 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             *reinterpret_cast<float4*>(rf + 4) = *reinterpret_cast<const float4*>(sRho + 8 * d8 + 4);
             *reinterpret_cast<float4*>(sf) = *reinterpret_cast<const float4*>(sSig + 8 * d8);
             *reinterpret_cast<float4*>(sf + 4) = *reinterpret_cast<const float4*>(sSig + 8 * d8 + 4);
-            uint32_t wq_[8], wc_[8];
+            *reinterpret_cast<float4*>(ef) = *reinterpret_cast<const float4*>(sERho + 8 * d8);
+            *reinterpret_cast<float4*>(ef + 4) = *reinterpret_cast<const float4*>(sERho + 8 * d8 + 4);
+            *reinterpret_cast<float4*>(ff) = *reinterpret_cast<const float4*>(sFend + 8 * d8);
+            *reinterpret_cast<float4*>(ff + 4) = *reinterpret_cast<const float4*>(sFend + 8 * d8 + 4);
+            uint32_t wq_[8], wc_[8], qt[8], ke[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 const float e1 = __expf(gf[t] - rf[t]), e2 = __expf(sf[t] - gf[t]);
-                wq_[t] = to_tf32(scale * qf[t] * e1);
+                const float qh = scale * qf[t] * e1, kc = kf[t] * e2;
+                wq_[t] = to_tf32(qh);
+                qt[t] = to_tf32(qh * ef[t]);
                 kh[it][t] = to_tf32(-kf[t] * e1);
-                wc_[t] = to_tf32(kf[t] * e2);
+                wc_[t] = to_tf32(kc);
+                ke[t] = to_tf32(kc * ff[t]);
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -305,19 +317,21 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                     make_uint4(wq_[4 * hh], wq_[4 * hh + 1], wq_[4 * hh + 2], wq_[4 * hh + 3]);
                 *reinterpret_cast<uint4*>(smem + L::CK + cm_off(i, d, KD)) =
                     make_uint4(wc_[4 * hh], wc_[4 * hh + 1], wc_[4 * hh + 2], wc_[4 * hh + 3]);
+                *reinterpret_cast<uint4*>(smem + L::QT + cm_off(i, d, KD)) =
+                    make_uint4(qt[4 * hh], qt[4 * hh + 1], qt[4 * hh + 2], qt[4 * hh + 3]);
             }
-            // Kchk^T: lanes that share a bank (same i & 3) take different d of their group of 8
-            rotate_groups8(wc_, rot);
+            // Kend (transposed): lanes that share a bank (same i & 3) take different d of their group of 8
+            rotate_groups8(ke, rot);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) = wc_[t];
+                *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) = ke[t];
             rotate_groups8(kh[it], rot);  // stored transposed the same way below
         }
         fence_proxy_async();
         cta_sync_tc();
-        if (tid == 32) {  // Qhat and Kchk^T are final: their record stores run while M1 does
-            bulk_store(rec + Rec::WQ + 32768, s_base + L::X1 + 32768, 32768);  // W goes straight out later
-            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);  // A goes straight to the record later
+        if (tid == 32) {  // Qtil and Kend are final: their record stores run while M1 does
+            bulk_store(rec + Rec::WQ + 32768, s_base + L::QT, 32768);  // Wtil goes straight out later
+            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);         // A goes straight to the record later
             bulk_commit();
         }
 
@@ -415,6 +429,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 and 192-255 ----------
         tri_inverse_diag16(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
+        if (tid == 32) bulk_wait_read();  // the Qtil store has read QT before Tb overwrites it
         tri_inverse_step32(sRT, sX, tid);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
@@ -454,13 +469,17 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             uint32_t r0[32];
             tmem_ld32(taddr(tmem, 32 * wq, (wq < 2 ? 0 : 128) + 32 * wc), r0);
             tmem_wait_ld();
-            if (wq < 2) {  // W -> record WQ rows 0-63 (tf32, operand tiling)
+            if (wq < 2) {  // Wtil = W diag(e^rho) -> record WQ rows 0-63 (tf32, operand tiling)
                 unsigned char* rw = rec + Rec::WQ;
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 er = *reinterpret_cast<const float4*>(sERho + 32 * wc + 4 * c4);
                     *reinterpret_cast<uint4*>(rw + cm_off(i, 32 * wc + 4 * c4, KD)) =
-                        make_uint4(to_tf32(__uint_as_float(r0[4 * c4])), to_tf32(__uint_as_float(r0[4 * c4 + 1])),
-                                   to_tf32(__uint_as_float(r0[4 * c4 + 2])), to_tf32(__uint_as_float(r0[4 * c4 + 3])));
+                        make_uint4(to_tf32(er.x * __uint_as_float(r0[4 * c4])),
+                                   to_tf32(er.y * __uint_as_float(r0[4 * c4 + 1])),
+                                   to_tf32(er.z * __uint_as_float(r0[4 * c4 + 2])),
+                                   to_tf32(er.w * __uint_as_float(r0[4 * c4 + 3])));
+                }
             } else {  // U^T (fp32, row = value column) -> CK region, free once Tb was built
                 float* ut = reinterpret_cast<float*>(smem + L::CK);
 #pragma unroll
@@ -549,7 +568,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         mbar_expect_tx(bar, L::KA_STRIDE);
         bulk_load(s_base + L::ka(buf), rec(c) + Rec::KA, Rec::KA_BYTES, bar);
         bulk_load(s_base + L::ka(buf) + L::UT_OFF, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
-        bulk_load(s_base + L::ka(buf) + L::VEC_OFF, rec(c) + Rec::VEC, 3 * 512, bar);
+        bulk_load(s_base + L::ka(buf) + L::VEC_OFF, rec(c) + Rec::VEC, 512, bar);
         pending |= 2u << buf;
     };
     // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32
@@ -564,10 +583,6 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         s[j + 2] = x.z;
         s[j + 3] = x.w;
     }
-    // per-key vectors of the chunk held in KA buffer `buf`: e^rho, e^sig, f
-    auto vec = [&](int buf, int which) {
-        return reinterpret_cast<const float*>(smem + L::ka(buf) + L::VEC_OFF)[which * KD + d];
-    };
     // the chunk records are written by the preceding prep kernel: wait for it (a no-op unless this
     // grid was launched as its programmatic dependent; the prep CTAs release it once their records
     // are complete, so only the launch itself overlaps their tail)
@@ -577,11 +592,11 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         load_ka(0, 0);
         if (L::NKA == 2 && NC > 1) load_ka(1, 1);
     }
-    // tf32(e^rho S)^T into the B operand of M8; lanes sharing a bank store different columns
-    auto write_sop = [&](float er) {
+    // tf32(S)^T into the B operand of M8; lanes sharing a bank store different columns
+    auto write_sop = [&]() {
         uint32_t w[HALF];
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) w[j] = to_tf32(er * s[j]);
+        for (int j = 0; j < HALF; ++j) w[j] = to_tf32(s[j]);
         rotate_groups8(w, rot);
 #pragma unroll
         for (int j = 0; j < HALF; ++j)
@@ -589,19 +604,13 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     };
     uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0, ph_out = 0;
     bool aborted = false;
-    {
-        const bool ok = mbar_wait(bar_ka0, 0, WAIT_POLLS);  // chunk 0's KA group holds its vectors
-        if (!__syncthreads_and(ok)) aborted = true;
-    }
-    if (!aborted) write_sop(vec(0, 0));
+    write_sop();
     fence_proxy_async();
     cta_sync_tc();
     for (int c = 0; c < NC && !aborted; ++c) {
         const int buf = (L::NKA == 2) ? (c & 1) : 0;
         const int n = min(CH, T - c * CH);
-        float er_n = 0.f;  // with one KA buffer the next chunk's e^rho comes from the record directly
-        if (L::NKA == 1 && c + 1 < NC) er_n = __ldg(reinterpret_cast<const float*>(rec(c + 1) + Rec::VEC) + d);
-        // ---- M8: D1 = [W; Qhat] S~ ------------------------------------------------------------
+        // ---- M8: D1 = [Wtil; Qtil] S ------------------------------------------------------------
         bool ok = true;
         if (tid == 0) {
             ok = mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
@@ -620,13 +629,13 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         ph_wq ^= 1u;
         ph_mma ^= 1u;
         ph_ka ^= 1u << buf;
-        // this chunk's e^sig and f, read before a single KA buffer is refilled below
-        const float es = vec(buf, 1), ef = vec(buf, 2);
+        // this chunk's e^{Gam_end}, read before a single KA buffer is refilled below
+        const float eg = reinterpret_cast<const float*>(smem + L::ka(buf) + L::VEC_OFF)[d];
         if (tid == 0) {
             pending &= ~(2u << buf);
             if (c + 1 < NC) load_wq(c + 1);  // M8 has read WQ
         }
-        // ---- E = U - W S~ (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
+        // ---- E = U - Wtil S (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
         const uint32_t ka = s_base + L::ka(buf);
         if (wq < 2) {
             const int j = d;
@@ -643,7 +652,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         }
         fence_proxy_async();
         cta_sync_tc();
-        // ---- M10: D2 = Kchk^T E (the state side), then M9: D1[64:] += A E (the outputs), each with its
+        // ---- M10: D2 = Kend E (the state side), then M9: D1[64:] += A E (the outputs), each with its
         //      own commit, so that the state update starts after M10 while M9 still runs -------------
         if (tid == 0) {
             gemm_tf32(tmem + L::D2, ka, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
@@ -657,13 +666,13 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         fence_after_sync();
         if (!__syncthreads_and(ok)) { aborted = true; break; }
         ph_mma ^= 1u;
-        // ---- state: S = f (e^sig S + D2) --------------------------------------------------------
+        // ---- state: S = e^{Gam_end} S + D2 --------------------------------------------------------
         {
             uint32_t r[HALF];
             tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D2 + c0), r);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < HALF; ++j) s[j] = ef * fmaf(es, s[j], __uint_as_float(r[j]));
+            for (int j = 0; j < HALF; ++j) s[j] = fmaf(eg, s[j], __uint_as_float(r[j]));
         }
         // ---- outputs (rows 64-127 of D1: lane quarters 2, 3), once M9 is done; thread 0 waits for it
         //      too before a KA buffer M9 reads is refilled -----------------------------------------
@@ -695,16 +704,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             }
         }
         if (L::NKA == 1 && tid == 0 && ok_out && c + 1 < NC) load_ka(c + 1, 0);
-        // ---- S~ of the next chunk ---------------------------------------------------------------
-        if (c + 1 < NC) {
-            if (L::NKA == 2) {  // the next chunk's KA group (loaded a chunk ago) holds its e^rho
-                const int nb = buf ^ 1;
-                const bool okn = mbar_wait(bar_ka0 + 8 * nb, (ph_ka >> nb) & 1u, WAIT_POLLS) && ok_out;
-                if (!__syncthreads_and(okn)) { aborted = true; break; }
-                er_n = vec(nb, 0);
-            }
-            write_sop(er_n);
-        }
+        // ---- the next chunk's S operand --------------------------------------------------------
+        if (c + 1 < NC) write_sop();
         fence_proxy_async();
         fence_before_sync();
         if (!__syncthreads_and(ok_out)) { aborted = true; break; }

@@ -13,7 +13,8 @@
 // not accurate enough for the stated tolerance once the output itself is rounded to bf16.
 //
 // Decay factors.  Products of the form x_i . (y_j e^{Gam_i - Gam_j}) are factorised around a
-// per-channel reference rho = Gam_m (m the middle token of the chunk):
+// per-channel reference rho = Gam_31 (the middle row of a full chunk; for a chunk of at most 32
+// tokens, its last row):
 //   Qhat_i = s q_i e^{Gam_i - rho},  Khat_i = k_i e^{Gam_i - rho},  Kchk_j = k_j e^{sig - Gam_j},
 // with sig = rho, so [Qhat; -Khat] Kchk^T gives A and -R/beta in one M = 128 MMA.  That is exact as
 // long as no factor overflows, which holds when max(Gam_0 - rho, rho - Gam_end) <= 40 on every
