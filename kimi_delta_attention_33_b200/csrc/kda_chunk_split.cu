@@ -56,15 +56,14 @@ struct Rec {
 };
 
 struct PrepLayout {
-    static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1); Qhat is the record's WQ rows
-                                             //   64-127; once M1 is done (and Qhat's record store has read
-                                             //   it) X1 stages the next chunk's input tiles, bf16 [64][128]
-                                             //   each: g, v (plain rows), q, k (two 64-column halves each,
-                                             //   rows of 128 bytes with the 128-byte swizzle)
+    static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1); once M1 is done X1 stages
+                                             //   the next chunk's input tiles, bf16 [64][128] each: g, v
+                                             //   (plain rows), q, k (two 64-column halves each, rows of 128
+                                             //   bytes with the 128-byte swizzle)
     static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling
                                              //   scratch; then U^T [128][64] fp32 (record UT)
     static constexpr uint32_t XS = CK + 64 * RP * 4;
-    static constexpr uint32_t KA = 98304;    // [256][64]: Kchk^T rows 0-127 (record KA, first part),
+    static constexpr uint32_t KA = 98304;    // [256][64]: Kend^T rows 0-127 (record KA, first part),
                                              //   Tb twice in rows 128-255 (A of M7)
     static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
     static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)

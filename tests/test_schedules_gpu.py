@@ -117,6 +117,26 @@ def test_strong_decay_takes_exact_path(schedule):
     assert rel_err(S, S_ref) <= TOL[w.dtype]
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("c_last", [-1.75, -2.5])
+def test_short_last_chunk_decay_spans(schedule, c_last):
+    # a 20-token last chunk with a constant log-decay per token: its span Gam_0 - Gam_end is
+    # 19 |c_last| = 33.25 (factorised path, reference point = its last row) or 47.5 (exact path);
+    # the full first chunk decays gently (-0.5 per token)
+    w = _wl(T=84)
+    x = make_inputs(w)
+    g_log = torch.full((w.B, w.T, w.HV, 128), -0.5, dtype=torch.float32)
+    g_log[:, 64:] = c_last
+    x2 = dict(x, g=g_log.to(torch.bfloat16))
+    w2 = Workload(96, "short chunk", w.B, w.T, w.H, w.HV, 128, 128, 64, torch.bfloat16, GATE_NONE, 0.0, None, 0.0, 0.0,
+                  0.02)
+    o, S = _run(w2, to_dev(x2), schedule)
+    o_ref, S_ref = oracle.forward(x2["q"], x2["k"], x2["v"], x2["g"], x2["beta"], None, None, x2["S0"],
+                                  gate_mode=GATE_NONE)
+    assert rel_err(o, o_ref) <= TOL[w.dtype]
+    assert rel_err(S, S_ref) <= TOL[w.dtype]
+
+
 def test_schedules_agree_with_each_other():
     w = _wl(B=2, T=333, H=2, HV=6)
     xd = to_dev(make_inputs(w))
