@@ -36,28 +36,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
     }
 }
 
-// The same for 16 rows (CTAs with four threads per key channel).
-template <int MODE, typename Idx>
-__device__ __forceinline__ float gate_rows16_to(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
-                                                float lower_bound, float* dst, Idx idx) {
-    float acc = 0.f;
-#pragma unroll
-    for (int r0 = 0; r0 < 16; r0 += 8) {
-        float x[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float gr = __bfloat162float(col[(r0 + r) * stride]);
-            x[r] = (r0 + r < nn) ? gate_value_fast(gr, bias, rate, MODE, lower_bound) : 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            acc += x[r];
-            dst[idx(r0 + r)] = acc;
-        }
-    }
-    return acc;
-}
-
 // Gate values of one key channel for 16 consecutive rows as their running sum in registers.
 template <int MODE>
 __device__ __forceinline__ float gate_rows16_regs(const __nv_bfloat16* col, int stride, int nn, float bias, float rate,
@@ -74,14 +52,6 @@ __device__ __forceinline__ float gate_rows16_regs(const __nv_bfloat16* col, int 
         gv[r] = acc;
     }
     return acc;
-}
-
-__device__ __forceinline__ float gate_rows16_regs(int mode, const __nv_bfloat16* col, int stride, int nn, float bias,
-                                                  float rate, float lower_bound, float (&gv)[16]) {
-    if (mode == KDA_GATE_SAFE) return gate_rows16_regs<KDA_GATE_SAFE>(col, stride, nn, bias, rate, lower_bound, gv);
-    if (mode == KDA_GATE_STANDARD)
-        return gate_rows16_regs<KDA_GATE_STANDARD>(col, stride, nn, bias, rate, lower_bound, gv);
-    return gate_rows16_regs<KDA_GATE_NONE>(col, stride, nn, bias, rate, lower_bound, gv);
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
