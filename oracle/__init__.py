@@ -19,6 +19,9 @@ What it computes (page title, then section):
 * ``dplr``        -- DeltaNet-family digest, "diagonal-low-rank transition": the
   same recurrence through explicit dense K x K transition matrices, a third
   independent form used only to pin ``recurrent``.
+* ``backward`` (module ``oracle.backward``) -- the reverse mode of ``forward``,
+  derived step by step from the recurrence and the gates, pinned by central
+  finite differences of ``forward``: the reference for a backward pass.
 
 Every pinned property is listed in the tests; nothing here is "parity
 unpinned".  The compiled part lives in ``kda_oracle.c`` (plain C, float64,
