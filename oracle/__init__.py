@@ -21,7 +21,9 @@ What it computes (page title, then section):
   independent form used only to pin ``recurrent``.
 * ``backward`` (module ``oracle.backward``) -- the reverse mode of ``forward``,
   derived step by step from the recurrence and the gates, pinned by central
-  finite differences of ``forward``: the reference for a backward pass.
+  finite differences of ``forward``: the reference for a backward pass; and
+  ``chunkwise_backward``, the reverse mode of the chunkwise equations, pinned
+  against it.
 
 Every pinned property is listed in the tests; nothing here is "parity
 unpinned".  The compiled part lives in ``kda_oracle.c`` (plain C, float64,

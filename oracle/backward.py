@@ -120,3 +120,139 @@ def backward(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, dO=None, dS_T=
         out["dg_raw"], out["ddt_bias"], out["dA_log"] = gate_backward(g, A_log, dt_bias, out["dg"], mode=gate_mode,
                                                                       lower_bound=lower_bound)
     return out
+
+
+def chunkwise_backward(q, k, v, g, beta, S0=None, dO=None, dS_T=None, *, chunk=64, scale=None):
+    """The same gradients as ``recurrent_backward``, computed chunk by chunk in the form a chunked
+    backward pass uses: the reverse mode of the chunkwise equations (DeltaNet-family digest,
+    "Chunkwise KDA"), with every decay an explicit exponential of a prefix-sum difference.
+
+    Per chunk of n tokens entering with state S (Gam_i = sum_{m<=i} g_m, e = exp):
+        Ebar_i = beta_i (v_i - sum_d k_id e^{Gam_id} S[d,:])
+        rho_ij = beta_i sum_d k_id k_jd e^{Gam_id - Gam_jd}              (j < i)
+        E_i    = Ebar_i - sum_{j<i} rho_ij E_j
+        a_ij   = scale sum_d q_id k_jd e^{Gam_id - Gam_jd}               (j <= i)
+        O_i    = scale sum_d q_id e^{Gam_id} S[d,:] + sum_{j<=i} a_ij E_j
+        S'[d,:] = e^{Gam_end,d} S[d,:] + sum_j k_jd e^{Gam_end,d - Gam_jd} E_j
+    Reverse, given dO and dS' (the gradient with respect to S'):
+        dE_j  = sum_{i>=j} a_ij dO_i + sum_d k_jd e^{Gam_end,d - Gam_jd} dS'[d,:]
+        lam   = (I + rho)^{-T} dE          (back substitution; lam is the gradient of Ebar)
+        drho_ij = -lam_i . E_j,  da_ij = dO_i . E_j
+    and every factor above gives its q, k, beta, v, Gam and S terms; dg is the reverse cumulative
+    sum of dGam within the chunk, and the S terms are the next (earlier) chunk's dS'.
+    """
+    q, k, v, g, beta, S0, dO, dS_T = (_f64(x) for x in (q, k, v, g, beta, S0, dO, dS_T))
+    B, T, H, HV, K, V = _shapes(q, v)
+    G = HV // H
+    if scale is None:
+        scale = 1.0 / np.sqrt(K)
+    if dO is None:
+        dO = np.zeros((B, T, HV, V))
+    dq, dk = np.zeros_like(q), np.zeros_like(k)
+    dv, dg, dbeta = np.zeros_like(v), np.zeros_like(g), np.zeros_like(beta)
+    dS0 = np.zeros((B, HV, K, V))
+    starts = list(range(0, T, chunk))
+    for b in range(B):
+        for hv in range(HV):
+            h = hv // G
+            # forward over chunks, keeping the state entering each one
+            S = np.zeros((K, V)) if S0 is None else S0[b, hv].copy()
+            entering = []
+            for c0 in starts:
+                n = min(chunk, T - c0)
+                qc, kc, vc = q[b, c0:c0 + n, h], k[b, c0:c0 + n, h], v[b, c0:c0 + n, hv]
+                bc = beta[b, c0:c0 + n, hv]
+                Gam = np.cumsum(g[b, c0:c0 + n, hv], axis=0)
+                entering.append(S.copy())
+                Ebar = bc[:, None] * (vc - (kc * np.exp(Gam)) @ S)
+                E = np.zeros((n, V))
+                for i in range(n):
+                    acc = Ebar[i].copy()
+                    for j in range(i):
+                        rho = bc[i] * np.sum(kc[i] * kc[j] * np.exp(Gam[i] - Gam[j]))
+                        acc -= rho * E[j]
+                    E[i] = acc
+                gend = Gam[n - 1]
+                S = np.exp(gend)[:, None] * S + (kc * np.exp(gend - Gam)).T @ E
+            # reverse over chunks
+            dSn = np.zeros((K, V)) if dS_T is None else dS_T[b, hv].copy()   # gradient of S'
+            for ci in range(len(starts) - 1, -1, -1):
+                c0 = starts[ci]
+                n = min(chunk, T - c0)
+                S = entering[ci]
+                qc, kc, vc = q[b, c0:c0 + n, h], k[b, c0:c0 + n, h], v[b, c0:c0 + n, hv]
+                bc = beta[b, c0:c0 + n, hv]
+                dOc = dO[b, c0:c0 + n, hv]
+                Gam = np.cumsum(g[b, c0:c0 + n, hv], axis=0)
+                gend = Gam[n - 1]
+                # recompute the chunk's forward quantities
+                eG = np.exp(Gam)                                   # [n, K]
+                Kt = kc * eG                                       # k_i e^{Gam_i}
+                Ebar = bc[:, None] * (vc - Kt @ S)
+                rho = np.zeros((n, n))
+                a = np.zeros((n, n))
+                for i in range(n):
+                    for j in range(n):
+                        f = np.exp(Gam[i] - Gam[j])
+                        if j < i:
+                            rho[i, j] = bc[i] * np.sum(kc[i] * kc[j] * f)
+                        if j <= i:
+                            a[i, j] = scale * np.sum(qc[i] * kc[j] * f)
+                E = np.zeros((n, V))
+                for i in range(n):
+                    E[i] = Ebar[i] - rho[i, :i] @ E[:i]
+                Kend = kc * np.exp(gend - Gam)                     # k_j e^{Gam_end - Gam_j}
+                # gradients of E, then of Ebar (back substitution through the unit lower solve)
+                dE = a.T @ dOc + Kend @ dSn
+                lam = np.zeros((n, V))
+                for j in range(n - 1, -1, -1):
+                    lam[j] = dE[j] - rho[j + 1:, j] @ lam[j + 1:]
+                dGam = np.zeros((n, K))
+                dkc = np.zeros((n, K))
+                dqc = np.zeros((n, K))
+                dS = np.exp(gend)[:, None] * dSn                  # from e^{Gam_end} S
+                # O_i's direct term scale q_i e^{Gam_i} S
+                QS_grad = dOc @ S.T                                # [n, K]: S[d,:] . dO_i
+                dqc += scale * eG * QS_grad
+                dGam += scale * qc * eG * QS_grad
+                dS += scale * (qc * eG).T @ dOc
+                # S' = e^{Gam_end} S + Kend^T E
+                SdS = np.sum(S * dSn, axis=1)                       # S[d,:] . dS'[d,:]
+                dGam[n - 1] += np.exp(gend) * SdS
+                EdS = E @ dSn.T                                    # [n, K]: E_j . dS'[d,:]
+                dkc += np.exp(gend - Gam) * EdS
+                dGam[n - 1] += np.sum(Kend * EdS, axis=0)
+                dGam -= Kend * EdS
+                # Ebar_i = beta_i (v_i - Kt_i S)
+                dv[b, c0:c0 + n, hv] = bc[:, None] * lam
+                dbeta[b, c0:c0 + n, hv] += np.sum((vc - Kt @ S) * lam, axis=1)
+                SL = lam @ S.T                                     # [n, K]: S[d,:] . lam_i
+                dkc -= bc[:, None] * eG * SL
+                dGam -= bc[:, None] * kc * eG * SL
+                dS -= (bc[:, None] * Kt).T @ lam
+                # rho and a
+                drho = -(lam @ E.T)                                # drho_ij = -lam_i . E_j
+                da = dOc @ E.T                                     # da_ij = dO_i . E_j
+                for i in range(n):
+                    for j in range(i + 1):
+                        f = np.exp(Gam[i] - Gam[j])
+                        if j < i:
+                            w = drho[i, j]
+                            dbeta[b, c0 + i, hv] += w * np.sum(kc[i] * kc[j] * f)
+                            t_ = w * bc[i] * kc[i] * kc[j] * f
+                            dkc[i] += w * bc[i] * kc[j] * f
+                            dkc[j] += w * bc[i] * kc[i] * f
+                            dGam[i] += t_
+                            dGam[j] -= t_
+                        w = da[i, j]
+                        t_ = w * scale * qc[i] * kc[j] * f
+                        dqc[i] += w * scale * kc[j] * f
+                        dkc[j] += w * scale * qc[i] * f
+                        dGam[i] += t_
+                        dGam[j] -= t_
+                dg[b, c0:c0 + n, hv] = np.cumsum(dGam[::-1], axis=0)[::-1]
+                dq[b, c0:c0 + n, h] += dqc
+                dk[b, c0:c0 + n, h] += dkc
+                dSn = dS
+            dS0[b, hv] = dSn
+    return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dbeta": dbeta, "dS0": dS0}

@@ -4,7 +4,8 @@ The reverse mode is derived, not printed on the pages, so it is pinned to someth
 itself: central finite differences of the forward oracle (which has its own pins), and two
 structural facts of the recurrence -- outputs and final state are linear in (v, S0), so their
 gradient with respect to v does not depend on v; and with beta = 0 nothing is written, so v has
-no effect at all.
+no effect at all.  The chunkwise reverse mode, written separately from the chunk equations, must
+agree with the token-by-token one for every chunk length, ragged tails included.
 """
 import numpy as np
 import pytest
@@ -98,3 +99,39 @@ def test_nothing_written_means_no_value_gradient():
     x["beta"] = np.zeros_like(x["beta"])
     gr = obw.recurrent_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], dO, dS_T)
     assert np.all(gr["dv"] == 0.0)
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 7, 16, 70])
+@pytest.mark.parametrize("H,HV", [(1, 2), (2, 2)])
+def test_chunkwise_reverse_mode_equals_recurrent(chunk, H, HV):
+    # the chunked form a backward kernel would follow, against the token-by-token reverse mode:
+    # ragged last chunk (T = 19), a chunk longer than the sequence, GVA
+    rng = np.random.default_rng(100 + chunk + HV)
+    B, T, K, V = 2, 19, 4, 3
+    q = rng.standard_normal((B, T, H, K))
+    k = rng.standard_normal((B, T, H, K))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, HV, V))
+    g = -rng.uniform(0.02, 1.5, (B, T, HV, K))
+    beta = rng.uniform(0.05, 0.95, (B, T, HV))
+    S0 = rng.standard_normal((B, HV, K, V))
+    dO = rng.standard_normal((B, T, HV, V))
+    dS_T = rng.standard_normal((B, HV, K, V))
+    ref = obw.recurrent_backward(q, k, v, g, beta, S0, dO, dS_T)
+    got = obw.chunkwise_backward(q, k, v, g, beta, S0, dO, dS_T, chunk=chunk)
+    for key in ref:
+        np.testing.assert_allclose(got[key], ref[key], rtol=1e-10, atol=1e-12 * np.abs(ref[key]).max(),
+                                   err_msg=key)
+
+
+def test_chunkwise_reverse_mode_without_state_terms():
+    # no initial state and no final-state gradient: only the outputs drive the gradients
+    rng = np.random.default_rng(4)
+    B, T, H, HV, K, V = 1, 10, 1, 1, 3, 2
+    q, k = rng.standard_normal((B, T, H, K)), rng.standard_normal((B, T, H, K))
+    v, g = rng.standard_normal((B, T, HV, V)), -rng.uniform(0.1, 0.8, (B, T, HV, K))
+    beta, dO = rng.uniform(0.1, 0.9, (B, T, HV)), rng.standard_normal((B, T, HV, V))
+    ref = obw.recurrent_backward(q, k, v, g, beta, None, dO, None)
+    got = obw.chunkwise_backward(q, k, v, g, beta, None, dO, None, chunk=4)
+    for key in ref:
+        np.testing.assert_allclose(got[key], ref[key], rtol=1e-10, atol=1e-13, err_msg=key)
