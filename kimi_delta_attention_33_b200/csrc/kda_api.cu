@@ -70,6 +70,15 @@ constexpr long long kTwoPassMaxPairs = 96;
 // on the CUDA-core kernel in fp32.
 bool split_shape(int K, int V, int chunk) { return K == 128 && V == 128 && chunk == 64; }
 
+// Sizes the two-pass schedule takes: at most kTwoPassMaxPairs pairs; fewer than 2^30 chunks in all (the
+// prep kernel counts its tasks in an int); the tensor maps of its input copies need a token stride
+// (heads x 256 bytes) times T below 2^40 bytes.
+bool two_pass_sizes(int B, int T, int HV) {
+    const long long pairs = (long long)B * HV;
+    return pairs <= kTwoPassMaxPairs && pairs * (((long long)T + 63) / 64) < (1ll << 30) &&
+           (long long)T * HV * 256 < (1ll << 40);
+}
+
 }  // namespace
 
 namespace kda {
@@ -104,9 +113,7 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk) {
     if (!sizes_ok(B, T, H, HV, K, V, chunk)) return 0;
-    if (split_shape(K, V, chunk) && (long long)B * HV <= kTwoPassMaxPairs &&
-        (long long)B * HV * ((T + 63) / 64) < (1ll << 30))
-        return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
+    if (split_shape(K, V, chunk) && two_pass_sizes(B, T, HV)) return kStatusBytes + kda::chunk_split_workspace(B, T, HV);
     return kStatusBytes;
 }
 
@@ -115,9 +122,7 @@ int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk,
     if (!sizes_ok(B, T, H, HV, K, V, chunk) || (dtype != KDA_F32 && dtype != KDA_BF16) || workspace_bytes < kStatusBytes)
         return -1;
     if (dtype != KDA_BF16 || !split_shape(K, V, chunk)) return KDA_SCHEDULE_CUDA_CORE;
-    const long long chunks = (long long)B * HV * ((T + 63) / 64);  // one prep task per chunk, counted in an int
-    if ((long long)B * HV <= kTwoPassMaxPairs && chunks < (1ll << 30) &&
-        workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
+    if (two_pass_sizes(B, T, HV) && workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
         return KDA_SCHEDULE_TC_TWO_PASS;
     return KDA_SCHEDULE_TC_SINGLE_PASS;
 }

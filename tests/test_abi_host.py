@@ -138,3 +138,16 @@ def test_schedule_choice():
     assert kda.schedule(2, 1000, 4, 8, 128, 128, 64) == kda.SCHEDULE_TC_TWO_PASS
     assert L.kda_chunk_fwd_schedule(8, 1000, 16, 16, 128, 128, 64, kda.BF16, 1 << 40) == kda.SCHEDULE_TC_SINGLE_PASS
     assert kda.uses_tensor_cores(128, 128, 64) and not kda.uses_tensor_cores(64, 64, 64)
+
+
+def test_two_pass_limits():
+    L = kda.lib
+    # token stride (HV x 256 bytes) x T must stay below 2^40 bytes for the prep pass's tensor maps
+    T = 1 << 27  # 32 heads x 256 B x 2^27 = 2^40
+    assert kda.workspace_size(1, T, 8, 32, 128, 128, 64) == 256
+    assert L.kda_chunk_fwd_schedule(1, T, 8, 32, 128, 128, 64, kda.BF16, 1 << 62) == kda.SCHEDULE_TC_SINGLE_PASS
+    assert kda.workspace_size(1, T - 64, 8, 32, 128, 128, 64) > 256
+    # fewer than 2^30 chunks in all: 64 pairs x 2^24 chunks of 64 tokens is 2^30
+    T2 = 1 << 30
+    assert kda.workspace_size(64, T2, 1, 1, 128, 128, 64) == 256
+    assert kda.workspace_size(64, T2 - 64, 1, 1, 128, 128, 64) > 256
