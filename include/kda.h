@@ -83,8 +83,9 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
  * runs its fastest schedule for these sizes.  Always >= 256: the first 256 bytes hold
  * the on-device status word read by kda_read_status.  For K = V = 128, chunk 64 and at
  * most 96 (sequence, value head) pairs (B * HV) it adds the per-chunk records of the
- * two-pass schedule (146 KiB per chunk of 64 tokens per pair).  Returns 0 for sizes
- * kda_chunk_fwd rejects.
+ * two-pass schedule (146 KiB per chunk of 64 tokens per pair), as long as there are fewer
+ * than 2^30 chunks in all and T * HV * 256 < 2^40.  Returns 0 for sizes kda_chunk_fwd
+ * rejects.
  */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk);
 
