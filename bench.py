@@ -6,10 +6,15 @@ plus the fused decode step's state GB/s.
 
 One step = one pass of the forward pass over one batch of the workload with inputs resident in
 HBM: one ``kda_chunk_fwd`` call for the prefill workloads (1-4), one ``kda_recurrent_step`` call for
-the decode workload (5).  Rank 0 prints ONE JSON line.  With N > 1 (launched by torch.distributed.run)
-every rank runs the same workload on its own GPU over its own independent (b, hv) shard -- the
-forward pass has no exchange step, so there is no collective on the data path (weak scaling);
-a barrier and a MAX all-reduce of the device times are the only communication.
+the decode workload (5).  The headline line is workload 4 (B1 T65536 H8->HV32, the largest
+single-GPU configuration); the other prefill workloads (2, 3) and the decode workload (5) are
+measured in the same run and reported as extra keys, each with its own roofline.
+
+Rank 0 prints ONE JSON line.  ``--gpus N`` with N > 1 relaunches this script under
+torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1) unless it already runs under
+it.  Every rank runs the same workload on its own GPU over its own independent (b, hv) shard -- the
+forward pass has no exchange step, so there is no collective on the data path (weak scaling); a
+barrier and a MAX all-reduce of the device times are the only communication.
 """
 from __future__ import annotations
 
@@ -210,109 +215,184 @@ def _step_inputs_decode(x, w, dev):
     return {n: x[n].to(dev).transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
 
 
+def l2_note(w) -> str:
+    """How the timed steps keep the L2 cache from serving the inputs: a flush between steps for a
+    workload whose bytes fit in L2 twice over, else nothing (its inputs alone exceed L2)."""
+    small = (not w.is_decode) and prefill_bytes(w) < 2 * (126 << 20)
+    return "flushed between timed steps (256 MiB write)" if small else "inputs larger than L2"
+
+
+def workload_config(w, ws):
+    """The `config` object of a line; identical for both arms of the same workload."""
+    return {"workload": f"workload {w.wid}: {w.name}", "B": w.B, "T": w.T, "H": w.H, "HV": w.HV, "K": w.K,
+            "V": w.V, "chunk": w.chunk, "gate": "standard" if w.gate_mode == GATE_STANDARD else "safe",
+            "inputs": "bf16" if w.dtype == torch.bfloat16 else "fp32", "state": "fp32",
+            "S0": w.S0_std is not None, "l2": l2_note(w),
+            "parallelism": f"dp{ws} (independent (b, hv) shards per GPU, no collective)"}
+
+
+def _time_steps(step, steps, stream, dev, flush, ws, clk=None):
+    """Device time (ms) of each of `steps` calls of step(i), CUDA events on `stream`, bracketed by a
+    barrier and a synchronize on both sides; `flush` (or None) is zeroed before every step."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    if clk is not None:
+        clk.__enter__()
+    try:
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            evs[i][0].record(stream)
+            step(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    finally:
+        if clk is not None:
+            clk.__exit__()
+    barrier(ws)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def _roofline(bytes_per_launch, flops, sec_per_launch, hbm_peak, peak_kind, kernel_file, wid):
+    achieved = bytes_per_launch / sec_per_launch / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": ncu_traffic(kernel_file, wid),
+            "kernel_file": kernel_file, "algorithmic_bytes_per_launch": bytes_per_launch}
+    if flops:
+        roof["algorithmic_flops_per_launch"] = flops
+        roof["achieved_tflops"] = round(flops / sec_per_launch / 1e12, 2)
+    return roof
+
+
+class Prefill:
+    """One prefill workload resident on the device: inputs, outputs and the workspace that selects
+    the fastest schedule, and one ``kda_chunk_fwd`` call per step."""
+
+    def __init__(self, w, seed, dev, kda):
+        self.w, self.kda, self.dev = w, kda, dev
+        self.x = make_inputs(w, seed=seed, device=str(dev))
+        self.ws_bytes = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
+        self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.o = torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev)
+        self.S_T = torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev)
+        self.sched = kda.schedule(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, self.ws_bytes)
+        self.kernel_file = PREFILL_KERNEL_FILES[self.sched]
+        self.launches = kda.schedule_launches(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, self.ws_bytes)
+
+    def step(self, i=0):
+        x, w = self.x, self.w
+        self.kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["S0"],
+                           chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=self.o, S_T=self.S_T,
+                           workspace=self.workspace)
+
+    def measure(self, steps, warmup, ws, flush, hbm_peak, peak_kind, clk=None):
+        w = self.w
+        for i in range(warmup):
+            self.step(i)
+        torch.cuda.synchronize(self.dev)
+        self.kda.read_status(self.workspace)
+        stream = torch.cuda.current_stream(self.dev)
+        ms = _time_steps(self.step, steps, stream, self.dev, flush if l2_note(w).startswith("flushed") else None,
+                         ws, clk)
+        self.kda.read_status(self.workspace)
+        value, ms_per_step = aggregate(w.B * w.T, steps, sum(ms), ws)
+        # one library call per step: its kernels are timed together, since the algorithmic bytes
+        # belong to the pass as a whole
+        roof = _roofline(prefill_bytes(w), prefill_flops(w), (sum(ms) / steps) / 1e3, hbm_peak, peak_kind,
+                         self.kernel_file, w.wid)
+        roof["schedule"] = self.kda.SCHEDULE_NAMES[self.sched]
+        roof["kernels_per_call"] = self.launches
+        return value, ms_per_step, roof
+
+
+def measure_decode(w, seed, dev, kda, hbm_peak, peak_kind, ws=1, steps=None, warmup=3, clk=None):
+    """`steps` consecutive kda_recurrent_step calls (default: the workload's 128) on the workload's token
+    stream, the state updated in place; returns (tokens/s, ms per step, roofline)."""
+    x = make_inputs(w, seed=seed, device=str(dev))
+    steps_in = _step_inputs_decode(x, w, dev)
+    S = x["S0"].clone()
+    o = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
+    nsteps = steps_in["q"].shape[0]
+    steps = steps or w.decode_steps
+
+    def step(i):
+        t = i % nsteps
+        kda.recurrent_step(steps_in["q"][t], steps_in["k"][t], steps_in["v"][t], steps_in["g"][t],
+                           steps_in["beta"][t], S, x["A_log"], x["dt_bias"], gate_mode=w.gate_mode,
+                           lower_bound=w.lower_bound, o=o)
+    for i in range(warmup):
+        step(i)
+    # 512 MiB of state per step: far more than L2, no flush needed
+    ms = _time_steps(lambda i: step(warmup + i), steps, torch.cuda.current_stream(dev), dev, None, ws, clk)
+    value, ms_per_step = aggregate(w.B, steps, sum(ms), ws)
+    roof = _roofline(decode_bytes(w), 0, (sum(ms) / steps) / 1e3, hbm_peak, peak_kind, DECODE_KERNEL_FILE, w.wid)
+    return value, ms_per_step, roof
+
+
+EXTRA_STEPS = {1: 200, 2: 200, 3: 40, 4: 20}
+
+
 def run_ours(args, ws, rank, local):
     from kimi_delta_attention_33_b200 import kda
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
     if args.B is not None:
         w = w.scaled(B=args.B)
+    if args.T is not None:
+        w = w.scaled(T=args.T)
     torch.manual_seed(0)
-    x = make_inputs(w, seed=rank_seed(w, rank), device=str(dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm_peak, _, peak_kind = measured_peaks()
-    stream = torch.cuda.current_stream(dev)
+    clk = ClockSampler(local, period_s=0.002)
 
     if w.is_decode:
-        steps_in = _step_inputs_decode(x, w, dev)
-        S = x["S0"].clone()
-        o = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
-        nsteps = steps_in["q"].shape[0]
-
-        def step(i):
-            t = i % nsteps
-            kda.recurrent_step(steps_in["q"][t], steps_in["k"][t], steps_in["v"][t], steps_in["g"][t],
-                               steps_in["beta"][t], S, x["A_log"], x["dt_bias"], gate_mode=w.gate_mode,
-                               lower_bound=w.lower_bound, o=o)
-        units_per_step = w.B                    # one token per sequence per step
-        bytes_per_launch = decode_bytes(w)
-        kernel_file, flush_needed = DECODE_KERNEL_FILE, False   # 512 MiB of state >> L2
-        sched, launches_per_step = None, 1
+        value, ms_per_step, roof = measure_decode(w, rank_seed(w, rank), dev, kda, hbm_peak, peak_kind, ws,
+                                                  steps=args.steps, warmup=args.warmup, clk=clk)
+        launches_per_step, x = 1, None
     else:
-        ws_bytes = kda.workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk)
-        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
-        o = torch.empty(w.B, w.T, w.HV, w.V, dtype=w.dtype, device=dev)
-        S_T = torch.empty(w.B, w.HV, w.K, w.V, dtype=torch.float32, device=dev)
+        pf = Prefill(w, rank_seed(w, rank), dev, kda)
+        value, ms_per_step, roof = pf.measure(args.steps, args.warmup, ws, flush, hbm_peak, peak_kind, clk)
+        launches_per_step, x = pf.launches, pf.x
+        sched = pf.sched
+        del pf
 
-        def step(i):
-            kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["S0"],
-                          chunk=w.chunk, gate_mode=w.gate_mode, lower_bound=w.lower_bound, o=o, S_T=S_T,
-                          workspace=workspace)
-        units_per_step = w.B * w.T
-        bytes_per_launch = prefill_bytes(w)
-        sched = kda.schedule(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, ws_bytes)
-        kernel_file = PREFILL_KERNEL_FILES[sched]
-        launches_per_step = kda.SCHEDULE_LAUNCHES[sched]
-        flush_needed = prefill_bytes(w) < 2 * (126 << 20)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    if not w.is_decode:
-        kda.read_status(workspace)
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(ws)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            if flush_needed:
-                flush.zero_()
-            evs[i][0].record(stream)
-            step(args.warmup + i)
-            evs[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(ws)
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    value, ms_per_step = aggregate(units_per_step, args.steps, sum(step_ms), ws)
-    # one library call per step: its kernels (one, or the two of the two-pass schedule) are timed
-    # together, since the algorithmic bytes belong to the pass as a whole
-    kern_s = (sum(step_ms) / args.steps) / 1e3
-    achieved = bytes_per_launch / kern_s / 1e9
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind,
-            "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": ncu_traffic(kernel_file, w.wid),
-            "kernel_file": kernel_file, "algorithmic_bytes_per_launch": bytes_per_launch}
-    if sched is not None:
-        roof["schedule"] = kda.SCHEDULE_NAMES[sched]
-        roof["kernels_per_call"] = launches_per_step
-    if not w.is_decode:
-        roof["algorithmic_flops_per_launch"] = prefill_flops(w)
-        roof["achieved_tflops"] = round(prefill_flops(w) / kern_s / 1e12, 2)
-
-    e2e = run_e2e(args, w, x, dev, kda) if (rank == 0 and not args.no_e2e) else None
-    decode_extra = None
-    if not w.is_decode and not args.no_decode_extra and rank == 0:
-        decode_extra = run_decode_extra(args, dev, kda, hbm_peak)
-    cpu = cpu_baseline(w) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
-
+    line = None
     if rank == 0:
+        e2e = None if args.no_e2e else run_e2e(args, w, x if x is not None else make_inputs(w, device=str(dev)),
+                                               dev, kda)
         line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None,
-                "dtype": "tf32" if sched in (1, 2) else "f32", "data": "synthetic",
-                "config": workload_config(w, ws, flush_needed), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "dtype": "f32" if w.is_decode or sched == kda.SCHEDULE_CUDA_CORE else "tf32",
+                "data": "synthetic", "config": workload_config(w, ws), "roofline": roof, "e2e": e2e,
                 "gpu_launches": args.steps * launches_per_step, "clocks": clk.summary()}
-        if decode_extra is not None:
-            line["decode"] = decode_extra
+    x = None
+    torch.cuda.empty_cache()
+
+    # the other workloads, measured in the same run on rank 0 (extra keys, each with its roofline)
+    if rank == 0 and not args.no_extras:
+        extras = {}
+        for wid in (2, 3, 4):
+            if wid == w.wid:
+                continue
+            pf = Prefill(WORKLOADS[wid], rank_seed(WORKLOADS[wid], 0), dev, kda)
+            v, mps, r = pf.measure(EXTRA_STEPS[wid], 3, 1, flush, hbm_peak, peak_kind)
+            extras[f"workload{wid}"] = {"workload": workload_config(WORKLOADS[wid], 1)["workload"],
+                                        "steps": EXTRA_STEPS[wid], "ms_per_step": round(mps, 5),
+                                        "tokens_per_s": round(v, 1), "roofline": r}
+            del pf
+            torch.cuda.empty_cache()
+        if not w.is_decode:
+            w5 = WORKLOADS[5]
+            v, mps, r = measure_decode(w5, rank_seed(w5, 0), dev, kda, hbm_peak, peak_kind)
+            extras["decode"] = {"workload": workload_config(w5, 1)["workload"], "steps": w5.decode_steps,
+                                "us_per_step": round(mps * 1e3, 2), "tokens_per_s": round(v, 1),
+                                "state_GBps": r["achieved"], "frac": r["frac"], "roofline": r}
+        line.update(extras)
+    if rank == 0:
+        line["cpu_baseline"] = cpu_baseline(w) if (ws == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(line), flush=True)
-
-
-def workload_config(w, ws, flushed):
-    return {"workload": f"workload {w.wid}: {w.name}", "B": w.B, "T": w.T, "H": w.H, "HV": w.HV, "K": w.K,
-            "V": w.V, "chunk": w.chunk, "gate": "standard" if w.gate_mode == GATE_STANDARD else "safe",
-            "inputs": "bf16" if w.dtype == torch.bfloat16 else "fp32", "state": "fp32",
-            "S0": w.S0_std is not None, "l2": ("flushed between timed steps (256 MiB write)" if flushed
-                                               else "inputs larger than L2"),
-            "parallelism": f"dp{ws} (independent (b, hv) shards per GPU, no collective)"}
 
 
 def run_e2e(args, w, x, dev, kda):
@@ -397,36 +477,6 @@ def run_e2e(args, w, x, dev, kda):
             "copy while step i runs (two buffer sets, three streams)"}
 
 
-def run_decode_extra(args, dev, kda, hbm_peak):
-    """The decode workload's step, measured in the same run: state GB/s against the HBM roofline."""
-    w = WORKLOADS[5]
-    x = make_inputs(w, device=str(dev))
-    steps_in = _step_inputs_decode(x, w, dev)
-    S = x["S0"].clone()
-    o = torch.empty(w.B, w.HV, w.V, dtype=w.dtype, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(t):
-        kda.recurrent_step(steps_in["q"][t], steps_in["k"][t], steps_in["v"][t], steps_in["g"][t],
-                           steps_in["beta"][t], S, x["A_log"], x["dt_bias"], gate_mode=w.gate_mode,
-                           lower_bound=w.lower_bound, o=o)
-    for t in range(3):
-        step(t)
-    torch.cuda.synchronize(dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for t in range(w.decode_steps):
-        step(t)
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    sec = a.elapsed_time(b) / 1e3 / w.decode_steps
-    gbs = decode_bytes(w) / sec / 1e9
-    return {"workload": f"workload 5: {w.name}", "steps": w.decode_steps, "us_per_step": round(sec * 1e6, 2),
-            "tokens_per_s": round(w.B / sec, 1), "state_GBps": round(gbs, 1), "peak": hbm_peak,
-            "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_step": decode_bytes(w),
-            "traffic": ncu_traffic(DECODE_KERNEL_FILE, 5)}
-
-
 # ------------------------------------------------------------------------ CPU oracle legs -----
 
 def _oracle_sample(w, budget_s: float):
@@ -483,6 +533,7 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
     run, desc, threads = _oracle_sample(w, budget_s=2.0)
     for _ in range(args.warmup):
         run()
@@ -491,14 +542,45 @@ def run_reference(args):
     el = time.perf_counter() - t0
     v = round(tokens / el, 2)
     print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
-                      "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+                      "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
                       "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
                       "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                      "config": dict(workload_config(w, 1, False), l2="not applicable: the oracle runs on the host cores"),
+                      "config": workload_config(w, ws),
+                      "note": "the float64 oracle on the host cores; the config's L2 note describes the GPU arm",
                       "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                        "sample": desc + " per step"},
                       "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
           flush=True)
+
+
+def run_dry_plumbing(args):
+    """The multi-rank plumbing alone, on CPU (gloo): set-up, barrier, MAX over ranks and the weak-
+    scaling aggregate of a synthetic per-rank time, and rank 0's one line.  Touches no device; for
+    testing ``--gpus N`` without GPUs."""
+    ws, rank, local = dist_setup(backend="gloo")
+    try:
+        barrier(ws)
+        value, ms_per_step = aggregate(1000, args.steps, 10.0 * (rank + 1) * args.steps, ws)
+        if rank == 0:
+            print(json.dumps({"dry_plumbing": True, "n_gpus": ws, "steps": args.steps, "value": value,
+                              "ms_per_step": ms_per_step, "scaling": "weak"}), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def relaunch_under_torchrun(n: int) -> int:
+    """Run this script again as n ranks under torch.distributed.run (rendezvous on 127.0.0.1), with
+    the same arguments; returns the launcher's exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
 
 
 def main():
@@ -506,16 +588,25 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode-extra", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' extra keys")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dry-plumbing", action="store_true",
+                    help="multi-rank plumbing only, on CPU over gloo (no device is touched)")
     ap.add_argument("--B", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures; not a bench line)")
+    ap.add_argument("--T", type=int, default=None,
+                    help="override the workload's length (smaller cases for profiler captures; not a bench line)")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args.gpus))
     if args.steps is None:
-        args.steps = {1: 200, 2: 200, 3: 20, 4: 10, 5: 128}[args.workload] if args.impl == "ours" else 10
+        args.steps = {1: 200, 2: 200, 3: 40, 4: 20, 5: 128}[args.workload] if args.impl == "ours" else 10
+    if args.dry_plumbing:
+        run_dry_plumbing(args)
+        return
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     if args.impl == "reference":
         run_reference(args)

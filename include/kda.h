@@ -164,24 +164,33 @@ kda_status kda_read_status(const void* workspace, kda_stream_t stream);
  * library supplies it from a fixed array of KDA_NOALLOC_SCRATCH_BYTES bytes of device memory that
  * is part of the library (every GPU that loads the library holds it until the process exits).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.
- *   - The first call on a device resolves the array's device address on that device
- *     (cudaGetSymbolAddress with the device current); make that first call before any stream
- *     capture.
+ *   - Every call resolves the array's address in the current device's context
+ *     (cudaGetSymbolAddress), so a context that was reset or replaced since an earlier call is
+ *     handled.  The first call on a device may also load the library's device code there; make
+ *     that first call before any stream capture.
  *   - The array is smaller than the two-pass schedule's per-chunk records, so these calls
- *     run the single-pass schedule (see kda_chunk_fwd).  Sizes that would need more
- *     workspace than KDA_NOALLOC_SCRATCH_BYTES even so return KDA_ERR_UNSUPPORTED with a
- *     message; nothing is launched.
+ *     run the single-pass schedule (see kda_chunk_fwd), which needs only the 256-byte status
+ *     block: every size kda_chunk_fwd accepts fits.  A size that needed more workspace than
+ *     KDA_NOALLOC_SCRATCH_BYTES would return KDA_ERR_UNSUPPORTED with a message, nothing launched.
  *   - Every call uses the same array and leaves its contents behind; each call clears the part
  *     that must start at zero (the status word).  Calls whose work overlaps on the GPU (for
- *     example on two streams at once) race on the array: order them on one stream.  The status
- *     word is internal, so a bounded on-device wait that gives up cannot be read back through
- *     kda_read_status here.
+ *     example on two streams at once) race on the array: order them on one stream.
  */
 kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
                                  const void* beta, const float* A_log, const float* dt_bias,
                                  const float* S0, int B, int T, int H, int HV, int K, int V, int chunk,
                                  kda_gate_mode gate_mode, float lower_bound, float scale,
                                  kda_dtype dtype, void* o, float* S_T, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_noalloc_read_status -- kda_read_status for the built-in workspace of
+ * kda_chunk_fwd_noalloc on the current device: synchronises `stream`, then reads and clears the
+ * status word the last kda_chunk_fwd_noalloc call left there.  Returns KDA_OK, KDA_ERR_TIMEOUT if a
+ * bounded on-device wait of that call gave up (its outputs are then undefined), or KDA_ERR_CUDA.
+ * Call it before the next kda_chunk_fwd_noalloc call on that device, which clears the word again.
+ * The pages have no counterpart to this call.
+ */
+kda_status kda_chunk_fwd_noalloc_read_status(kda_stream_t stream);
 
 /*
  * kda_recurrent_step -- one decode step for a batch of sequences, fused

@@ -33,7 +33,8 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Every symbol include/kda.h declares, in declaration order.
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
-           "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc", "kda_recurrent_step")
+           "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_noalloc_read_status",
+           "kda_recurrent_step")
 SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS = 0, 1, 2
 SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass"}
 # kernels one kda_chunk_fwd call launches, per schedule
@@ -70,6 +71,8 @@ lib.kda_read_status.argtypes = [_vp, _vp]
 lib.kda_chunk_fwd_noalloc.restype = _i
 lib.kda_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, _vp, _fp,
                                                                                           _vp]
+lib.kda_chunk_fwd_noalloc_read_status.restype = _i
+lib.kda_chunk_fwd_noalloc_read_status.argtypes = [_vp]
 lib.kda_recurrent_step.restype = _i
 lib.kda_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, _fp, _vp, _vp]
 
@@ -186,6 +189,12 @@ def chunk_fwd_noalloc(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, ch
     return o, S_T
 
 
+def noalloc_read_status(device=None):
+    """Synchronise the current stream and raise ``KdaError`` if the last ``chunk_fwd_noalloc`` call on
+    this device had a bounded wait give up."""
+    _check(lib.kda_chunk_fwd_noalloc_read_status(_stream(device)))
+
+
 def read_status(workspace: torch.Tensor):
     """Synchronise the current stream and raise ``KdaError`` if a chunk call's bounded wait gave up."""
     _check(lib.kda_read_status(_ptr(workspace), _stream(workspace.device)))
@@ -220,6 +229,12 @@ def schedule(B, T, H, HV, K, V, chunk, dtype: torch.dtype = torch.bfloat16, work
     if s < 0:
         raise KdaError(ERR_INVALID_ARG, "kda_chunk_fwd rejects these sizes")
     return s
+
+
+def schedule_launches(B, T, H, HV, K, V, chunk, dtype: torch.dtype = torch.bfloat16,
+                      workspace_bytes: int | None = None) -> int:
+    """Number of kernels one ``chunk_fwd`` call launches for these sizes and workspace."""
+    return SCHEDULE_LAUNCHES[schedule(B, T, H, HV, K, V, chunk, dtype, workspace_bytes)]
 
 
 def uses_tensor_cores(K: int, V: int, chunk: int, dtype: torch.dtype = torch.bfloat16) -> bool:

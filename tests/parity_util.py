@@ -1,6 +1,8 @@
 """Shared helpers for the GPU parity tests: run the CUDA path, run the oracle on the same bits, compare."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -11,12 +13,20 @@ from kimi_delta_attention_33_b200.inputs import make_inputs
 TOL = {torch.float32: 1e-4, torch.bfloat16: 5e-3}
 
 
+# Every relative error measured in this session, as (test id, error), in call order; the terminal
+# summary (conftest.py) prints them so the headroom under the bar is visible in every run.
+ERRORS: list = []
+
+
 def rel_err(x, ref) -> float:
     x = np.asarray(x.detach().cpu().double() if hasattr(x, "detach") else x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert np.all(np.isfinite(x)), "non-finite values in GPU output"
     denom = np.abs(ref).max()
-    return float(np.abs(x - ref).max() / (denom if denom > 0 else 1.0))
+    err = float(np.abs(x - ref).max() / (denom if denom > 0 else 1.0))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    ERRORS.append((test, err))
+    return err
 
 
 def to_dev(x: dict, device="cuda") -> dict:

@@ -50,3 +50,21 @@ def test_reference_arm_prints_from_rank0_only():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2`, started as a plain process, relaunches itself as two ranks under
+    torch.distributed.run; --dry-plumbing keeps it on CPU (gloo), touching no device."""
+    e = dict(os.environ)
+    e.pop("CUDA_VISIBLE_DEVICES", None)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        e.pop(k, None)
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--dry-plumbing", "--steps", "3"], cwd=ROOT,
+                       env=e, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["steps"] == 3 and d["scaling"] == "weak"
+    # slowest rank: 20 ms per step; both ranks' 1000 units per step
+    assert d["ms_per_step"] == pytest.approx(20.0) and d["value"] == pytest.approx(2 * 1000 / 0.02)
