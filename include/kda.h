@@ -57,6 +57,16 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  * §Gate 在 API 中的位置): NONE means `g` already holds the log-space decay. */
 typedef enum { KDA_GATE_NONE = 0, KDA_GATE_SAFE = 1, KDA_GATE_STANDARD = 2 } kda_gate_mode;
 
+/* Input options of kda_chunk_fwd_ex and kda_recurrent_step_ex (bit flags).  By default the op takes
+ * q, k as given and beta as the write strength itself (KDA notes, "KDA 递归核心": beta is an input
+ * write strength; DeltaNet-family digest: keys are assumed L2-normalised).  These options move the
+ * two input-side steps into the kernels' load stage, so that a caller holding raw projections does
+ * not pay a separate pass over HBM for them:
+ *   KDA_INPUT_L2NORM_QK   q and k are divided by their L2 norm over the K channels, per token and
+ *                         q/k head, in float32: x / max(||x||, 1e-6).
+ *   KDA_INPUT_BETA_LOGITS beta holds logits; the kernels use sigmoid(beta) = 1 / (1 + exp(-beta)). */
+typedef enum { KDA_INPUT_RAW = 0, KDA_INPUT_L2NORM_QK = 1, KDA_INPUT_BETA_LOGITS = 2 } kda_input_flags;
+
 /* Thread-local description of the last failure on the calling thread ("" if none). */
 const char* kda_last_error(void);
 
@@ -126,6 +136,17 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
                          void* o, float* S_T, void* workspace, size_t workspace_bytes,
                          kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_ex -- kda_chunk_fwd with input options: `input_flags` is a bitwise OR of
+ * kda_input_flags values (0 gives exactly kda_chunk_fwd).  Every other argument, layout, schedule
+ * and error is that of kda_chunk_fwd; unknown flag bits return KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                            const float* A_log, const float* dt_bias, const float* S0, int B, int T, int H,
+                            int HV, int K, int V, int chunk, kda_gate_mode gate_mode, float lower_bound,
+                            float scale, kda_dtype dtype, unsigned int input_flags, void* o, float* S_T,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /* Schedules of kda_chunk_fwd. */
 typedef enum {
@@ -211,6 +232,15 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
                               int B, int H, int HV, int K, int V, kda_gate_mode gate_mode,
                               float lower_bound, float scale, kda_dtype dtype, float* S, void* o,
                               kda_stream_t stream);
+
+/*
+ * kda_recurrent_step_ex -- kda_recurrent_step with input options (see kda_chunk_fwd_ex):
+ * `input_flags` is a bitwise OR of kda_input_flags values; 0 gives exactly kda_recurrent_step.
+ */
+kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                 const float* A_log, const float* dt_bias, int B, int H, int HV, int K, int V,
+                                 kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
+                                 unsigned int input_flags, float* S, void* o, kda_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -54,6 +54,7 @@ kda_status check_common(const void* q, const void* k, const void* v, const void*
 }
 
 constexpr size_t kStatusBytes = kda::kChunkStatusBytes;
+constexpr unsigned int kInputFlagsAll = KDA_INPUT_L2NORM_QK | KDA_INPUT_BETA_LOGITS;
 
 bool sizes_ok(int B, int T, int H, int HV, int K, int V, int chunk) {
     return B >= 1 && T >= 1 && H >= 1 && HV >= 1 && HV % H == 0 && kv_dim_ok(K) && kv_dim_ok(V) &&
@@ -127,13 +128,14 @@ int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk,
     return KDA_SCHEDULE_TC_SINGLE_PASS;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                         const float* A_log, const float* dt_bias, const float* S0, int B, int T, int H, int HV,
-                         int K, int V, int chunk, kda_gate_mode gate_mode, float lower_bound, float scale,
-                         kda_dtype dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes,
-                         kda_stream_t stream) {
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                            const float* A_log, const float* dt_bias, const float* S0, int B, int T, int H, int HV,
+                            int K, int V, int chunk, kda_gate_mode gate_mode, float lower_bound, float scale,
+                            kda_dtype dtype, unsigned int input_flags, void* o, float* S_T, void* workspace,
+                            size_t workspace_bytes, kda_stream_t stream) {
     kda_status s = check_common(q, k, v, g, beta, A_log, B, H, HV, K, V, (int)gate_mode, lower_bound, (int)dtype, o);
     if (s != KDA_OK) return s;
+    if (input_flags & ~kInputFlagsAll) return fail(KDA_ERR_INVALID_ARG, "unknown input flag bits 0x%x", input_flags);
     if (T < 1) return fail(KDA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
     if (chunk != 16 && chunk != 64) return fail(KDA_ERR_UNSUPPORTED, "chunk must be 16 or 64 (got %d)", chunk);
     if ((long long)B * T * HV * (K > V ? K : V) >= (1ll << 40)) return fail(KDA_ERR_UNSUPPORTED, "tensor too large");
@@ -146,7 +148,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     if (o == q || o == k || o == v || o == g || o == beta) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
     if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
     kda::ChunkArgs a{q, k, v, g, beta, A_log, dt_bias, S0, B, T, H, HV, K, V, chunk, (int)gate_mode, lower_bound,
-                     scale, (int)dtype, o, S_T, static_cast<unsigned int*>(workspace),
+                     scale, (int)dtype, input_flags, o, S_T, static_cast<unsigned int*>(workspace),
                      static_cast<char*>(workspace) + kStatusBytes, workspace_bytes - kStatusBytes,
                      (cudaStream_t)stream};
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), (cudaStream_t)stream);
@@ -165,6 +167,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     return ok();
 }
 
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         const float* A_log, const float* dt_bias, const float* S0, int B, int T, int H, int HV,
+                         int K, int V, int chunk, kda_gate_mode gate_mode, float lower_bound, float scale,
+                         kda_dtype dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream) {
+    return kda_chunk_fwd_ex(q, k, v, g, beta, A_log, dt_bias, S0, B, T, H, HV, K, V, chunk, gate_mode, lower_bound,
+                            scale, dtype, 0u, o, S_T, workspace, workspace_bytes, stream);
+}
+
 kda_status kda_read_status(const void* workspace, kda_stream_t stream) {
     if (!workspace) return fail(KDA_ERR_INVALID_ARG, "null workspace");
     unsigned int word = 0;
@@ -180,12 +191,13 @@ kda_status kda_read_status(const void* workspace, kda_stream_t stream) {
     return ok();
 }
 
-kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                              const float* A_log, const float* dt_bias, int B, int H, int HV, int K, int V,
-                              kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype, float* S,
-                              void* o, kda_stream_t stream) {
+kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                 const float* A_log, const float* dt_bias, int B, int H, int HV, int K, int V,
+                                 kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
+                                 unsigned int input_flags, float* S, void* o, kda_stream_t stream) {
     kda_status s = check_common(q, k, v, g, beta, A_log, B, H, HV, K, V, (int)gate_mode, lower_bound, (int)dtype, o);
     if (s != KDA_OK) return s;
+    if (input_flags & ~kInputFlagsAll) return fail(KDA_ERR_INVALID_ARG, "unknown input flag bits 0x%x", input_flags);
     if (!S) return fail(KDA_ERR_INVALID_ARG, "null state pointer S");
     if ((long long)B * HV >= (1ll << 31)) return fail(KDA_ERR_UNSUPPORTED, "B*HV must be < 2^31");
     const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, S, o};
@@ -194,10 +206,18 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
     if (o == q || o == k || o == v || o == g || o == beta || o == S) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
     if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
     kda::DecodeArgs a{q, k, v, g, beta, A_log, dt_bias, B, H, HV, K, V, (int)gate_mode, lower_bound, scale,
-                      (int)dtype, S, o, (cudaStream_t)stream};
+                      (int)dtype, input_flags, S, o, (cudaStream_t)stream};
     cudaError_t e = kda::launch_decode_step(a);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return ok();
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                              const float* A_log, const float* dt_bias, int B, int H, int HV, int K, int V,
+                              kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype, float* S,
+                              void* o, kda_stream_t stream) {
+    return kda_recurrent_step_ex(q, k, v, g, beta, A_log, dt_bias, B, H, HV, K, V, gate_mode, lower_bound, scale,
+                                 dtype, 0u, S, o, stream);
 }
 
 }  // extern "C"

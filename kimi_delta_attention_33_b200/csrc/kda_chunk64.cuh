@@ -54,6 +54,46 @@ __device__ __forceinline__ float gate_rows16_regs(const __nv_bfloat16* col, int 
     return acc;
 }
 
+// KDA_INPUT_L2NORM_QK: the sums of squares of this thread's two q / k operand units (8 channels of
+// row i = 8 (u / 128) + u % 8, u = tid + 512 it) added into per-row totals.  Lanes that share a row
+// differ in lane bits 3 and 4, so two shuffles sum four units and lanes 0-7 add them in shared memory
+// (four warps per row).  The totals must start at zero and are complete after the next barrier.
+__device__ __forceinline__ void add_row_sumsq(const uint4 (&qr)[2], const uint4 (&kr)[2], float* sSqQ, float* sSqK,
+                                              int tid, int lane) {
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        float qf[8], kf[8];
+        bf16x8_to_f32(qr[it], qf);
+        bf16x8_to_f32(kr[it], kf);
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            sq = fmaf(qf[t], qf[t], sq);
+            sk = fmaf(kf[t], kf[t], sk);
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 8);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 8);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 16);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 16);
+        if (lane < 8) {
+            const int u = tid + INV_THREADS * it;
+            const int i = ((u >> 7) << 3) + (u & 7);
+            atomicAdd(sSqQ + i, sq);
+            atomicAdd(sSqK + i, sk);
+        }
+    }
+}
+
+// Divides 8 channels of one q row and one k row by their norms, given their sums of squares.
+__device__ __forceinline__ void scale_row8(float (&qf)[8], float (&kf)[8], float sumsq_q, float sumsq_k) {
+    const float iq = inv_l2norm(sumsq_q), ik = inv_l2norm(sumsq_k);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        qf[t] *= iq;
+        kf[t] *= ik;
+    }
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
 
 // The doubling steps with blocks of 2, 4, 8 and 16 rows never cross a 16 x 16 diagonal block, so

@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(SIMT_THREADS)
 chunk_simt_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const Elt* __restrict__ v,
                   const Elt* __restrict__ g, const Elt* __restrict__ beta, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, const float* __restrict__ S0, int T, int H, int HV, int V,
-                  int gate_mode, float lower_bound, float scale, Elt* __restrict__ o, float* __restrict__ S_T) {
+                  int gate_mode, float lower_bound, float scale, unsigned int flags, Elt* __restrict__ o,
+                  float* __restrict__ S_T) {
     using Sm = SimtSmem<K, C, VT>;
     constexpr int KP = Sm::KP, CP = Sm::CP, VP = Sm::VP;
     constexpr int NT = SIMT_THREADS;
@@ -87,8 +88,31 @@ chunk_simt_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const El
             const int i = idx / VT, c = idx - i * VT;
             sV[idx] = (i < n) ? to_f32(v[(((size_t)b * T + t0 + i) * HV + hv) * V + v0 + c]) : 0.0f;
         }
-        for (int i = tid; i < C; i += NT) sB[i] = (i < n) ? to_f32(beta[((size_t)b * T + t0 + i) * HV + hv]) : 0.0f;
+        for (int i = tid; i < C; i += NT) {
+            const float bl = (i < n) ? to_f32(beta[((size_t)b * T + t0 + i) * HV + hv]) : 0.0f;
+            sB[i] = (i < n && (flags & KDA_INPUT_BETA_LOGITS)) ? beta_from_logit(bl) : bl;
+        }
         __syncthreads();
+        if (flags & KDA_INPUT_L2NORM_QK) {  // q, k rows divided by their norms, one warp per row
+            for (int i = warp; i < n; i += NT / 32) {
+                float qq = 0.f, kk = 0.f;
+                for (int d = lane; d < K; d += 32) {
+                    qq += sQ[i * KP + d] * sQ[i * KP + d];
+                    kk += sK[i * KP + d] * sK[i * KP + d];
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    qq += __shfl_xor_sync(0xffffffffu, qq, off);
+                    kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                }
+                const float iq = inv_l2norm(qq), ik = inv_l2norm(kk);
+                for (int d = lane; d < K; d += 32) {
+                    sQ[i * KP + d] *= iq;
+                    sK[i * KP + d] *= ik;
+                }
+            }
+            __syncthreads();
+        }
 
         // in-chunk inclusive prefix sums of the log decay, one key channel per thread
         for (int d = tid; d < K; d += NT) {
@@ -192,7 +216,7 @@ static cudaError_t launch_simt(const ChunkArgs& a) {
     kern<<<grid, SIMT_THREADS, Sm::bytes, a.stream>>>(
         static_cast<const Elt*>(a.q), static_cast<const Elt*>(a.k), static_cast<const Elt*>(a.v),
         static_cast<const Elt*>(a.g), static_cast<const Elt*>(a.beta), a.A_log, a.dt_bias, a.S0, a.T, a.H, a.HV, a.V,
-        a.gate_mode, a.lower_bound, a.scale, static_cast<Elt*>(a.o), a.S_T);
+        a.gate_mode, a.lower_bound, a.scale, a.flags, static_cast<Elt*>(a.o), a.S_T);
     return cudaGetLastError();
 }
 

@@ -70,11 +70,12 @@ struct PrepLayout {
     static constexpr uint32_t VEC = 229376;
     static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024, ERHO = VEC + 1280, FEND = VEC + 1792;
     static constexpr uint32_t MBAR = VEC + 2304, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8;
+    static constexpr uint32_t SQQ = VEC + 2336, SQK = VEC + 2592;  // [64] row sums of squares of q, k
     static constexpr uint32_t QT = KA + 32768;    // record Qtil staging, in the Tb rows (free until the inverse)
     static constexpr uint32_t PART = KA + 32768;  // gate: per-channel quarter totals and Gam_0 (5 x [128] fp32),
                                                   //   in the Tb rows, which are free until the inverse
     static constexpr uint32_t STG_G = X1, STG_V = X1 + 16384, STG_Q = X1 + 32768, STG_K = X1 + 49152;
-    static constexpr uint32_t BYTES = TBASE + 4;
+    static constexpr uint32_t BYTES = SQK + 256;
     static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
     static_assert(GM + 32768 == VT, "M7's B operand spans GM and VT");
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 1)
 chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                   const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, int T, int H, int HV, int NC, int ntasks,
-                  float lower_bound, float scale, unsigned char* __restrict__ rec_base,
+                  float lower_bound, float scale, unsigned int flags, unsigned char* __restrict__ rec_base,
                   unsigned int* __restrict__ status, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_g) {
@@ -143,6 +144,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
     float* sERho = reinterpret_cast<float*>(smem + L::ERHO);
     float* sFend = reinterpret_cast<float*>(smem + L::FEND);
+    float* sSqQ = reinterpret_cast<float*>(smem + L::SQQ);
+    float* sSqK = reinterpret_cast<float*>(smem + L::SQK);
+    const bool norm_qk = (flags & KDA_INPUT_L2NORM_QK) != 0;
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
@@ -160,6 +164,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         mbar_init(mbar_in, 1);
     }
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
+    if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
     uint32_t phase = 0, phase_in = 0;
@@ -213,7 +218,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (!__syncthreads_and(ok_in)) { aborted = true; break; }
             phase_in ^= 1u;
             in_pending = false;
-            if (tid < CH) sBeta[tid] = __uint_as_float(beta_bits << 16);
+            if (tid < CH) {
+                const float bl = __uint_as_float(beta_bits << 16);
+                sBeta[tid] = (tid < nn && (flags & KDA_INPUT_BETA_LOGITS)) ? beta_from_logit(bl) : bl;
+            }
             const int gd = tid & (KD - 1), gq = tid >> 7;  // channel, quarter of the rows (16 each)
             float gv[16];
             const float acc = gate_rows16_regs<MODE>(sG + 16 * gq * KD + gd, KD, nn - 16 * gq, bias_in, rate,
@@ -263,6 +271,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 qr[it] = *reinterpret_cast<const uint4*>(smem + L::STG_Q + off);
                 kr[it] = *reinterpret_cast<const uint4*>(smem + L::STG_K + off);
             }
+            if (norm_qk) add_row_sumsq(qr, kr, sSqQ, sSqK, tid, lane);  // totals complete after the barrier
             // the previous chunk's record stores must be done reading CK before P3 rewrites it, and
             // the staged tiles in X1 must all be read
             if (tid == 32) bulk_wait_read();
@@ -286,6 +295,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             float qf[8], kf[8], gf[8], rf[8], sf[8], ef[8], ff[8];
             bf16x8_to_f32(qr[it], qf);
             bf16x8_to_f32(kr[it], kf);
+            if (norm_qk) scale_row8(qf, kf, sSqQ[i], sSqK[i]);
             *reinterpret_cast<float4*>(gf) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8));
             *reinterpret_cast<float4*>(gf + 4) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8 + 4));
             *reinterpret_cast<float4*>(rf) = *reinterpret_cast<const float4*>(sRho + 8 * d8);
@@ -410,6 +420,11 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                         r += to_f32(ki[d]) * kd;
                     }
                 }
+                if (norm_qk && j <= i && i < tk.nn) {
+                    const float ikj = inv_l2norm(sSqK[j]);
+                    a *= inv_l2norm(sSqQ[i]) * ikj;
+                    r *= inv_l2norm(sSqK[i]) * ikj;
+                }
                 av[x] = (j <= i) ? scale * a : 0.f;
                 rr[x] = (j < i) ? sBeta[i] * r : 0.f;
             }
@@ -447,6 +462,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, 4 * j4, CH)) = w4;
             *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, 4 * j4, CH)) = w4;
         }
+        if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;  // read for the last time above; the next chunk's sums follow
         fence_proxy_async();
         cta_sync_tc();
 
@@ -782,7 +798,7 @@ cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
     chunk_prep_kernel<MODE><<<grid, PREP_THREADS, PrepLayout::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.T, a.H, a.HV, NC,
-        ntasks, a.lower_bound, a.scale, static_cast<unsigned char*>(a.scratch), a.status, tq, tk, tv, tg);
+        ntasks, a.lower_bound, a.scale, a.flags, static_cast<unsigned char*>(a.scratch), a.status, tq, tk, tv, tg);
     return cudaGetLastError();
 }
 

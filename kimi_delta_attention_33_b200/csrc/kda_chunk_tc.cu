@@ -63,9 +63,11 @@ struct TcLayout {
     static constexpr uint32_t BETA = VEC + 3072;  // [64]
     static constexpr uint32_t MBAR = BETA + 256;  // 8 B
     static constexpr uint32_t TBASE = MBAR + 8;   // 4 B
+    static constexpr uint32_t SQQ = VEC + 3456;   // [64] sums of squares of the q rows (KDA_INPUT_L2NORM_QK)
+    static constexpr uint32_t SQK = VEC + 3712;   // [64] sums of squares of the k rows
     static constexpr uint32_t VS = VEC + 4096;    // bf16 [64][128] staging of the next chunk's v tile
     static constexpr uint32_t BYTES = VS + 64 * VD * 2;
-    static_assert(TBASE + 4 <= VS, "vector region");
+    static_assert(TBASE + 4 <= SQQ && SQK + 256 <= VS, "vector region");
     // TMEM columns (all accumulators M = 128: TMEM lane = row)
     static constexpr int D4 = 0;     // state^T [v][d], 128 columns
     static constexpr int D3 = 128;   // [v][i]: 0-63 outputs, 64-127 -P
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const bf16* __restrict__ g, const bf16* __restrict__ beta, const float* __restrict__ A_log,
                 const float* __restrict__ dt_bias, const float* __restrict__ S0, int T, int H, int HV,
-                float lower_bound, float scale, bf16* __restrict__ o, float* __restrict__ S_T,
+                float lower_bound, float scale, unsigned int flags, bf16* __restrict__ o, float* __restrict__ S_T,
                 unsigned int* __restrict__ status) {
     using L = TcLayout;
     constexpr int gate_mode = MODE;
@@ -94,6 +96,9 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     float* sERho = reinterpret_cast<float*>(smem + L::ERHO);
     float* sESig = reinterpret_cast<float*>(smem + L::ESIG);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
+    float* sSqQ = reinterpret_cast<float*>(smem + L::SQQ);
+    float* sSqK = reinterpret_cast<float*>(smem + L::SQK);
+    const bool norm_qk = (flags & KDA_INPUT_L2NORM_QK) != 0;
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::GM);  // R, overwritten in place by T
     float* sX = reinterpret_cast<float*>(smem + L::XS);
@@ -116,6 +121,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     if (tid == 0) mbar_init(mbar, 1);
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
     if (tid < KD) sFpend[tid] = 1.0f;
+    if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
     {
@@ -163,6 +169,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             }
         }
         bload = (tid < nn) ? to_f32(beta[(tk0 + tid) * HV + hv]) : 0.f;  // tid < nn <= 64
+        if (tid < nn && (flags & KDA_INPUT_BETA_LOGITS)) bload = beta_from_logit(bload);
     };
     // Gate + inclusive in-chunk cumulative log decay of the chunk at tc0 (four threads per key channel),
     // its beta, the fast/exact decision and the per-channel vectors.  Uses sFpend, the pending state
@@ -170,6 +177,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     auto stage_gate = [&](int tc0) -> bool {
         const int nn = min(CH, T - tc0);
         cp_async_wait_all();
+        if (norm_qk) add_row_sumsq(qr, kr, sSqQ, sSqK, tid, lane);  // complete after the barriers below
         __syncthreads();
         if (tid < CH) sBeta[tid] = bload;
         const int gd = tid & (KD - 1), gq = tid >> 7;  // channel, quarter of the rows (16 each)
@@ -243,6 +251,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             float qf[8], kf[8], gf[8], rf[8], sf[8];
             bf16x8_to_f32(qr[it], qf);
             bf16x8_to_f32(kr[it], kf);
+            if (norm_qk) scale_row8(qf, kf, sSqQ[i], sSqK[i]);
             *reinterpret_cast<float4*>(gf) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8));
             *reinterpret_cast<float4*>(gf + 4) = *reinterpret_cast<const float4*>(sGam + gidx(i, 8 * d8 + 4));
             *reinterpret_cast<float4*>(rf) = *reinterpret_cast<const float4*>(sRho + 8 * d8);
@@ -345,6 +354,11 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                         r += to_f32(ki[d]) * kd;
                     }
                 }
+                if (norm_qk && j <= i && i < n) {
+                    const float ikj = inv_l2norm(sSqK[j]);
+                    a *= inv_l2norm(sSqQ[i]) * ikj;
+                    r *= inv_l2norm(sSqK[i]) * ikj;
+                }
                 av[x] = (j <= i) ? scale * a : 0.f;
                 rr[x] = (j < i) ? sBeta[i] * r : 0.f;
             }
@@ -379,6 +393,7 @@ chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
             }
             *reinterpret_cast<uint4*>(smem + L::AT + cm_off(64 + i, 4 * j4, CH)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;  // read for the last time above; the next chunk's sums follow
         fence_proxy_async();
         cta_sync_tc();
         // ---- state chain: M3, M2, M4, M5, M6 back to back (fast path) --------------------------
@@ -483,7 +498,7 @@ cudaError_t launch_tc(const ChunkArgs& a) {
     chunk_tc_kernel<MODE><<<a.B * a.HV, SP_THREADS, L::BYTES, a.stream>>>(
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), static_cast<const bf16*>(a.v),
         static_cast<const bf16*>(a.g), static_cast<const bf16*>(a.beta), a.A_log, a.dt_bias, a.S0, a.T, a.H, a.HV,
-        a.lower_bound, a.scale, static_cast<bf16*>(a.o), a.S_T, a.status);
+        a.lower_bound, a.scale, a.flags, static_cast<bf16*>(a.o), a.S_T, a.status);
     return cudaGetLastError();
 }
 }  // namespace

@@ -49,4 +49,10 @@ __device__ __forceinline__ float gate_value_fast(float graw, float bias, float r
     return graw;
 }
 
+// ---- optional input-side steps (kda_input_flags) ---------------------------------------------
+// 1 / max(||x||, 1e-6) from the sum of squares of x (KDA_INPUT_L2NORM_QK).
+__device__ __forceinline__ float inv_l2norm(float sumsq) { return rsqrtf(fmaxf(sumsq, 1e-12f)); }
+// Write strength from a logit (KDA_INPUT_BETA_LOGITS).
+__device__ __forceinline__ float beta_from_logit(float x) { return 1.0f / (1.0f + expf(-x)); }
+
 }  // namespace kda

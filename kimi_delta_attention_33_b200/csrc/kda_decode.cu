@@ -31,13 +31,13 @@ __global__ void __launch_bounds__(DecodeShape<K, V, NSPLIT>::NT)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const T* __restrict__ g, const T* __restrict__ beta, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, int H, int HV, int gate_mode, float lower_bound,
-                   float scale, float* __restrict__ S, T* __restrict__ o) {
+                   float scale, unsigned int flags, float* __restrict__ S, T* __restrict__ o) {
     using Sh = DecodeShape<K, V, NSPLIT>;
     constexpr int NT = Sh::NT, TPR = Sh::TPR, RPP = Sh::RPP, R = Sh::R, VC = Sh::VC;
     __shared__ float s_q[K], s_k[K], s_a[K];
     __shared__ float s_p[RPP][VC], s_u[RPP][VC];
     __shared__ float s_r[VC];
-    __shared__ float s_qk;
+    __shared__ float s_qk, s_iq, s_ik;  // q . k; 1 / ||q||, 1 / ||k|| (1 unless q, k are normalised here)
 
     const int pair = blockIdx.x / NSPLIT;  // b * HV + hv
     const int v0 = (blockIdx.x - pair * NSPLIT) * VC;
@@ -61,12 +61,29 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
         s_a[d] = expf(gate_value(to_f32(g[(size_t)pair * K + d]), bias, rate, gate_mode, lower_bound));
     }
     __syncthreads();
+    // q . k, and the norms when q and k are normalised here: the reductions below run on the raw
+    // vectors and are rescaled where their results are used (p by 1/||k||, u by 1/||q||, the write
+    // by 1/||k||), so the normalisation needs no extra pass over the state
     if (tid < 32) {
-        float acc = 0.0f;
-        for (int d = tid; d < K; d += 32) acc += s_q[d] * s_k[d];
+        float acc = 0.0f, qq = 0.0f, kk = 0.0f;
+        for (int d = tid; d < K; d += 32) {
+            acc += s_q[d] * s_k[d];
+            qq += s_q[d] * s_q[d];
+            kk += s_k[d] * s_k[d];
+        }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (tid == 0) s_qk = acc;
+        for (int off = 16; off > 0; off >>= 1) {
+            acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            qq += __shfl_xor_sync(0xffffffffu, qq, off);
+            kk += __shfl_xor_sync(0xffffffffu, kk, off);
+        }
+        if (tid == 0) {
+            const bool norm = (flags & KDA_INPUT_L2NORM_QK) != 0;
+            const float iq = norm ? inv_l2norm(qq) : 1.0f, ik = norm ? inv_l2norm(kk) : 1.0f;
+            s_iq = iq;
+            s_ik = ik;
+            s_qk = acc * iq * ik;
+        }
     }
 
     // 3. decay rows (step 1) and the two partial reductions over this thread's rows
@@ -84,11 +101,15 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     __syncthreads();
 
     // 4. finish the reductions per value column: residual r (step 2) and the read-out (step 4)
-    const float bt = to_f32(beta[pair]);
+    const float braw = to_f32(beta[pair]);
+    const float bt = (flags & KDA_INPUT_BETA_LOGITS) ? beta_from_logit(braw) : braw;
+    const float iq = s_iq, ik = s_ik;
     if (tid < VC) {
         float pp = 0.0f, uu = 0.0f;
 #pragma unroll
         for (int j = 0; j < RPP; ++j) { pp += s_p[j][tid]; uu += s_u[j][tid]; }
+        pp *= ik;
+        uu *= iq;
         const float r = to_f32(v[(size_t)pair * V + v0 + tid]) - pp;
         s_r[tid] = r;
         o[(size_t)pair * V + v0 + tid] = from_f32<T>(scale * (uu + bt * s_qk * r));
@@ -100,7 +121,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 #pragma unroll
     for (int i = 0; i < R; ++i) {
         const int d = rg + RPP * i;
-        const float w = bt * s_k[d];
+        const float w = bt * ik * s_k[d];
         st[i].x += w * r4.x; st[i].y += w * r4.y; st[i].z += w * r4.z; st[i].w += w * r4.w;
         __stcs(reinterpret_cast<float4*>(Sp + (size_t)d * V + 4 * cg), st[i]);
     }
@@ -112,7 +133,7 @@ static cudaError_t launch_decode(const DecodeArgs& a) {
     decode_step_kernel<T, K, V, NSPLIT><<<a.B * a.HV * NSPLIT, Sh::NT, 0, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
         static_cast<const T*>(a.g), static_cast<const T*>(a.beta), a.A_log, a.dt_bias, a.H, a.HV, a.gate_mode,
-        a.lower_bound, a.scale, a.S, static_cast<T*>(a.o));
+        a.lower_bound, a.scale, a.flags, a.S, static_cast<T*>(a.o));
     return cudaGetLastError();
 }
 

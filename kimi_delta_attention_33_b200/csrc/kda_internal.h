@@ -15,6 +15,7 @@ struct DecodeArgs {
     int gate_mode;
     float lower_bound, scale;
     int dtype;
+    unsigned int flags;  // kda_input_flags
     float* S;
     void* o;
     cudaStream_t stream;
@@ -27,6 +28,7 @@ struct ChunkArgs {
     int gate_mode;
     float lower_bound, scale;
     int dtype;
+    unsigned int flags;  // kda_input_flags
     void* o;
     float* S_T;
     unsigned int* status;  // device status word (first bytes of the workspace)

@@ -74,8 +74,12 @@ def _l2norm(x: torch.Tensor) -> torch.Tensor:
     return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-6)
 
 
-def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu") -> dict:
+def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu", raw: bool = False) -> dict:
     """Draw one workload's inputs.  Per-token tensors in ``w.dtype``; A_log, dt_bias, S0 fp32.
+
+    ``raw=True`` returns the same draws without the two input-side steps: q and k as drawn (not
+    normalised) and beta as its logits, each cast to ``w.dtype`` -- the inputs of the op's
+    in-kernel input options.
 
     Returns a dict with q, k [B,T,H,K]; v [B,T,HV,V]; g [B,T,HV,K] (g_raw when the
     workload gates in the op); beta [B,T,HV]; A_log [HV]; dt_bias [HV,K]; S0
@@ -99,6 +103,9 @@ def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu") -> di
         A_log = lo + (hi - lo) * torch.rand(HV, **f32)
     dt_bias = w.dt_bias_mean + w.dt_bias_std * torch.randn(HV, K, **f32)
     S0 = None if w.S0_std is None else w.S0_std * torch.randn(B, HV, K, V, **f32)
+    if raw:
+        return dict(q=q.to(w.dtype), k=k.to(w.dtype), v=v.to(w.dtype), g=g.to(w.dtype), beta=beta_logit.to(w.dtype),
+                    A_log=A_log, dt_bias=dt_bias.contiguous(), S0=S0)
     q = _l2norm(q).to(w.dtype)
     k = _l2norm(k).to(w.dtype)
     return dict(q=q, k=k, v=v.to(w.dtype), g=g.to(w.dtype), beta=torch.sigmoid(beta_logit).to(w.dtype),

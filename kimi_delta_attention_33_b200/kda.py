@@ -33,8 +33,9 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Every symbol include/kda.h declares, in declaration order.
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
-           "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_noalloc_read_status",
-           "kda_recurrent_step")
+           "kda_chunk_fwd_ex", "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc",
+           "kda_chunk_fwd_noalloc_read_status", "kda_recurrent_step", "kda_recurrent_step_ex")
+INPUT_RAW, INPUT_L2NORM_QK, INPUT_BETA_LOGITS = 0, 1, 2
 SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS = 0, 1, 2
 SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass"}
 # kernels one kda_chunk_fwd call launches, per schedule
@@ -64,6 +65,9 @@ lib.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
 lib.kda_chunk_fwd.restype = _i
 lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, _vp, _fp, _vp,
                                                                                   _sz, _vp]
+lib.kda_chunk_fwd_ex.restype = _i
+lib.kda_chunk_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp] + [_i] * 7 + [_i, _f, _f, _i, ctypes.c_uint,
+                                                                                     _vp, _fp, _vp, _sz, _vp]
 lib.kda_chunk_fwd_schedule.restype = _i
 lib.kda_chunk_fwd_schedule.argtypes = [_i] * 7 + [_i, _sz]
 lib.kda_read_status.restype = _i
@@ -75,6 +79,9 @@ lib.kda_chunk_fwd_noalloc_read_status.restype = _i
 lib.kda_chunk_fwd_noalloc_read_status.argtypes = [_vp]
 lib.kda_recurrent_step.restype = _i
 lib.kda_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, _fp, _vp, _vp]
+lib.kda_recurrent_step_ex.restype = _i
+lib.kda_recurrent_step_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, ctypes.c_uint,
+                                                                                     _fp, _vp, _vp]
 
 
 def version() -> str:
@@ -137,12 +144,18 @@ def workspace_size(B, T, H, HV, K, V, chunk) -> int:
     return int(lib.kda_chunk_fwd_workspace_size(B, T, H, HV, K, V, chunk))
 
 
+def _input_flags(l2norm_qk: bool, beta_logits: bool) -> int:
+    return (INPUT_L2NORM_QK if l2norm_qk else 0) | (INPUT_BETA_LOGITS if beta_logits else 0)
+
+
 def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int = 64,
               gate_mode: int = GATE_NONE, lower_bound: float | None = None, scale: float | None = None,
               output_final_state: bool = True, S_T: torch.Tensor | None = None, o: torch.Tensor | None = None,
-              workspace: torch.Tensor | None = None, check_status: bool = False):
+              workspace: torch.Tensor | None = None, check_status: bool = False, l2norm_qk: bool = False,
+              beta_logits: bool = False):
     """Chunked prefill.  q, k [B,T,H,K]; v [B,T,HV,V]; g [B,T,HV,K] (g_raw if gate_mode != NONE);
-    beta [B,T,HV]; S0 [B,HV,K,V] fp32 or None.  Returns ``(o, S_T)`` (``S_T`` None unless requested)."""
+    beta [B,T,HV]; S0 [B,HV,K,V] fp32 or None.  Returns ``(o, S_T)`` (``S_T`` None unless requested).
+    ``l2norm_qk`` / ``beta_logits`` select the in-kernel input steps (``kda_chunk_fwd_ex``)."""
     _require_cuda(q, k, v, g, beta, A_log, dt_bias, S0)
     B, T, H, K = q.shape
     HV, V = v.shape[2], v.shape[3]
@@ -158,9 +171,16 @@ def chunk_fwd(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, chunk: int
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     lb = float("nan") if lower_bound is None else float(lower_bound)
     sc = -1.0 if scale is None else float(scale)
-    _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias), _ptr(S0),
-                             B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q), _ptr(o),
-                             _ptr(S_T), _ptr(workspace), workspace.numel(), _stream(q.device)))
+    flags = _input_flags(l2norm_qk, beta_logits)
+    if flags == 0:
+        _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                                 _ptr(S0), B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q),
+                                 _ptr(o), _ptr(S_T), _ptr(workspace), workspace.numel(), _stream(q.device)))
+    else:
+        _check(lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                                    _ptr(S0), B, T, H, HV, K, V, int(chunk), int(gate_mode), lb, sc, _dtype_code(q),
+                                    flags, _ptr(o), _ptr(S_T), _ptr(workspace), workspace.numel(),
+                                    _stream(q.device)))
     if check_status:
         read_status(workspace)
     return o, S_T
@@ -201,7 +221,8 @@ def read_status(workspace: torch.Tensor):
 
 
 def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: int = GATE_NONE,
-                   lower_bound: float | None = None, scale: float | None = None, o: torch.Tensor | None = None):
+                   lower_bound: float | None = None, scale: float | None = None, o: torch.Tensor | None = None,
+                   l2norm_qk: bool = False, beta_logits: bool = False):
     """One fused decode step.  q, k [B,H,K] (or [B,1,H,K]); v [B,HV,V]; g [B,HV,K]; beta [B,HV];
     S [B,HV,K,V] fp32 updated in place.  Returns o [B,HV,V] (shaped like v)."""
     _require_cuda(q, k, v, g, beta, S, A_log, dt_bias)
@@ -213,9 +234,15 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
     _require_out(S, (B, HV, K, V), torch.float32)
     lb = float("nan") if lower_bound is None else float(lower_bound)
     sc = -1.0 if scale is None else float(scale)
-    _check(lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
-                                  B, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q), _ptr(S), _ptr(o),
-                                  _stream(q.device)))
+    flags = _input_flags(l2norm_qk, beta_logits)
+    if flags == 0:
+        _check(lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                                      B, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q), _ptr(S), _ptr(o),
+                                      _stream(q.device)))
+    else:
+        _check(lib.kda_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log),
+                                         _ptr(dt_bias), B, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q),
+                                         flags, _ptr(S), _ptr(o), _stream(q.device)))
     return o
 
 

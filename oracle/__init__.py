@@ -19,6 +19,11 @@ What it computes (page title, then section):
 * ``dplr``        -- DeltaNet-family digest, "diagonal-low-rank transition": the
   same recurrence through explicit dense K x K transition matrices, a third
   independent form used only to pin ``recurrent``.
+* ``input_side``  -- the op's optional input-side steps as a separate float64
+  pre-step: q, k divided by their L2 norm over the K channels per token and
+  head (the DeltaNet-family digest assumes L2-normalised keys), and beta taken
+  as a logit through the logistic sigmoid (KDA notes, "KDA 递归核心": beta is the
+  write strength, a value in (0, 1)).  ``forward`` applies it when asked.
 * ``backward`` (module ``oracle.backward``) -- the reverse mode of ``forward``,
   derived step by step from the recurrence and the gates, pinned by central
   finite differences of ``forward``: the reference for a backward pass; and
@@ -197,9 +202,30 @@ def dplr(q, k, v, g, beta, S0=None, *, scale=None):
     return o, S_out
 
 
+NORM_FLOOR = 1e-6  # a vector with a smaller norm is divided by this instead (a zero vector stays zero)
+
+
+def input_side(q, k, beta, *, l2norm_qk=False, beta_logits=False):
+    """The optional input-side steps, float64: returns ``(q, k, beta)``.
+
+    ``l2norm_qk``: every q and k vector (last axis, the K channels of one token and head) is divided by
+    ``max(||x||_2, NORM_FLOOR)``.  ``beta_logits``: beta is mapped through ``1 / (1 + exp(-beta))``.
+    With both off the inputs come back unchanged (upcast to float64)."""
+    q, k, beta = _f64(q), _f64(k), _f64(beta)
+    if l2norm_qk:
+        q = q / np.maximum(np.sqrt(np.sum(q * q, axis=-1, keepdims=True)), NORM_FLOOR)
+        k = k / np.maximum(np.sqrt(np.sum(k * k, axis=-1, keepdims=True)), NORM_FLOOR)
+    if beta_logits:
+        beta = 1.0 / (1.0 + np.exp(-beta))
+    return q, k, beta
+
+
 def forward(q, k, v, g, beta, A_log=None, dt_bias=None, S0=None, *, gate_mode=GATE_NONE,
-            lower_bound=None, scale=None):
-    """Gate (if ``gate_mode`` is SAFE or STANDARD, ``g`` holds g_raw) then the recurrence."""
+            lower_bound=None, scale=None, l2norm_qk=False, beta_logits=False):
+    """The input-side steps (when asked), the gate (if ``gate_mode`` is SAFE or STANDARD, ``g`` holds
+    g_raw), then the recurrence."""
+    if l2norm_qk or beta_logits:
+        q, k, beta = input_side(q, k, beta, l2norm_qk=l2norm_qk, beta_logits=beta_logits)
     if gate_mode != GATE_NONE:
         g = gate(g, A_log, dt_bias, mode=gate_mode, lower_bound=lower_bound)
     return recurrent(q, k, v, g, beta, S0, scale=scale)

@@ -151,3 +151,20 @@ def test_two_pass_limits():
     T2 = 1 << 30
     assert kda.workspace_size(64, T2, 1, 1, 128, 128, 64) == 256
     assert kda.workspace_size(64, T2 - 64, 1, 1, 128, 128, 64) > 256
+
+
+def test_input_option_entry_points_validate_before_launch():
+    L = kda.lib
+    # unknown flag bits
+    assert L.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, 2, 128, 128, 64,
+                              kda.GATE_SAFE, -5.0, -1.0, kda.BF16, 8, FAKE * 2, None, FAKE * 3, 1 << 20,
+                              None) == kda.ERR_INVALID_ARG
+    assert L.kda_recurrent_step_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 2, 4, 128, 128, kda.GATE_SAFE, -5.0,
+                                   -1.0, kda.BF16, 4, FAKE * 4, FAKE * 2, None) == kda.ERR_INVALID_ARG
+    # the documented flags pass validation and fail on the next bad argument as kda_chunk_fwd does
+    flags = kda.INPUT_L2NORM_QK | kda.INPUT_BETA_LOGITS
+    assert L.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, 2, 128, 128, 32,
+                              kda.GATE_SAFE, -5.0, -1.0, kda.BF16, flags, FAKE * 2, None, FAKE * 3, 1 << 20,
+                              None) == kda.ERR_UNSUPPORTED
+    assert L.kda_recurrent_step_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 2, 4, 128, 128, kda.GATE_SAFE, -5.0,
+                                   -1.0, kda.BF16, flags, None, FAKE * 2, None) == kda.ERR_INVALID_ARG
