@@ -41,7 +41,8 @@ L2_FLUSH_BYTES = 256 << 20
 # source file of the kernels each kda_chunk_fwd schedule runs (keys: kda.SCHEDULE_* values)
 PREFILL_KERNEL_FILES = {0: "kimi_delta_attention_33_b200/csrc/kda_chunk_simt.cu",
                         1: "kimi_delta_attention_33_b200/csrc/kda_chunk_tc.cu",
-                        2: "kimi_delta_attention_33_b200/csrc/kda_chunk_split.cu"}
+                        2: "kimi_delta_attention_33_b200/csrc/kda_chunk_split.cu",
+                        3: "kimi_delta_attention_33_b200/csrc/kda_chunk_split.cu"}
 DECODE_KERNEL_FILE = "kimi_delta_attention_33_b200/csrc/kda_decode.cu"
 
 

@@ -94,8 +94,9 @@ kda_status kda_gate(const void* g_raw, kda_dtype dtype, const float* A_log, cons
  * the on-device status word read by kda_read_status.  For K = V = 128, chunk 64 and at
  * most 96 (sequence, value head) pairs (B * HV) it adds the per-chunk records of the
  * two-pass schedule (146 KiB per chunk of 64 tokens per pair), as long as there are fewer
- * than 2^30 chunks in all and T * HV * 256 < 2^40.  Returns 0 for sizes kda_chunk_fwd
- * rejects.
+ * than 2^30 chunks in all and T * HV * 256 < 2^40; where that schedule splits its state pass
+ * along the sequence (long sequences, few pairs), 128 KiB per segment per pair more for the
+ * segments' chunk maps.  Returns 0 for sizes kda_chunk_fwd rejects.
  */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int HV, int K, int V, int chunk);
 
@@ -152,7 +153,10 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
 typedef enum {
     KDA_SCHEDULE_CUDA_CORE = 0,     /* one kernel on the CUDA cores (float32 inputs, other shapes)     */
     KDA_SCHEDULE_TC_SINGLE_PASS = 1, /* one tensor-core kernel, one CTA per (sequence, value head)      */
-    KDA_SCHEDULE_TC_TWO_PASS = 2     /* two tensor-core kernels: all chunks' local work, then the state */
+    KDA_SCHEDULE_TC_TWO_PASS = 2,    /* two tensor-core kernels: all chunks' local work, then the state */
+    KDA_SCHEDULE_TC_TWO_PASS_SCAN = 3 /* the two passes with the state pass split along the sequence:
+                                        segments' chunk maps, the segment chain, then the outputs (four
+                                        kernels); taken for long sequences with few (sequence, head) pairs */
 } kda_schedule;
 
 /*

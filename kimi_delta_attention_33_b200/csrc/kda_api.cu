@@ -124,7 +124,8 @@ int kda_chunk_fwd_schedule(int B, int T, int H, int HV, int K, int V, int chunk,
         return -1;
     if (dtype != KDA_BF16 || !split_shape(K, V, chunk)) return KDA_SCHEDULE_CUDA_CORE;
     if (two_pass_sizes(B, T, HV) && workspace_bytes - kStatusBytes >= kda::chunk_split_workspace(B, T, HV))
-        return KDA_SCHEDULE_TC_TWO_PASS;
+        return kda::chunk_scan_plan((long long)B * HV, (T + 63) / 64).NS > 1 ? KDA_SCHEDULE_TC_TWO_PASS_SCAN
+                                                                              : KDA_SCHEDULE_TC_TWO_PASS;
     return KDA_SCHEDULE_TC_SINGLE_PASS;
 }
 
@@ -154,7 +155,7 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "status word reset");
     const int schedule = kda_chunk_fwd_schedule(B, T, H, HV, K, V, chunk, dtype, workspace_bytes);
-    if (schedule == KDA_SCHEDULE_TC_TWO_PASS) {
+    if (schedule == KDA_SCHEDULE_TC_TWO_PASS || schedule == KDA_SCHEDULE_TC_TWO_PASS_SCAN) {
         e = kda::launch_chunk_split(a);
         if (e != cudaSuccess) return cuda_fail(e, "two-pass tensor-core chunk kernel launch");
     } else if (schedule == KDA_SCHEDULE_TC_SINGLE_PASS) {

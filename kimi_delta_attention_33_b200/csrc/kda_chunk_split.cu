@@ -85,20 +85,26 @@ struct PrepLayout {
 template <int VB>
 struct StateLayout {
     static constexpr int NKA = VB <= 32 ? 2 : 1;              // KA / U buffers
+    // With 128 value columns the E^T operand takes the place of the U^T rows it is computed from.
+    static constexpr bool ALIAS_E = VB > 64;
     static constexpr uint32_t WQ = 0;                          // [128][128]
     static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], U^T [VB][64], e^{Gam_end}
     static constexpr uint32_t UT_OFF = Rec::KA_BYTES, VEC_OFF = Rec::KA_BYTES + VB * 256;
     static constexpr uint32_t KA_STRIDE = VEC_OFF + 512;
     static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S^T [VB][128]    (B of M8)
-    static constexpr uint32_t EOP = SOP + VB * 128 * 4;        // tf32 E^T  [VB][64]    (B of M9, M10)
-    static constexpr uint32_t MBAR = EOP + VB * 64 * 4;        // wq, mma, ka[0], ka[1], out
+    static constexpr uint32_t EOP = ALIAS_E ? KA0 + UT_OFF : SOP + VB * 128 * 4;  // tf32 E^T [VB][64] (B of M9, M10)
+    static constexpr uint32_t MBAR = ALIAS_E ? SOP + VB * 128 * 4 : EOP + VB * 64 * 4;  // wq, mma, ka[0], ka[1], out
     static constexpr uint32_t TBASE = MBAR + 40;
     static constexpr uint32_t BYTES = TBASE + 16;
     static constexpr uint32_t TMEM_COLS = 2 * VB < 32 ? 32 : 2 * VB;
     static constexpr int D1 = 0, D2 = VB;
     static __device__ __forceinline__ uint32_t ka(int buf) { return KA0 + buf * KA_STRIDE; }
+    static_assert(!ALIAS_E || VB * 64 * 4 <= VB * 256, "E^T fits in the U^T rows");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
+
+// What one state-pass CTA computes over its chunks (see chunk_state_kernel).
+enum : int { STATE_OUT = 0, STATE_CARRY = 1 };
 
 constexpr int STATE_THREADS = 256;
 constexpr int PREP_THREADS = 512;
@@ -541,17 +547,42 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
 
 // Thread layout: warp w serves TMEM lane quarter w % 4 (rows 32 (w % 4) + lane of every
 // accumulator) and column half w / 4 of the value block (HALF = VB / 2 columns).
-template <int VB>
+//
+// One CTA runs chunks [seg L, min(NC, seg L + L)) of one (sequence, value head) pair for one block of
+// VB state columns.  With NS = 1 that is the whole sequence.  For long sequences the chunks are split
+// into NS segments: the chunk map S -> e^{Gam_end} S + Kend (U - Wtil S) is affine in S, so a segment
+// maps its entering state by S -> M S + b, and the segments can run in parallel (DeltaNet-family digest,
+// "Chunkwise Triton pipeline": the state pass is the only traversal between chunks).
+//   STATE_CARRY  two CTA halves per (pair, segment but the last) carry X = [M | b] through the segment
+//                from [I | 0]:
+//                half 0 the M columns (identity start, no U: E = -Wtil X), half 1 the b columns (zero
+//                start); X is written to `carry` at the end.  No outputs.
+//   STATE_OUT    the chunks from the state entering the segment, with the outputs; the last segment
+//                writes S_T.  Unsplit (NS = 1) the entering state is S0; split, every segment reads it
+//                from `carry`, where scan_chain_kernel left it (so S_T may alias S0 in both cases).
+template <int VB, int MODE>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __restrict__ S0, int T, int HV, int NC,
-                   bf16* __restrict__ o, float* __restrict__ S_T, unsigned int* __restrict__ status) {
-    using L = StateLayout<VB>;
+                   int L, int NS, bf16* __restrict__ o, float* __restrict__ S_T, float* __restrict__ carry,
+                   unsigned int* __restrict__ status) {
+    using Lay = StateLayout<VB>;
+    constexpr bool OUTS = MODE == STATE_OUT;
     constexpr int NVB = VD / VB;
+    constexpr int NH = OUTS ? 1 : 2;
     constexpr int HALF = VB / 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t bar_wq = s_base + L::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16, bar_out = bar_wq + 32;
-    const int pair = blockIdx.x / NVB, vb0 = (blockIdx.x - pair * NVB) * VB;
+    const uint32_t bar_wq = s_base + Lay::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16, bar_out = bar_wq + 32;
+    int rest = blockIdx.x;
+    const int vbi = rest % NVB;
+    rest /= NVB;
+    const int half = rest % NH;  // STATE_CARRY: 0 = the M columns, 1 = the b columns
+    rest /= NH;
+    const int nseg = OUTS ? NS : NS - 1;  // the last segment's map is never applied: no carry CTAs for it
+    const int seg = rest % nseg, pair = rest / nseg;
+    const int vb0 = vbi * VB;
+    const int c_begin = seg * L, c_end = min(NC, c_begin + L);
+    const bool use_u = OUTS || half == 1;
     const int b = pair / HV, hv = pair - b * HV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, c0 = (warp >> 2) * HALF;  // lane quarter, first column of this half
@@ -559,6 +590,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     const size_t v_row = (size_t)HV * VD;
     const unsigned char* rec0 = rec_base + (size_t)pair * NC * Rec::BYTES;
     auto rec = [&](int c) { return rec0 + (size_t)c * Rec::BYTES; };
+    // carry slots of (pair, segment): [2][KD][VD] fp32, M then b
+    auto carry_slot = [&](int sg, int hf) { return carry + (((size_t)pair * NS + sg) * 2 + hf) * KD * VD; };
 
     if (tid == 0) {
         mbar_init(bar_wq, 1);
@@ -567,45 +600,56 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         mbar_init(bar_ka0 + 8, 1);
         mbar_init(bar_out, 1);
     }
-    if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
+    if (warp == 0) tmem_alloc(s_base + Lay::TBASE, Lay::TMEM_COLS);
     cta_sync_tc();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::TBASE);
 
     // loads in flight, for the bounded drain on abort: bit 0 wq, bit 1 + buf ka
     uint32_t pending = 0;
     auto load_wq = [&](int c) {
         mbar_expect_tx(bar_wq, 65536);
-        bulk_load(s_base + L::WQ, rec(c) + Rec::WQ, 65536, bar_wq);
+        bulk_load(s_base + Lay::WQ, rec(c) + Rec::WQ, 65536, bar_wq);
         pending |= 1u;
     };
+    // the carry pass reads Kend only (no A) and, for the M columns, no U
+    constexpr uint32_t KA_LOAD = OUTS ? Rec::KA_BYTES : 32768u;
     auto load_ka = [&](int c, int buf) {
         const uint32_t bar = bar_ka0 + 8 * buf;
-        mbar_expect_tx(bar, L::KA_STRIDE);
-        bulk_load(s_base + L::ka(buf), rec(c) + Rec::KA, Rec::KA_BYTES, bar);
-        bulk_load(s_base + L::ka(buf) + L::UT_OFF, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
-        bulk_load(s_base + L::ka(buf) + L::VEC_OFF, rec(c) + Rec::VEC, 512, bar);
+        mbar_expect_tx(bar, KA_LOAD + (use_u ? VB * 256u : 0u) + 512u);
+        bulk_load(s_base + Lay::ka(buf), rec(c) + Rec::KA, KA_LOAD, bar);
+        if (use_u) bulk_load(s_base + Lay::ka(buf) + Lay::UT_OFF, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
+        bulk_load(s_base + Lay::ka(buf) + Lay::VEC_OFF, rec(c) + Rec::VEC, 512, bar);
         pending |= 2u << buf;
     };
     // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32
     const int d = 32 * wq + lane;
     float s[HALF];
+    {
+        const float* src = nullptr;  // row-major [KD][VD] source of the entering state, or none (zeros)
+        if (OUTS) src = NS == 1 ? (S0 ? S0 + (size_t)pair * KD * VD : nullptr) : carry_slot(seg == 0 ? NS - 1 : seg - 1, seg == 0 ? 0 : 1);
 #pragma unroll
-    for (int j = 0; j < HALF; j += 4) {
-        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * KD + d) * VD + vb0 + c0 + j)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        s[j] = x.x;
-        s[j + 1] = x.y;
-        s[j + 2] = x.z;
-        s[j + 3] = x.w;
+        for (int j = 0; j < HALF; j += 4) {
+            float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)d * VD + vb0 + c0 + j)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!OUTS && half == 0) {  // identity: row d has its 1 in column d
+                const int col = vb0 + c0 + j;
+                x = make_float4(col == d ? 1.f : 0.f, col + 1 == d ? 1.f : 0.f, col + 2 == d ? 1.f : 0.f,
+                                col + 3 == d ? 1.f : 0.f);
+            }
+            s[j] = x.x;
+            s[j + 1] = x.y;
+            s[j + 2] = x.z;
+            s[j + 3] = x.w;
+        }
     }
     // the chunk records are written by the preceding prep kernel: wait for it (a no-op unless this
     // grid was launched as its programmatic dependent; the prep CTAs release it once their records
     // are complete, so only the launch itself overlaps their tail)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {
-        load_wq(0);
-        load_ka(0, 0);
-        if (L::NKA == 2 && NC > 1) load_ka(1, 1);
+        load_wq(c_begin);
+        load_ka(c_begin, 0);
+        if (Lay::NKA == 2 && c_begin + 1 < c_end) load_ka(c_begin + 1, 1);
     }
     // tf32(S)^T into the B operand of M8; lanes sharing a bank store different columns
     auto write_sop = [&]() {
@@ -615,15 +659,15 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         rotate_groups8(w, rot);
 #pragma unroll
         for (int j = 0; j < HALF; ++j)
-            *reinterpret_cast<uint32_t*>(smem + L::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
+            *reinterpret_cast<uint32_t*>(smem + Lay::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
     };
     uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0, ph_out = 0;
     bool aborted = false;
     write_sop();
     fence_proxy_async();
     cta_sync_tc();
-    for (int c = 0; c < NC && !aborted; ++c) {
-        const int buf = (L::NKA == 2) ? (c & 1) : 0;
+    for (int c = c_begin; c < c_end && !aborted; ++c) {
+        const int buf = (Lay::NKA == 2) ? ((c - c_begin) & 1) : 0;
         const int n = min(CH, T - c * CH);
         // ---- M8: D1 = [Wtil; Qtil] S ------------------------------------------------------------
         bool ok = true;
@@ -631,7 +675,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             ok = mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
             if (ok) {
                 pending &= ~1u;
-                gemm_tf32(tmem + L::D1, s_base + L::WQ, KD / 4 * 128, s_base + L::SOP, KD / 4 * 128,
+                gemm_tf32(tmem + Lay::D1, s_base + Lay::WQ, KD / 4 * 128, s_base + Lay::SOP, KD / 4 * 128,
                           idesc_tf32(128, VB), KD / 8, false);
                 mma_commit(bar_mma);
             }
@@ -645,37 +689,45 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         ph_mma ^= 1u;
         ph_ka ^= 1u << buf;
         // this chunk's e^{Gam_end}, read before a single KA buffer is refilled below
-        const float eg = reinterpret_cast<const float*>(smem + L::ka(buf) + L::VEC_OFF)[d];
+        const float eg = reinterpret_cast<const float*>(smem + Lay::ka(buf) + Lay::VEC_OFF)[d];
         if (tid == 0) {
             pending &= ~(2u << buf);
-            if (c + 1 < NC) load_wq(c + 1);  // M8 has read WQ
+            if (c + 1 < c_end) load_wq(c + 1);  // M8 has read WQ
         }
         // ---- E = U - Wtil S (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
-        const uint32_t ka = s_base + L::ka(buf);
-        if (wq < 2) {
-            const int j = d;
-            const float* sU = reinterpret_cast<const float*>(smem + L::ka(buf) + L::UT_OFF);
+        const uint32_t ka = s_base + Lay::ka(buf);
+        {
             uint32_t r[HALF];
-            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
-            tmem_wait_ld();
+            if (wq < 2) {
+                const float* sU = reinterpret_cast<const float*>(smem + Lay::ka(buf) + Lay::UT_OFF);
+                tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D1 + c0), r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int vv = 0; vv < HALF; ++vv) r[vv] = to_tf32(sU[(c0 + vv) * CH + j] - __uint_as_float(r[vv]));
-            rotate_groups8(r, rot);
+                for (int vv = 0; vv < HALF; ++vv)
+                    r[vv] = to_tf32((use_u ? sU[(c0 + vv) * CH + d] : 0.f) - __uint_as_float(r[vv]));
+                rotate_groups8(r, rot);
+            }
+            if constexpr (Lay::ALIAS_E) __syncthreads();  // every U^T read done before E^T overwrites them
+            if (wq < 2) {
 #pragma unroll
-            for (int vv = 0; vv < HALF; ++vv)
-                *reinterpret_cast<uint32_t*>(smem + L::EOP + cm_off(c0 + (vv & ~7) + ((vv + rot) & 7), j, CH)) = r[vv];
+                for (int vv = 0; vv < HALF; ++vv)
+                    *reinterpret_cast<uint32_t*>(smem + Lay::EOP + cm_off(c0 + (vv & ~7) + ((vv + rot) & 7), d, CH)) =
+                        r[vv];
+            }
         }
         fence_proxy_async();
         cta_sync_tc();
         // ---- M10: D2 = Kend E (the state side), then M9: D1[64:] += A E (the outputs), each with its
         //      own commit, so that the state update starts after M10 while M9 still runs -------------
         if (tid == 0) {
-            gemm_tf32(tmem + L::D2, ka, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
+            gemm_tf32(tmem + Lay::D2, ka, CH / 4 * 128, s_base + Lay::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
                       false);
             mma_commit(bar_mma);
-            gemm_tf32(tmem + L::D1, ka + 16384, CH / 4 * 128, s_base + L::EOP, CH / 4 * 128, idesc_tf32(128, VB),
-                      CH / 8, true);
-            mma_commit(bar_out);
+            if (OUTS) {
+                gemm_tf32(tmem + Lay::D1, ka + 16384, CH / 4 * 128, s_base + Lay::EOP, CH / 4 * 128,
+                          idesc_tf32(128, VB), CH / 8, true);
+                mma_commit(bar_out);
+            }
         }
         ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
         fence_after_sync();
@@ -684,49 +736,53 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         // ---- state: S = e^{Gam_end} S + D2 --------------------------------------------------------
         {
             uint32_t r[HALF];
-            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D2 + c0), r);
+            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D2 + c0), r);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < HALF; ++j) s[j] = fmaf(eg, s[j], __uint_as_float(r[j]));
         }
-        // ---- outputs (rows 64-127 of D1: lane quarters 2, 3), once M9 is done; thread 0 waits for it
-        //      too before a KA buffer M9 reads is refilled -----------------------------------------
         bool ok_out = true;
-        if (wq >= 2 || tid == 0) {
-            ok_out = mbar_wait(bar_out, ph_out, WAIT_POLLS);
-            fence_after_sync();
-        }
-        if (wq >= 2 && ok_out) {
-            const int i = d - 64;
-            uint32_t r[HALF];
-            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, L::D1 + c0), r);
-            tmem_wait_ld();
-            if (i < n) {
-                bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0 + c0;
+        if constexpr (OUTS) {
+            // ---- outputs (rows 64-127 of D1: lane quarters 2, 3), once M9 is done; thread 0 waits for
+            //      it too before a KA buffer M9 reads is refilled -------------------------------------
+            if (wq >= 2 || tid == 0) {
+                ok_out = mbar_wait(bar_out, ph_out, WAIT_POLLS);
+                fence_after_sync();
+            }
+            if (wq >= 2 && ok_out) {
+                const int i = d - 64;
+                uint32_t r[HALF];
+                tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D1 + c0), r);
+                tmem_wait_ld();
+                if (i < n) {
+                    bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0 + c0;
 #pragma unroll
-                for (int j = 0; j < HALF; j += 8) {
-                    uint4 w;
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
-                    __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                    __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
-                    __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                    w.x = *reinterpret_cast<uint32_t*>(&p0);
-                    w.y = *reinterpret_cast<uint32_t*>(&p1);
-                    w.z = *reinterpret_cast<uint32_t*>(&p2);
-                    w.w = *reinterpret_cast<uint32_t*>(&p3);
-                    *reinterpret_cast<uint4*>(op + j) = w;
+                    for (int j = 0; j < HALF; j += 8) {
+                        uint4 w;
+                        __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+                        __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                        __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                        w.x = *reinterpret_cast<uint32_t*>(&p0);
+                        w.y = *reinterpret_cast<uint32_t*>(&p1);
+                        w.z = *reinterpret_cast<uint32_t*>(&p2);
+                        w.w = *reinterpret_cast<uint32_t*>(&p3);
+                        *reinterpret_cast<uint4*>(op + j) = w;
+                    }
                 }
             }
         }
-        if (L::NKA == 1 && tid == 0 && ok_out && c + 1 < NC) load_ka(c + 1, 0);
+        // a single KA buffer (and, with 128 columns, the E^T operand over its U^T rows) is refilled once
+        // the products that read it (M10, and M9 when there are outputs) are done
+        if (Lay::NKA == 1 && tid == 0 && ok_out && c + 1 < c_end) load_ka(c + 1, 0);
         // ---- the next chunk's S operand --------------------------------------------------------
-        if (c + 1 < NC) write_sop();
+        if (c + 1 < c_end) write_sop();
         fence_proxy_async();
         fence_before_sync();
         if (!__syncthreads_and(ok_out)) { aborted = true; break; }
         fence_after_sync();
-        ph_out ^= 1u;
-        if (L::NKA == 2 && tid == 0 && c + 2 < NC) load_ka(c + 2, buf);
+        if (OUTS) ph_out ^= 1u;
+        if (Lay::NKA == 2 && tid == 0 && c + 2 < c_end) load_ka(c + 2, buf);
     }
 
     if (aborted) {
@@ -734,25 +790,117 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             atomicOr(status, STATUS_TIMEOUT);
             // bounded drain of copies and MMAs still in flight before shared memory and TMEM go away
             if (pending & 1u) mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
-            for (int bb = 0; bb < L::NKA; ++bb)
+            for (int bb = 0; bb < Lay::NKA; ++bb)
                 if (pending & (2u << bb)) mbar_wait(bar_ka0 + 8 * bb, (ph_ka >> bb) & 1u, WAIT_POLLS);
             mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
-            mbar_wait(bar_out, ph_out, WAIT_POLLS);
+            if (OUTS) mbar_wait(bar_out, ph_out, WAIT_POLLS);
         }
-    } else if (S_T) {
+    } else {
+        float* dst = nullptr;
+        if (!OUTS) dst = carry_slot(seg, half);
+        else if (S_T && seg == NS - 1) dst = S_T + (size_t)pair * KD * VD;
+        if (dst) {
 #pragma unroll
-        for (int j = 0; j < HALF; j += 4)
-            *reinterpret_cast<float4*>(S_T + ((size_t)pair * KD + d) * VD + vb0 + c0 + j) =
-                make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+            for (int j = 0; j < HALF; j += 4)
+                *reinterpret_cast<float4*>(dst + (size_t)d * VD + vb0 + c0 + j) =
+                    make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+        }
     }
     cta_sync_tc();
-    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+    if (warp == 0) tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------------------------------------
+// Between the two state passes: the segments of each pair in order, S_{s+1} = M_s S_s + b_s in fp32
+// on the CUDA cores (value columns are independent: one CTA per (pair, block of 16 columns)).  The
+// state entering segment s + 1 overwrites b_s in `carry`, where the STATE_OUT pass reads it.  The last
+// segment's map M_{NS-1} is never applied, so its slot receives the state entering segment 0 (S0 or
+// zeros): the output pass then reads no S0, and S_T may alias S0.
+// ---------------------------------------------------------------------------------------------
+constexpr int CHAIN_THREADS = 256, CHAIN_COLS = 16;
+
+__global__ void __launch_bounds__(CHAIN_THREADS)
+scan_chain_kernel(const float* __restrict__ S0, float* __restrict__ carry, int NS) {
+    __shared__ __align__(16) float sS[KD][CHAIN_COLS];
+    constexpr int NCB = VD / CHAIN_COLS;
+    const int pair = blockIdx.x / NCB, col0 = (blockIdx.x % NCB) * CHAIN_COLS;
+    const int tid = threadIdx.x, d = tid >> 1, cc = (tid & 1) * 8;  // row d, 8 columns from cc
+    const float* s0 = S0 ? S0 + (size_t)pair * KD * VD : nullptr;
+#pragma unroll
+    for (int j = 0; j < 8; j += 4)
+        *reinterpret_cast<float4*>(&sS[d][cc + j]) =
+            s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)d * VD + col0 + cc + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+        float* first = carry + ((size_t)pair * NS + NS - 1) * 2 * KD * VD + (size_t)d * VD + col0 + cc;
+        *reinterpret_cast<float4*>(first) = *reinterpret_cast<const float4*>(&sS[d][cc]);
+        *reinterpret_cast<float4*>(first + 4) = *reinterpret_cast<const float4*>(&sS[d][cc + 4]);
+    }
+    __syncthreads();
+    for (int sg = 0; sg + 1 < NS; ++sg) {
+        const float* M = carry + ((size_t)pair * NS + sg) * 2 * KD * VD;
+        float* bs = carry + (((size_t)pair * NS + sg) * 2 + 1) * KD * VD + (size_t)d * VD + col0 + cc;
+        float acc[8];
+        {
+            const float4 b0 = *reinterpret_cast<const float4*>(bs), b1 = *reinterpret_cast<const float4*>(bs + 4);
+            acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
+            acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
+        }
+        const float* Mrow = M + (size_t)d * VD;
+#pragma unroll 4
+        for (int e4 = 0; e4 < KD; e4 += 4) {
+            const float4 m = __ldg(reinterpret_cast<const float4*>(Mrow + e4));
+            const float mv[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float4 x0 = *reinterpret_cast<const float4*>(&sS[e4 + t][cc]);
+                const float4 x1 = *reinterpret_cast<const float4*>(&sS[e4 + t][cc + 4]);
+                acc[0] = fmaf(mv[t], x0.x, acc[0]); acc[1] = fmaf(mv[t], x0.y, acc[1]);
+                acc[2] = fmaf(mv[t], x0.z, acc[2]); acc[3] = fmaf(mv[t], x0.w, acc[3]);
+                acc[4] = fmaf(mv[t], x1.x, acc[4]); acc[5] = fmaf(mv[t], x1.y, acc[5]);
+                acc[6] = fmaf(mv[t], x1.z, acc[6]); acc[7] = fmaf(mv[t], x1.w, acc[7]);
+            }
+        }
+        __syncthreads();  // every row of the old state read
+        *reinterpret_cast<float4*>(&sS[d][cc]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(&sS[d][cc + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4*>(bs) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(bs + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Segments of the state pass.  Cost model, in chunk steps of one CTA per SM: the unsplit pass is a
+// chain of NC steps per wave of (pair, value block) CTAs (blocks of 16, 32 or 64 columns, as
+// launch_chunk_split picks them); the split one runs 2 x pairs x (NS - 1) carry CTAs, then pairs x NS output
+// CTAs, of L chunks each, in waves over the SMs, plus the segment chain at about 0.6 step per segment.
+// The number of SMs is a planning constant (a B200's 148), so that the workspace size does not depend
+// on the device; the split is taken only where the model gains at least a quarter.
+ScanPlan chunk_scan_plan(long long pairs, int NC) {
+    constexpr long long kPlanSMs = 148;
+    const long long nvb = pairs * 8 <= kPlanSMs ? 8 : pairs * 4 <= kPlanSMs ? 4 : 2;
+    ScanPlan plan{NC, 1};
+    double best = 0.75 * (double)NC * (double)((pairs * nvb + kPlanSMs - 1) / kPlanSMs);
+    for (int Lc : {8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256}) {
+        if (Lc >= NC) break;
+        const long long NS = (NC + Lc - 1) / Lc;
+        const long long wa = (2 * pairs * (NS - 1) + kPlanSMs - 1) / kPlanSMs;
+        const long long wc = (pairs * NS + kPlanSMs - 1) / kPlanSMs;
+        const double cost = (double)(wa + wc) * Lc + 0.6 * (double)NS;
+        if (cost < best) {
+            best = cost;
+            plan = ScanPlan{Lc, (int)NS};
+        }
+    }
+    return plan;
+}
+
 size_t chunk_split_workspace(int B, int T, int HV) {
     const size_t NC = ((size_t)T + CH - 1) / CH;
-    return (size_t)B * HV * NC * Rec::BYTES;
+    const long long pairs = (long long)B * HV;
+    const ScanPlan plan = chunk_scan_plan(pairs, (int)NC);
+    const size_t carry = plan.NS > 1 ? (size_t)pairs * plan.NS * 2 * KD * VD * sizeof(float) : 0;
+    return (size_t)pairs * NC * Rec::BYTES + carry;
 }
 
 namespace {
@@ -802,26 +950,27 @@ cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
     return cudaGetLastError();
 }
 
-template <int VB>
-cudaError_t launch_state(const ChunkArgs& a, int NC) {
+template <int VB, int MODE>
+cudaError_t launch_state(const ChunkArgs& a, int NC, ScanPlan plan, float* carry, bool dependent) {
     using L = StateLayout<VB>;
-    cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::BYTES);
+    auto kern = chunk_state_kernel<VB, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    // programmatic dependent launch: the state kernel's set-up may overlap the prep kernel's tail;
-    // it waits (griddepcontrol.wait) for the prep grid's completion before reading any record
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.B * a.HV * (VD / VB));
+    const long long nseg = MODE == STATE_OUT ? plan.NS : plan.NS - 1;
+    cfg.gridDim = dim3((unsigned)((long long)a.B * a.HV * nseg * (MODE == STATE_OUT ? 1 : 2) * (VD / VB)));
     cfg.blockDim = dim3(STATE_THREADS);
     cfg.dynamicSmemBytes = L::BYTES;
     cfg.stream = a.stream;
+    // programmatic dependent launch right after the prep kernel: the state kernel's set-up may overlap
+    // the prep kernel's tail; it waits (griddepcontrol.wait) for the prep grid before reading a record
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chunk_state_kernel<VB>, static_cast<const unsigned char*>(a.scratch), a.S0, a.T,
-                              a.HV, NC, static_cast<bf16*>(a.o), a.S_T, a.status);
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const unsigned char*>(a.scratch), a.S0, a.T, a.HV, NC, plan.L,
+                              plan.NS, static_cast<bf16*>(a.o), a.S_T, carry, a.status);
 }
 }  // namespace
 
@@ -838,11 +987,20 @@ cudaError_t launch_chunk_split(const ChunkArgs& a) {
         : a.gate_mode == KDA_GATE_STANDARD ? launch_prep<KDA_GATE_STANDARD>(a, NC, ntasks, grid)
                                            : launch_prep<KDA_GATE_NONE>(a, NC, ntasks, grid);
     if (e != cudaSuccess) return e;
-    // value-block width: enough (pair, block) CTAs to cover the SMs, blocks as wide as that allows
     const long long pairs = (long long)a.B * a.HV;
-    if (pairs * 8 <= nsm) return launch_state<16>(a, NC);
-    if (pairs * 4 <= nsm) return launch_state<32>(a, NC);
-    return launch_state<64>(a, NC);
+    const ScanPlan plan = chunk_scan_plan(pairs, NC);
+    if (plan.NS == 1) {
+        // value-block width: enough (pair, block) CTAs to cover the SMs, blocks as wide as that allows
+        if (pairs * 8 <= nsm) return launch_state<16, STATE_OUT>(a, NC, plan, nullptr, true);
+        if (pairs * 4 <= nsm) return launch_state<32, STATE_OUT>(a, NC, plan, nullptr, true);
+        return launch_state<64, STATE_OUT>(a, NC, plan, nullptr, true);
+    }
+    // long sequences: carry [M | b] through every segment, chain the segments, then the outputs
+    float* carry = reinterpret_cast<float*>(static_cast<unsigned char*>(a.scratch) + (size_t)pairs * NC * Rec::BYTES);
+    if ((e = launch_state<128, STATE_CARRY>(a, NC, plan, carry, true)) != cudaSuccess) return e;
+    scan_chain_kernel<<<(unsigned)(pairs * (VD / CHAIN_COLS)), CHAIN_THREADS, 0, a.stream>>>(a.S0, carry, plan.NS);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_state<128, STATE_OUT>(a, NC, plan, carry, false);
 }
 
 }  // namespace kda

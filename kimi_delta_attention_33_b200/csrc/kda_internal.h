@@ -59,8 +59,14 @@ cudaError_t launch_decode_step(const DecodeArgs& a);
 cudaError_t launch_gate(const GateArgs& a);
 cudaError_t launch_chunk_simt(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a);
-// Two-pass tensor-core prefill (same shapes as the single-pass one): per-chunk records need
-// chunk_split_workspace(B, T, HV) bytes of scratch beyond the status block.
+// Two-pass tensor-core prefill (same shapes as the single-pass one): per-chunk records (and, for
+// long sequences, the segment carries of the split state pass) need chunk_split_workspace(B, T, HV)
+// bytes of scratch beyond the status block.
+struct ScanPlan {
+    int L;   // chunks per segment of the state pass
+    int NS;  // segments (1: the state pass runs each sequence as one chain)
+};
+ScanPlan chunk_scan_plan(long long pairs, int NC);
 size_t chunk_split_workspace(int B, int T, int HV);
 cudaError_t launch_chunk_split(const ChunkArgs& a);
 

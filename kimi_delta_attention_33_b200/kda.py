@@ -36,10 +36,10 @@ EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace
            "kda_chunk_fwd_ex", "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc",
            "kda_chunk_fwd_noalloc_read_status", "kda_recurrent_step", "kda_recurrent_step_ex")
 INPUT_RAW, INPUT_L2NORM_QK, INPUT_BETA_LOGITS = 0, 1, 2
-SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS = 0, 1, 2
-SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass"}
+SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS, SCHEDULE_TC_TWO_PASS_SCAN = 0, 1, 2, 3
+SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass", 3: "tc_two_pass_scan"}
 # kernels one kda_chunk_fwd call launches, per schedule
-SCHEDULE_LAUNCHES = {0: 1, 1: 1, 2: 2}
+SCHEDULE_LAUNCHES = {0: 1, 1: 1, 2: 2, 3: 4}
 
 
 class KdaError(RuntimeError):

@@ -31,7 +31,8 @@ def _workspace(w, schedule):
         pytest.skip("more (sequence, head) pairs than the two-pass schedule takes")
     assert need > 256
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
-    assert kda.schedule(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, need) == kda.SCHEDULE_TC_TWO_PASS
+    assert kda.schedule(w.B, w.T, w.H, w.HV, w.K, w.V, w.chunk, w.dtype, need) in (kda.SCHEDULE_TC_TWO_PASS,
+                                                                                kda.SCHEDULE_TC_TWO_PASS_SCAN)
     return ws
 
 
