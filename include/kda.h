@@ -246,6 +246,41 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, co
                                  kda_gate_mode gate_mode, float lower_bound, float scale, kda_dtype dtype,
                                  unsigned int input_flags, float* S, void* o, kda_stream_t stream);
 
+/*
+ * kda_backward_workspace_size -- bytes of device workspace kda_backward needs for these sizes (the
+ * state saved every 8 tokens: B * HV * ceil(T / 8) * K * V * 4 bytes), or 0 for sizes it rejects.
+ */
+size_t kda_backward_workspace_size(int B, int T, int H, int HV, int K, int V);
+
+/*
+ * kda_backward -- reverse mode of kda_chunk_fwd: the gradients of a scalar loss L given
+ * dO = dL/do and dS_T = dL/dS_T, with respect to every input.  The pages define the forward pass
+ * only; the adjoint is derived from its four steps (KDA notes, "KDA 递归核心", §逐步公式) taken in
+ * reverse order, and from the gate formulas (KDA notes, "Gate 激活", table "两种 Gate").
+ *   q, k, v, g, beta, A_log, dt_bias, S0, B..V, gate_mode, lower_bound, scale, dtype
+ *            exactly as given to kda_chunk_fwd (the forward pass is recomputed)
+ *   dO       [B, T, HV, V]  dtype   gradient with respect to o (required)
+ *   dS_T     [B, HV, K, V]  float32 gradient with respect to the final state, or NULL for zeros
+ *   dq, dk   [B, T, H, K]   float32, written (summed over the value heads that read each q/k head)
+ *   dv       [B, T, HV, V]  float32, written
+ *   dg       [B, T, HV, K]  float32, written: the gradient with respect to the `g` argument -- the
+ *            log decay when gate_mode == KDA_GATE_NONE, else g_raw
+ *   dbeta    [B, T, HV]     float32, written
+ *   dS0      [B, HV, K, V]  float32 gradient with respect to S0, written; or NULL
+ *   dA_log   [HV] float32, ddt_bias [HV, K] float32: written when a gate ran (each may be NULL);
+ *            ignored for KDA_GATE_NONE
+ *   workspace, workspace_bytes  >= kda_backward_workspace_size(...) bytes, 16-byte aligned, scratch
+ * Constraints as kda_chunk_fwd's (no chunk argument: the gradients do not depend on it).  All work
+ * runs on the CUDA cores in float32 on `stream`; outputs summed from several CTAs use atomic adds, so
+ * their last bits may differ from run to run.  Outputs must not alias inputs or each other.
+ */
+kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        const float* A_log, const float* dt_bias, const float* S0, const void* dO,
+                        const float* dS_T, int B, int T, int H, int HV, int K, int V, kda_gate_mode gate_mode,
+                        float lower_bound, float scale, kda_dtype dtype, float* dq, float* dk, float* dv,
+                        float* dg, float* dbeta, float* dS0, float* dA_log, float* ddt_bias, void* workspace,
+                        size_t workspace_bytes, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -221,4 +221,40 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
                                  dtype, 0u, S, o, stream);
 }
 
+size_t kda_backward_workspace_size(int B, int T, int H, int HV, int K, int V) {
+    if (!sizes_ok(B, T, H, HV, K, V, 64)) return 0;
+    return kda::backward_workspace(B, T, HV, K, V);
+}
+
+kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        const float* A_log, const float* dt_bias, const float* S0, const void* dO, const float* dS_T,
+                        int B, int T, int H, int HV, int K, int V, kda_gate_mode gate_mode, float lower_bound,
+                        float scale, kda_dtype dtype, float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                        float* dS0, float* dA_log, float* ddt_bias, void* workspace, size_t workspace_bytes,
+                        kda_stream_t stream) {
+    kda_status s = check_common(q, k, v, g, beta, A_log, B, H, HV, K, V, (int)gate_mode, lower_bound, (int)dtype, dO);
+    if (s != KDA_OK) return s;
+    if (T < 1) return fail(KDA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    if (!dq || !dk || !dv || !dg || !dbeta) return fail(KDA_ERR_INVALID_ARG, "dq, dk, dv, dg and dbeta are required");
+    if ((long long)B * T * HV * (K > V ? K : V) >= (1ll << 40)) return fail(KDA_ERR_UNSUPPORTED, "tensor too large");
+    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    const size_t need = kda::backward_workspace(B, T, HV, K, V);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace of at least %zu bytes is required (got %zu)", need, workspace_bytes);
+    const void* outs[] = {dq, dk, dv, dg, dbeta, dS0, dA_log, ddt_bias};
+    const void* ins[] = {q, k, v, g, beta, A_log, dt_bias, S0, dO, dS_T};
+    for (const void* po : outs)
+        for (const void* pi : ins)
+            if (po && po == pi) return fail(KDA_ERR_INVALID_ARG, "outputs must not alias inputs");
+    if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)K);
+    kda::BackwardArgs a{q, k, v, g, beta, A_log, dt_bias, S0, dO, dS_T, B, T, H, HV, K, V, (int)gate_mode,
+                        lower_bound, scale, (int)dtype, dq, dk, dv, dg, dbeta, dS0, dA_log, ddt_bias, workspace,
+                        (cudaStream_t)stream};
+    cudaError_t e = kda::launch_backward(a);
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+    return ok();
+}
+
 }  // extern "C"

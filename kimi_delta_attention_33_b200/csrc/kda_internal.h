@@ -49,6 +49,20 @@ struct GateArgs {
     cudaStream_t stream;
 };
 
+struct BackwardArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias, *S0;
+    const void* dO;
+    const float* dS_T;
+    int B, T, H, HV, K, V;
+    int gate_mode;
+    float lower_bound, scale;
+    int dtype;
+    float *dq, *dk, *dv, *dg, *dbeta, *dS0, *dA_log, *ddt_bias;
+    void* workspace;
+    cudaStream_t stream;
+};
+
 // Status word values written by kernels with bounded waits.
 enum : unsigned int { STATUS_OK = 0u, STATUS_TIMEOUT = 1u };
 
@@ -69,6 +83,10 @@ struct ScanPlan {
 ScanPlan chunk_scan_plan(long long pairs, int NC);
 size_t chunk_split_workspace(int B, int T, int HV);
 cudaError_t launch_chunk_split(const ChunkArgs& a);
+
+// Reverse mode: saved states every few tokens, backward_workspace(B, T, HV, K, V) bytes.
+size_t backward_workspace(int B, int T, int HV, int K, int V);
+cudaError_t launch_backward(const BackwardArgs& a);
 
 // Bytes of status block at the start of every chunk-prefill workspace.
 constexpr size_t kChunkStatusBytes = 256;

@@ -34,7 +34,8 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 # Every symbol include/kda.h declares, in declaration order.
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
            "kda_chunk_fwd_ex", "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc",
-           "kda_chunk_fwd_noalloc_read_status", "kda_recurrent_step", "kda_recurrent_step_ex")
+           "kda_chunk_fwd_noalloc_read_status", "kda_recurrent_step", "kda_recurrent_step_ex",
+           "kda_backward_workspace_size", "kda_backward")
 INPUT_RAW, INPUT_L2NORM_QK, INPUT_BETA_LOGITS = 0, 1, 2
 SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS, SCHEDULE_TC_TWO_PASS_SCAN = 0, 1, 2, 3
 SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass", 3: "tc_two_pass_scan"}
@@ -82,6 +83,13 @@ lib.kda_recurrent_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5
 lib.kda_recurrent_step_ex.restype = _i
 lib.kda_recurrent_step_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp] + [_i] * 5 + [_i, _f, _f, _i, ctypes.c_uint,
                                                                                      _fp, _vp, _vp]
+
+
+lib.kda_backward_workspace_size.restype = _sz
+lib.kda_backward_workspace_size.argtypes = [_i] * 6
+lib.kda_backward.restype = _i
+lib.kda_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp, _vp, _fp] + [_i] * 6 + [_i, _f, _f, _i] + \
+    [_fp] * 8 + [_vp, _sz, _vp]
 
 
 def version() -> str:
@@ -243,6 +251,46 @@ def recurrent_step(q, k, v, g, beta, S, A_log=None, dt_bias=None, *, gate_mode: 
         _check(lib.kda_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log),
                                          _ptr(dt_bias), B, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q),
                                          flags, _ptr(S), _ptr(o), _stream(q.device)))
+    return o
+
+
+def backward_workspace_size(B, T, H, HV, K, V) -> int:
+    return int(lib.kda_backward_workspace_size(B, T, H, HV, K, V))
+
+
+def backward(q, k, v, g, beta, dO, A_log=None, dt_bias=None, S0=None, dS_T=None, *, gate_mode: int = GATE_NONE,
+             lower_bound: float | None = None, scale: float | None = None, need_dS0: bool = True,
+             workspace: torch.Tensor | None = None, out: dict | None = None) -> dict:
+    """Reverse mode of ``chunk_fwd`` (``kda_backward``): gradients of a loss given ``dO`` (and ``dS_T``).
+    Returns a dict of float32 tensors ``dq, dk, dv, dg, dbeta`` (+ ``dS0``; + ``dA_log, ddt_bias`` when a
+    gate ran); ``dg`` is the gradient with respect to the ``g`` argument (g_raw when a gate ran)."""
+    _require_cuda(q, k, v, g, beta, dO, A_log, dt_bias, S0, dS_T)
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    o = dict(out or {})
+    o.setdefault("dq", torch.empty(B, T, H, K, **f32))
+    o.setdefault("dk", torch.empty(B, T, H, K, **f32))
+    o.setdefault("dv", torch.empty(B, T, HV, V, **f32))
+    o.setdefault("dg", torch.empty(B, T, HV, K, **f32))
+    o.setdefault("dbeta", torch.empty(B, T, HV, **f32))
+    if need_dS0:
+        o.setdefault("dS0", torch.empty(B, HV, K, V, **f32))
+    if gate_mode != GATE_NONE:
+        o.setdefault("dA_log", torch.empty(HV, **f32))
+        if dt_bias is not None:
+            o.setdefault("ddt_bias", torch.empty(HV, K, **f32))
+    need = backward_workspace_size(B, T, H, HV, K, V)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    lb = float("nan") if lower_bound is None else float(lower_bound)
+    sc = -1.0 if scale is None else float(scale)
+    _check(lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias), _ptr(S0),
+                            _ptr(dO), _ptr(dS_T), B, T, H, HV, K, V, int(gate_mode), lb, sc, _dtype_code(q),
+                            _ptr(o["dq"]), _ptr(o["dk"]), _ptr(o["dv"]), _ptr(o["dg"]), _ptr(o["dbeta"]),
+                            _ptr(o.get("dS0")), _ptr(o.get("dA_log")), _ptr(o.get("ddt_bias")), _ptr(workspace),
+                            workspace.numel(), _stream(dev)))
     return o
 
 

@@ -168,3 +168,24 @@ def test_input_option_entry_points_validate_before_launch():
                               None) == kda.ERR_UNSUPPORTED
     assert L.kda_recurrent_step_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 2, 4, 128, 128, kda.GATE_SAFE, -5.0,
                                    -1.0, kda.BF16, flags, None, FAKE * 2, None) == kda.ERR_INVALID_ARG
+
+
+def test_backward_validates_before_launch():
+    L = kda.lib
+    assert kda.backward_workspace_size(2, 100, 2, 4, 128, 64) == 2 * 4 * 13 * 128 * 64 * 4
+    assert kda.backward_workspace_size(2, 100, 3, 4, 128, 64) == 0
+
+    def call(**over):
+        a = dict(q=FAKE, dq=FAKE * 5, K=128, ws_bytes=1 << 30, gate=kda.GATE_SAFE, lb=-5.0, HV=4, H=2)
+        a.update(over)
+        return L.kda_backward(a["q"], FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE * 2, None, 2, 100, a["H"],
+                              a["HV"], a["K"], 64, a["gate"], a["lb"], -1.0, kda.BF16, a["dq"], FAKE * 6, FAKE * 7,
+                              FAKE * 8, FAKE * 9, None, None, None, FAKE * 3, a["ws_bytes"], None)
+    assert call(q=None) == kda.ERR_INVALID_ARG
+    assert call(dq=None) == kda.ERR_INVALID_ARG
+    assert call(K=48) == kda.ERR_UNSUPPORTED
+    assert call(HV=3) == kda.ERR_INVALID_ARG
+    assert call(lb=float("nan")) == kda.ERR_INVALID_ARG
+    assert call(ws_bytes=1024) == kda.ERR_INVALID_ARG
+    assert call(dq=FAKE) == kda.ERR_INVALID_ARG  # an output aliasing an input
+    assert kda.last_error() != ""
