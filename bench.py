@@ -33,7 +33,8 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from kimi_delta_attention_33_b200.inputs import GATE_STANDARD, WORKLOADS, make_inputs  # noqa: E402
+from kimi_delta_attention_33_b200.inputs import (GATE_STANDARD, MLA_DECODE, WORKLOADS, make_inputs,  # noqa: E402
+                                                 make_mla_inputs)
 
 METRIC = "KDA fwd tokens/s (chunked prefill) & decode-step state GB/s, % of roofline, 1 B200"
 FALLBACK_HBM_GBS = 6650.0
@@ -44,6 +45,7 @@ PREFILL_KERNEL_FILES = {0: "kimi_delta_attention_33_b200/csrc/kda_chunk_simt.cu"
                         2: "kimi_delta_attention_33_b200/csrc/kda_chunk_split.cu",
                         3: "kimi_delta_attention_33_b200/csrc/kda_chunk_split.cu"}
 DECODE_KERNEL_FILE = "kimi_delta_attention_33_b200/csrc/kda_decode.cu"
+MLA_KERNEL_FILE = "kimi_delta_attention_33_b200/csrc/kda_mla.cu"
 
 
 # ------------------------------------------------------------------------ algorithmic counts ---
@@ -78,6 +80,16 @@ def decode_bytes(w) -> int:
     B, H, HV, K, V = w.B, w.H, w.HV, w.K, w.V
     return (2 * B * HV * K * V * 4 + 2 * B * H * K * e + B * HV * V * e + B * HV * K * e + B * HV * e + HV * 4
             + HV * K * 4 + B * HV * V * e)
+
+
+def mla_bytes(B, T, H, d_q, d_v, r) -> int:
+    """Absorbed MLA decode: the latent cache, both up-projections, q read once; o written (bf16)."""
+    return 2 * (B * T * r + H * d_q * r + H * d_v * r + B * H * d_q + B * H * d_v)
+
+
+def mla_flops(B, T, H, d_q, d_v, r) -> float:
+    """q W_UK, the scores, the weighted latent sum and the W_UV projection, 2 flops per multiply-add."""
+    return 2.0 * B * H * (d_q * r + 2 * T * r + d_v * r)
 
 
 # -------------------------------------------------------------------------------- peaks etc ----
@@ -331,6 +343,29 @@ def measure_decode(w, seed, dev, kda, hbm_peak, peak_kind, ws=1, steps=None, war
     return value, ms_per_step, roof
 
 
+def measure_mla(dev, kda, hbm_peak, peak_kind, bf16_peak, steps=50, warmup=3):
+    """The absorbed MLA decode step on its decode workload (B64 T4096 H96 d_q = d_v = 128 r = 512)."""
+    cfg = MLA_DECODE
+    x = {k: (v.to(dev) if v is not None else None) for k, v in make_mla_inputs(**cfg, device=str(dev)).items()}
+    ws = torch.empty(kda.mla_decode_workspace_size(cfg["B"], cfg["T"], cfg["H"], cfg["d_q"], cfg["d_v"], cfg["r"]),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(cfg["B"], cfg["H"], cfg["d_v"], dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        kda.mla_decode(x["q"], x["W_UK"], x["W_UV"], x["c"], x["lengths"], o=o, workspace=ws)
+    for i in range(warmup):
+        step(i)
+    # the 268 MB latent cache is larger than L2: no flush needed
+    ms = _time_steps(step, steps, torch.cuda.current_stream(dev), dev, None, 1)
+    sec = (sum(ms) / steps) / 1e3
+    nb, nf = mla_bytes(**cfg), mla_flops(**cfg)
+    roof = _roofline(nb, nf, sec, hbm_peak, peak_kind, MLA_KERNEL_FILE, 6)
+    roof["flop_bound_frac"] = round(nf / sec / 1e12 / bf16_peak, 4)
+    return {"workload": "absorbed MLA decode B64 T4096 H96 d_q=d_v=128 r=512 (bf16)", "steps": steps,
+            "us_per_step": round(sec * 1e6, 2), "tokens_per_s": round(cfg["B"] / sec, 1), "roofline": roof,
+            "kernels_per_call": 3}
+
+
 EXTRA_STEPS = {1: 200, 2: 200, 3: 40, 4: 20}
 
 
@@ -390,6 +425,8 @@ def run_ours(args, ws, rank, local):
             extras["decode"] = {"workload": workload_config(w5, 1)["workload"], "steps": w5.decode_steps,
                                 "us_per_step": round(mps * 1e3, 2), "tokens_per_s": round(v, 1),
                                 "state_GBps": r["achieved"], "frac": r["frac"], "roofline": r}
+        torch.cuda.empty_cache()
+        extras["mla_decode"] = measure_mla(dev, kda, hbm_peak, peak_kind, measured_peaks()[1])
         line.update(extras)
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(w) if (ws == 1 and not args.no_cpu_baseline) else None

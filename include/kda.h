@@ -281,6 +281,35 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
                         float* dg, float* dbeta, float* dS0, float* dA_log, float* ddt_bias, void* workspace,
                         size_t workspace_bytes, kda_stream_t stream);
 
+/*
+ * kda_mla_decode_workspace_size -- bytes of device workspace kda_mla_decode needs (q_abs and the
+ * per-split partial results), or 0 for sizes it rejects.
+ */
+size_t kda_mla_decode_workspace_size(int B, int T, int H, int d_q, int d_v, int r);
+
+/*
+ * kda_mla_decode -- absorbed MLA decode step: one query token per sequence attends, with softmax, to the
+ * sequence's cached latent vectors, without decompressing keys or values (KDA ledger, derivation DER2,
+ * claim C4: q_abs = q W_UK; score = q_abs c^T; o_lat = softmax(scale score) c; o = o_lat W_UV^T).  The
+ * MLA layer of the K3 architecture uses no positional encoding ("NoPE"), so none is applied.
+ *   q        [B, H, d_q]   bf16     the new token's queries
+ *   W_UK     [H, d_q, r]   bf16     key up-projection, absorbed into q
+ *   W_UV     [H, d_v, r]   bf16     value up-projection, applied to the attended latent
+ *   c        [B, T, r]     bf16     latent cache (shared by every head)
+ *   lengths  [B] int32 in [1, T], or NULL: positions of each sequence that take part (the rest of its
+ *            rows of c are not read)
+ *   scale    softmax scale on the scores; <= 0 selects 1 / sqrt(d_q)
+ *   dtype    KDA_BF16 (the only one built)
+ *   o        [B, H, d_v]   bf16, written
+ *   workspace, workspace_bytes  >= kda_mla_decode_workspace_size(...) bytes, 16-byte aligned, scratch
+ * Constraints: d_q, d_v in {64, 128}; r in {128, 256, 512}; H >= 1; T >= 1.  Scores and the weighted sum
+ * run on the tensor cores with float32 accumulation (q_abs enters them as two bf16 terms); the softmax
+ * and both projections in float32.
+ */
+kda_status kda_mla_decode(const void* q, const void* W_UK, const void* W_UV, const void* c, const int* lengths,
+                          int B, int T, int H, int d_q, int d_v, int r, float scale, kda_dtype dtype, void* o,
+                          void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -257,4 +257,35 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
     return ok();
 }
 
+static bool mla_sizes_ok(int B, int T, int H, int d_q, int d_v, int r) {
+    return B >= 1 && T >= 1 && H >= 1 && (d_q == 64 || d_q == 128) && (d_v == 64 || d_v == 128) &&
+           (r == 128 || r == 256 || r == 512) && (long long)B * T * r < (1ll << 40) && (long long)B * H < (1ll << 24);
+}
+
+size_t kda_mla_decode_workspace_size(int B, int T, int H, int d_q, int d_v, int r) {
+    return mla_sizes_ok(B, T, H, d_q, d_v, r) ? kda::mla_workspace(B, T, H, r) : 0;
+}
+
+kda_status kda_mla_decode(const void* q, const void* W_UK, const void* W_UV, const void* c, const int* lengths, int B,
+                          int T, int H, int d_q, int d_v, int r, float scale, kda_dtype dtype, void* o,
+                          void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+    if (!q || !W_UK || !W_UV || !c || !o) return fail(KDA_ERR_INVALID_ARG, "null tensor pointer (q, W_UK, W_UV, c, o)");
+    if (B < 1 || T < 1 || H < 1) return fail(KDA_ERR_INVALID_ARG, "sizes must be >= 1 (B=%d T=%d H=%d)", B, T, H);
+    if (dtype != KDA_BF16) return fail(KDA_ERR_UNSUPPORTED, "kda_mla_decode is built for bf16 only");
+    if (!mla_sizes_ok(B, T, H, d_q, d_v, r))
+        return fail(KDA_ERR_UNSUPPORTED, "unsupported sizes (d_q, d_v in {64, 128}; r in {128, 256, 512})");
+    const void* ptrs[] = {q, W_UK, W_UV, c, lengths, o, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    const size_t need = kda::mla_workspace(B, T, H, r);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace of at least %zu bytes is required (got %zu)", need, workspace_bytes);
+    if (o == q || o == c || o == W_UK || o == W_UV) return fail(KDA_ERR_INVALID_ARG, "o must not alias an input");
+    if (!(scale > 0.0f)) scale = 1.0f / std::sqrt((float)d_q);
+    kda::MlaArgs a{q, W_UK, W_UV, c, lengths, B, T, H, d_q, d_v, r, scale, o, workspace, (cudaStream_t)stream};
+    const cudaError_t e = kda::launch_mla_decode(a);
+    if (e != cudaSuccess) return cuda_fail(e, "MLA decode kernel launch");
+    return ok();
+}
+
 }  // extern "C"

@@ -63,6 +63,16 @@ struct BackwardArgs {
     cudaStream_t stream;
 };
 
+struct MlaArgs {
+    const void *q, *W_UK, *W_UV, *c;
+    const int* lengths;
+    int B, T, H, d_q, d_v, R;
+    float scale;
+    void* o;
+    void* workspace;
+    cudaStream_t stream;
+};
+
 // Status word values written by kernels with bounded waits.
 enum : unsigned int { STATUS_OK = 0u, STATUS_TIMEOUT = 1u };
 
@@ -87,6 +97,11 @@ cudaError_t launch_chunk_split(const ChunkArgs& a);
 // Reverse mode: saved states every few tokens, backward_workspace(B, T, HV, K, V) bytes.
 size_t backward_workspace(int B, int T, int HV, int K, int V);
 cudaError_t launch_backward(const BackwardArgs& a);
+
+// Absorbed MLA decode: q_abs, the per-split partial results; mla_workspace(B, T, H, R) bytes.
+int mla_nsplit(int B, int T, int H);
+size_t mla_workspace(int B, int T, int H, int R);
+cudaError_t launch_mla_decode(const MlaArgs& a);
 
 // Bytes of status block at the start of every chunk-prefill workspace.
 constexpr size_t kChunkStatusBytes = 256;

@@ -1,0 +1,411 @@
+// kda_mla.cu -- absorbed MLA decode: one query token per sequence against its cached latent vectors.
+//
+// KDA ledger, derivation DER2 ("MLA 矩阵吸收推导", claim C4): the query absorbs the key up-projection
+// and meets the latent cache directly, so K and V are never decompressed:
+//   1. q_abs = q . W_UK                   [B, H, r]      (W_UK [H, d_q, r])
+//   2. score = q_abs . c^T                 [B, H, T]      (c [B, T, r], shared by every head)
+//   3. o_lat = softmax(scale score) . c    [B, H, r]
+//   4. o     = o_lat . W_UV^T              [B, H, d_v]    (W_UV [H, d_v, r])
+// (the K3 MLA layer: global softmax attention without positional encoding).  Three kernels:
+//   mla_qabs_kernel    step 1 on the CUDA cores; q_abs is kept as two bf16 terms, hi + lo, so that the
+//                      tensor-core scores carry about 16 mantissa bits of it;
+//   mla_attend_kernel  steps 2-3 with bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation):
+//                      one CTA per (sequence, group of 48 heads, split of the positions) streams its
+//                      latent tiles once through shared memory, with an online softmax;
+//   mla_out_kernel     merges the splits and applies step 4 on the CUDA cores.
+// Every head reads the same latent vectors, so the CTA covers as many heads as its registers allow and
+// the cache crosses HBM once per head group.
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+using bf16 = __nv_bfloat16;
+
+namespace {
+
+constexpr int MLA_GH = 48;              // heads per CTA: three m16 tiles
+constexpr int MLA_TP = 32;              // positions per latent tile
+constexpr int MLA_WARPS = 12;           // (3 head tiles) x (4 position / value quarters)
+constexpr int MLA_THREADS = 32 * MLA_WARPS;
+
+template <int R>
+struct MlaSmem {
+    static constexpr int PITCH = R + 8;  // bf16 elements per row: conflict-free fragment loads
+    static constexpr int PP = MLA_TP + 8;
+    static constexpr size_t QA = 0;                                      // hi, lo: [48][PITCH] bf16 each
+    static constexpr size_t CT = QA + 2 * (size_t)MLA_GH * PITCH * 2;    // latent tiles: 2 x [32][PITCH] bf16
+    static constexpr size_t PB = CT + 2 * (size_t)MLA_TP * PITCH * 2;    // probabilities: 2 x [48][PP] bf16
+    static constexpr size_t ST = PB + 2 * (size_t)MLA_GH * PP * 2;       // row statistics (floats)
+    // ST: max partials 2 x [4][48], sum partials 2 x [4][48], running max 2 x [48], running sum [48]
+    static constexpr size_t BYTES = ST + (2 * 4 * MLA_GH + 2 * 4 * MLA_GH + 2 * MLA_GH + MLA_GH) * 4;
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t ld_u32(const bf16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two 8x8 b16 matrices from rows k0 .. k0 + 15 of a row-major [K][N] shared tile (lanes 0-15 give the
+// row addresses), transposed into the B fragment of an m16n8k16 MMA.
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& b0, uint32_t& b1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(b0), "=r"(b1) : "r"(addr));
+}
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool ok) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(ok ? 16u : 0u) : "memory");
+}
+
+}  // namespace
+
+// ---- step 1: q_abs = q W_UK per head, as bf16 hi + lo ------------------------------------------
+// Grid (H, R / 128, ceil(B / 16)); thread = one latent column, 16 sequences per CTA.
+template <int DQ, int R>
+__global__ void __launch_bounds__(128)
+mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B, int H, bf16* __restrict__ qa_hi,
+                bf16* __restrict__ qa_lo) {
+    __shared__ float sq[16][DQ];
+    const int h = blockIdx.x, col = blockIdx.y * 128 + threadIdx.x, b0 = blockIdx.z * 16;
+    for (int i = threadIdx.x; i < 16 * DQ; i += 128) {
+        const int bb = i / DQ, d = i - bb * DQ;
+        sq[bb][d] = (b0 + bb < B) ? __bfloat162float(q[((size_t)(b0 + bb) * H + h) * DQ + d]) : 0.f;
+    }
+    __syncthreads();
+    float acc[16];
+#pragma unroll
+    for (int bb = 0; bb < 16; ++bb) acc[bb] = 0.f;
+    const bf16* w = W_UK + (size_t)h * DQ * R + col;
+#pragma unroll 4
+    for (int d = 0; d < DQ; ++d) {
+        const float wv = __bfloat162float(w[(size_t)d * R]);
+#pragma unroll
+        for (int bb = 0; bb < 16; ++bb) acc[bb] = fmaf(sq[bb][d], wv, acc[bb]);
+    }
+#pragma unroll
+    for (int bb = 0; bb < 16; ++bb) {
+        if (b0 + bb >= B) break;
+        const bf16 hi = __float2bfloat16_rn(acc[bb]);
+        const size_t idx = ((size_t)(b0 + bb) * H + h) * R + col;
+        qa_hi[idx] = hi;
+        qa_lo[idx] = __float2bfloat16_rn(acc[bb] - __bfloat162float(hi));
+    }
+}
+
+// ---- steps 2-3: scores, online softmax, weighted latent sum -------------------------------------
+// Grid (B, ceil(H / 48), NSPLIT).  Warp w: head tile m = w / 4 (16 heads); for the scores it owns the 8
+// positions 8 (w % 4) of each 32-position tile, for the weighted sum the latent columns
+// (R / 4) (w % 4) .. + R / 4.  Writes the unnormalised o_lat, the running max and the running sum of
+// its split to the workspace.
+template <int R>
+__global__ void __launch_bounds__(MLA_THREADS, 1)
+mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo, const bf16* __restrict__ c,
+                  const int* __restrict__ lengths, int T, int H, int nsplit, int split_len, float scale_log2,
+                  float* __restrict__ part_o, float* __restrict__ part_ml) {
+    using Sm = MlaSmem<R>;
+    constexpr int P = Sm::PITCH, PP = Sm::PP;
+    constexpr int NC = R / 4;       // latent columns per warp in the weighted sum
+    constexpr int NT8 = NC / 8;     // n8 tiles per warp
+    extern __shared__ __align__(16) unsigned char msm[];
+    bf16* sQh = reinterpret_cast<bf16*>(msm + Sm::QA);
+    bf16* sQl = sQh + MLA_GH * P;
+    bf16* sC = reinterpret_cast<bf16*>(msm + Sm::CT);
+    bf16* sP = reinterpret_cast<bf16*>(msm + Sm::PB);
+    float* sMaxP = reinterpret_cast<float*>(msm + Sm::ST);  // 2 x [4][48]
+    float* sSumP = sMaxP + 2 * 4 * MLA_GH;                   // 2 x [4][48]
+    float* sM = sSumP + 2 * 4 * MLA_GH;                      // 2 x [48]
+    float* sL = sM + 2 * MLA_GH;                             // [48]
+
+    const int b = blockIdx.x, hg = blockIdx.y, split = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m = warp >> 2, quarter = warp & 3;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int len = lengths ? min(max(lengths[b], 0), T) : T;
+    const int p0 = split * split_len, p1 = min(len, p0 + split_len);
+    const int ntiles = p1 > p0 ? (p1 - p0 + MLA_TP - 1) / MLA_TP : 0;
+    const uint32_t c_base = (uint32_t)__cvta_generic_to_shared(sC);
+
+    // q_abs of this head group (rows past H are zero)
+    for (int i = tid; i < MLA_GH * (R / 8); i += MLA_THREADS) {
+        const int row = i / (R / 8), ch = i - row * (R / 8);
+        const int h = hg * MLA_GH + row;
+        uint4 vh = make_uint4(0u, 0u, 0u, 0u), vl = vh;
+        if (h < H) {
+            vh = *reinterpret_cast<const uint4*>(qa_hi + ((size_t)b * H + h) * R + 8 * ch);
+            vl = *reinterpret_cast<const uint4*>(qa_lo + ((size_t)b * H + h) * R + 8 * ch);
+        }
+        *reinterpret_cast<uint4*>(sQh + row * P + 8 * ch) = vh;
+        *reinterpret_cast<uint4*>(sQl + row * P + 8 * ch) = vl;
+    }
+    if (tid < MLA_GH) {
+        sM[tid] = -INFINITY;
+        sM[MLA_GH + tid] = -INFINITY;
+        sL[tid] = 0.f;
+    }
+    auto load_tile = [&](int tile, int buf) {  // positions past len read as zeros (masked below)
+        const int pos0 = p0 + tile * MLA_TP;
+        for (int i = tid; i < MLA_TP * (R / 8); i += MLA_THREADS) {
+            const int row = i / (R / 8), ch = i - row * (R / 8);
+            const int pos = pos0 + row;
+            const bool ok = pos < p1;
+            cp_async16_zfill(c_base + (uint32_t)(((buf * MLA_TP + row) * P + 8 * ch) * 2),
+                             ok ? (const void*)(c + ((size_t)b * T + pos) * R + 8 * ch) : (const void*)c, ok);
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    if (ntiles > 0) load_tile(0, 0);
+
+    float acc[NT8][4];
+#pragma unroll
+    for (int j = 0; j < NT8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+    for (int tile = 0; tile < ntiles; ++tile) {
+        const int buf = tile & 1, par = tile & 1;
+        // the next tile streams into the other buffer (the previous tile's, released by the barrier that
+        // ended the previous iteration) while this one is computed
+        if (tile + 1 < ntiles) {
+            load_tile(tile + 1, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+        }
+        __syncthreads();  // this tile has landed for every thread
+        const bf16* cT = sC + buf * MLA_TP * P;
+        // ---- scores for 16 heads x 8 positions: (q_hi + q_lo) . c over the R latent columns ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const bf16* qh = sQh + (16 * m) * P;
+            const bf16* ql = sQl + (16 * m) * P;
+            const bf16* cn = cT + (8 * quarter + g) * P;  // B fragment: column n = position g
+#pragma unroll 4
+            for (int k = 0; k < R; k += 16) {
+                const uint32_t b0 = ld_u32(cn + k + 2 * t4), b1 = ld_u32(cn + k + 2 * t4 + 8);
+                mma_bf16(s, ld_u32(qh + g * P + k + 2 * t4), ld_u32(qh + (g + 8) * P + k + 2 * t4),
+                         ld_u32(qh + g * P + k + 2 * t4 + 8), ld_u32(qh + (g + 8) * P + k + 2 * t4 + 8), b0, b1);
+                mma_bf16(s, ld_u32(ql + g * P + k + 2 * t4), ld_u32(ql + (g + 8) * P + k + 2 * t4),
+                         ld_u32(ql + g * P + k + 2 * t4 + 8), ld_u32(ql + (g + 8) * P + k + 2 * t4 + 8), b0, b1);
+            }
+        }
+        // scale into the log2 domain, mask positions past the split's end
+        const int posc = p0 + tile * MLA_TP + 8 * quarter + 2 * t4;
+        const bool v0 = posc < p1, v1 = posc + 1 < p1;
+        s[0] = v0 ? s[0] * scale_log2 : -INFINITY;
+        s[1] = v1 ? s[1] * scale_log2 : -INFINITY;
+        s[2] = v0 ? s[2] * scale_log2 : -INFINITY;
+        s[3] = v1 ? s[3] * scale_log2 : -INFINITY;
+        // row maxima over this warp's 8 positions (rows g and g + 8 of the head tile)
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const int r0 = 16 * m + g, r1 = r0 + 8;
+        float* maxp = sMaxP + par * 4 * MLA_GH;
+        float* sump = sSumP + par * 4 * MLA_GH;
+        if (t4 == 0) {
+            maxp[quarter * MLA_GH + r0] = mx0;
+            maxp[quarter * MLA_GH + r1] = mx1;
+        }
+        __syncthreads();
+        // new running maxima (every warp computes the same values), probabilities to shared memory
+        const float* mold = sM + par * MLA_GH;
+        auto new_max = [&](int r) {
+            return fmaxf(mold[r], fmaxf(fmaxf(maxp[r], maxp[MLA_GH + r]), fmaxf(maxp[2 * MLA_GH + r], maxp[3 * MLA_GH + r])));
+        };
+        const float mn0 = new_max(r0), mn1 = new_max(r1);
+        const float e0 = exp2f(s[0] - mn0), e1 = exp2f(s[1] - mn0), e2 = exp2f(s[2] - mn1), e3 = exp2f(s[3] - mn1);
+        bf16* Pt = sP + par * MLA_GH * PP;
+        *reinterpret_cast<__nv_bfloat162*>(Pt + r0 * PP + 8 * quarter + 2 * t4) = __floats2bfloat162_rn(e0, e1);
+        *reinterpret_cast<__nv_bfloat162*>(Pt + r1 * PP + 8 * quarter + 2 * t4) = __floats2bfloat162_rn(e2, e3);
+        float sm0 = e0 + e1, sm1 = e2 + e3;
+        sm0 += __shfl_xor_sync(0xffffffffu, sm0, 1);
+        sm0 += __shfl_xor_sync(0xffffffffu, sm0, 2);
+        sm1 += __shfl_xor_sync(0xffffffffu, sm1, 1);
+        sm1 += __shfl_xor_sync(0xffffffffu, sm1, 2);
+        if (t4 == 0) {
+            sump[quarter * MLA_GH + r0] = sm0;
+            sump[quarter * MLA_GH + r1] = sm1;
+        }
+        __syncthreads();
+        // ---- rescale the accumulators and add P . c for this warp's latent columns -----------------
+        const float a0 = exp2f(mold[r0] - mn0), a1 = exp2f(mold[r1] - mn1);
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+            acc[j][0] *= a0;
+            acc[j][1] *= a0;
+            acc[j][2] *= a1;
+            acc[j][3] *= a1;
+        }
+        if (quarter == 0 && t4 == 0) {  // running sums and maxima for the next tile (other parity)
+            sL[r0] = a0 * sL[r0] + sump[r0] + sump[MLA_GH + r0] + sump[2 * MLA_GH + r0] + sump[3 * MLA_GH + r0];
+            sL[r1] = a1 * sL[r1] + sump[r1] + sump[MLA_GH + r1] + sump[2 * MLA_GH + r1] + sump[3 * MLA_GH + r1];
+            sM[(par ^ 1) * MLA_GH + r0] = mn0;
+            sM[(par ^ 1) * MLA_GH + r1] = mn1;
+        }
+        const bf16* pa = Pt + (16 * m) * PP;
+#pragma unroll
+        for (int kk = 0; kk < MLA_TP; kk += 16) {
+            const uint32_t a_0 = ld_u32(pa + g * PP + kk + 2 * t4), a_1 = ld_u32(pa + (g + 8) * PP + kk + 2 * t4);
+            const uint32_t a_2 = ld_u32(pa + g * PP + kk + 2 * t4 + 8), a_3 = ld_u32(pa + (g + 8) * PP + kk + 2 * t4 + 8);
+            // lanes 0-15 address rows kk .. kk + 15 of the latent tile at this warp's column block
+            const int lrow = kk + (lane & 15);
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+                uint32_t b0, b1;
+                const uint32_t addr = c_base + (uint32_t)(((buf * MLA_TP + lrow) * P + NC * quarter + 8 * j) * 2);
+                ldmatrix_x2_trans(b0, b1, addr);
+                mma_bf16(acc[j], a_0, a_1, a_2, a_3, b0, b1);
+            }
+        }
+        __syncthreads();  // every warp is done with this tile's buffers before they are refilled
+    }
+    // ---- this split's unnormalised o_lat, running max (log2 domain) and sum ---------------------------
+    const int par_end = ntiles & 1;
+#pragma unroll
+    for (int j = 0; j < NT8; ++j) {
+        const int col = NC * quarter + 8 * j + 2 * t4;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int row = 16 * m + g + 8 * half, h = hg * MLA_GH + row;
+            if (h >= H) continue;
+            float* dst = part_o + (((size_t)blockIdx.x * nsplit + split) * H + h) * R + col;
+            *reinterpret_cast<float2*>(dst) = make_float2(acc[j][2 * half], acc[j][2 * half + 1]);
+        }
+    }
+    if (tid < MLA_GH) {
+        const int h = hg * MLA_GH + tid;
+        if (h < H) {
+            float* ml = part_ml + (((size_t)blockIdx.x * nsplit + split) * H + h) * 2;
+            ml[0] = sM[par_end * MLA_GH + tid];
+            ml[1] = sL[tid];
+        }
+    }
+}
+
+// ---- merge the splits and step 4: o = (o_lat / l) W_UV^T ---------------------------------------
+// Grid (H, ceil(B / 8)); 256 threads.  The merged o_lat of 8 sequences goes to shared memory, then
+// thread v (of d_v) and batch row b accumulate over the latent columns, W_UV read in 32-column tiles.
+template <int DV, int R>
+__global__ void __launch_bounds__(256)
+mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, const bf16* __restrict__ W_UV,
+               int B, int H, int nsplit, bf16* __restrict__ o) {
+    __shared__ float so[8][R];
+    __shared__ float sw[DV][33];
+    const int h = blockIdx.x, b0 = blockIdx.y * 8, tid = threadIdx.x;
+    // merge: o_lat = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s
+    for (int i = tid; i < 8 * R; i += 256) {
+        const int bb = i / R, col = i - bb * R, b = b0 + bb;
+        float val = 0.f;
+        if (b < B) {
+            float M = -INFINITY;
+            for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, part_ml[(((size_t)b * nsplit + sp) * H + h) * 2]);
+            float num = 0.f, den = 0.f;
+            for (int sp = 0; sp < nsplit; ++sp) {
+                const float* ml = part_ml + (((size_t)b * nsplit + sp) * H + h) * 2;
+                if (ml[0] == -INFINITY) continue;  // an empty split
+                const float w = exp2f(ml[0] - M);
+                num += w * part_o[(((size_t)b * nsplit + sp) * H + h) * R + col];
+                den += w * ml[1];
+            }
+            val = num / den;
+        }
+        so[bb][col] = val;
+    }
+    // thread (v = tid % DV, batch rows bb = tid / DV + k * (256 / DV))
+    constexpr int BPT = 8 / (256 / DV);  // batch rows per thread
+    const int v = tid % DV, bq = tid / DV;
+    float acc[BPT];
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) acc[i] = 0.f;
+    const bf16* w = W_UV + (size_t)h * DV * R;
+    for (int k0 = 0; k0 < R; k0 += 32) {
+        __syncthreads();  // previous W tile consumed (and o_lat merged, on the first pass)
+        for (int i = tid; i < DV * 32; i += 256) {
+            const int vv = i / 32, kk = i - vv * 32;
+            sw[vv][kk] = __bfloat162float(w[(size_t)vv * R + k0 + kk]);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            const float wv = sw[v][kk];
+#pragma unroll
+            for (int i = 0; i < BPT; ++i) acc[i] = fmaf(so[bq + i * (256 / DV)][k0 + kk], wv, acc[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+        const int b = b0 + bq + i * (256 / DV);
+        if (b < B) o[((size_t)b * H + h) * DV + v] = __float2bfloat16_rn(acc[i]);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+int mla_nsplit(int B, int T, int H) {
+    // as many (sequence, head group, split) CTAs as a B200 has SMs at most (one wave of one CTA per SM),
+    // splits of at least 256 positions
+    const long long groups = (long long)B * ((H + MLA_GH - 1) / MLA_GH);
+    int ns = (int)(148 / groups);
+    const int maxs = (T + 255) / 256;
+    if (ns > maxs) ns = maxs;
+    return ns < 1 ? 1 : ns;
+}
+
+size_t mla_workspace(int B, int T, int H, int R) {
+    const int ns = mla_nsplit(B, T, H);
+    return 2 * (size_t)B * H * R * sizeof(bf16) + (size_t)B * ns * H * R * sizeof(float) +
+           (size_t)B * ns * H * 2 * sizeof(float);
+}
+
+namespace {
+template <int DQ, int DV, int R>
+cudaError_t launch_mla_t(const MlaArgs& a) {
+    const int ns = mla_nsplit(a.B, a.T, a.H);
+    const int split_len = (a.T + ns - 1) / ns;
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    bf16* qa_hi = reinterpret_cast<bf16*>(ws);
+    bf16* qa_lo = qa_hi + (size_t)a.B * a.H * R;
+    float* part_o = reinterpret_cast<float*>(qa_lo + (size_t)a.B * a.H * R);
+    float* part_ml = part_o + (size_t)a.B * ns * a.H * R;
+    const bf16* q = static_cast<const bf16*>(a.q);
+    mla_qabs_kernel<DQ, R><<<dim3(a.H, R / 128, (a.B + 15) / 16), 128, 0, a.stream>>>(
+        q, static_cast<const bf16*>(a.W_UK), a.B, a.H, qa_hi, qa_lo);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    using Sm = MlaSmem<R>;
+    e = cudaFuncSetAttribute(mla_attend_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sm::BYTES);
+    if (e != cudaSuccess) return e;
+    const float scale_log2 = a.scale * 1.4426950408889634f;  // softmax with exp2: scores times log2(e)
+    mla_attend_kernel<R><<<dim3(a.B, (a.H + MLA_GH - 1) / MLA_GH, ns), MLA_THREADS, Sm::BYTES, a.stream>>>(
+        qa_hi, qa_lo, static_cast<const bf16*>(a.c), a.lengths, a.T, a.H, ns, split_len, scale_log2, part_o, part_ml);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mla_out_kernel<DV, R><<<dim3(a.H, (a.B + 7) / 8), 256, 0, a.stream>>>(part_o, part_ml,
+                                                                          static_cast<const bf16*>(a.W_UV), a.B, a.H,
+                                                                          ns, static_cast<bf16*>(a.o));
+    return cudaGetLastError();
+}
+
+template <int DQ, int DV>
+cudaError_t mla_r(const MlaArgs& a) {
+    switch (a.R) {
+        case 128: return launch_mla_t<DQ, DV, 128>(a);
+        case 256: return launch_mla_t<DQ, DV, 256>(a);
+        case 512: return launch_mla_t<DQ, DV, 512>(a);
+    }
+    return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_mla_decode(const MlaArgs& a) {
+    if (a.d_q == 64 && a.d_v == 64) return mla_r<64, 64>(a);
+    if (a.d_q == 128 && a.d_v == 128) return mla_r<128, 128>(a);
+    if (a.d_q == 64 && a.d_v == 128) return mla_r<64, 128>(a);
+    if (a.d_q == 128 && a.d_v == 64) return mla_r<128, 64>(a);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -114,3 +114,25 @@ def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu", raw: 
 
 def default_scale(K: int) -> float:
     return 1.0 / math.sqrt(K)
+
+
+# Absorbed MLA decode, with the MLA sizes of the real K3 configuration (H = 96 heads, head dimension
+# 128, kv_lora_rank r = 512) and a decode batch of 64 sequences with 4096 cached latent positions each.
+MLA_DECODE = dict(B=64, T=4096, H=96, d_q=128, d_v=128, r=512)
+
+
+def make_mla_inputs(B, T, H, d_q, d_v, r, seed=1006, device="cpu", ragged=False) -> dict:
+    """q ~ N(0,1) [B,H,d_q]; W_UK ~ N(0,1/d_q) [H,d_q,r]; W_UV ~ N(0,1/r) [H,d_v,r]; c ~ N(0,1) [B,T,r];
+    all bf16.  With ``ragged`` the lengths are drawn uniformly in [1, T] (int32), else None."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    q = torch.randn(B, H, d_q, **f32)
+    W_UK = torch.randn(H, d_q, r, **f32) / math.sqrt(d_q)
+    W_UV = torch.randn(H, d_v, r, **f32) / math.sqrt(r)
+    c = torch.randn(B, T, r, **f32)
+    lengths = None
+    if ragged:
+        lengths = torch.randint(1, T + 1, (B,), generator=gen, device=device, dtype=torch.int64).to(torch.int32)
+    bf = torch.bfloat16
+    return dict(q=q.to(bf), W_UK=W_UK.to(bf), W_UV=W_UV.to(bf), c=c.to(bf), lengths=lengths)

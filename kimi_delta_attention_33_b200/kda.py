@@ -35,7 +35,7 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 EXPORTS = ("kda_last_error", "kda_version", "kda_gate", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
            "kda_chunk_fwd_ex", "kda_chunk_fwd_schedule", "kda_read_status", "kda_chunk_fwd_noalloc",
            "kda_chunk_fwd_noalloc_read_status", "kda_recurrent_step", "kda_recurrent_step_ex",
-           "kda_backward_workspace_size", "kda_backward")
+           "kda_backward_workspace_size", "kda_backward", "kda_mla_decode_workspace_size", "kda_mla_decode")
 INPUT_RAW, INPUT_L2NORM_QK, INPUT_BETA_LOGITS = 0, 1, 2
 SCHEDULE_CUDA_CORE, SCHEDULE_TC_SINGLE_PASS, SCHEDULE_TC_TWO_PASS, SCHEDULE_TC_TWO_PASS_SCAN = 0, 1, 2, 3
 SCHEDULE_NAMES = {0: "cuda_core", 1: "tc_single_pass", 2: "tc_two_pass", 3: "tc_two_pass_scan"}
@@ -90,6 +90,12 @@ lib.kda_backward_workspace_size.argtypes = [_i] * 6
 lib.kda_backward.restype = _i
 lib.kda_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _fp, _fp, _vp, _fp] + [_i] * 6 + [_i, _f, _f, _i] + \
     [_fp] * 8 + [_vp, _sz, _vp]
+
+
+lib.kda_mla_decode_workspace_size.restype = _sz
+lib.kda_mla_decode_workspace_size.argtypes = [_i] * 6
+lib.kda_mla_decode.restype = _i
+lib.kda_mla_decode.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 6 + [_f, _i, _vp, _vp, _sz, _vp]
 
 
 def version() -> str:
@@ -291,6 +297,32 @@ def backward(q, k, v, g, beta, dO, A_log=None, dt_bias=None, S0=None, dS_T=None,
                             _ptr(o["dq"]), _ptr(o["dk"]), _ptr(o["dv"]), _ptr(o["dg"]), _ptr(o["dbeta"]),
                             _ptr(o.get("dS0")), _ptr(o.get("dA_log")), _ptr(o.get("ddt_bias")), _ptr(workspace),
                             workspace.numel(), _stream(dev)))
+    return o
+
+
+def mla_decode_workspace_size(B, T, H, d_q, d_v, r) -> int:
+    return int(lib.kda_mla_decode_workspace_size(B, T, H, d_q, d_v, r))
+
+
+def mla_decode(q, W_UK, W_UV, c, lengths=None, *, scale: float | None = None, o: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Absorbed MLA decode (``kda_mla_decode``).  q [B,H,d_q], W_UK [H,d_q,r], W_UV [H,d_v,r], c [B,T,r] (bf16);
+    lengths [B] int32 or None.  Returns o [B,H,d_v] bf16."""
+    _require_cuda(q, W_UK, W_UV, c, lengths)
+    B, H, d_q = q.shape
+    T, r = c.shape[1], c.shape[2]
+    d_v = W_UV.shape[1]
+    if o is None:
+        o = torch.empty(B, H, d_v, dtype=q.dtype, device=q.device)
+    _require_out(o, (B, H, d_v), q.dtype)
+    if lengths is not None and lengths.dtype != torch.int32:
+        raise KdaError(ERR_INVALID_ARG, "lengths must be int32")
+    need = mla_decode_workspace_size(B, T, H, d_q, d_v, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    sc = -1.0 if scale is None else float(scale)
+    _check(lib.kda_mla_decode(_ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(c), _ptr(lengths), B, T, H, d_q, d_v, r, sc,
+                              _dtype_code(q), _ptr(o), _ptr(workspace), workspace.numel(), _stream(q.device)))
     return o
 
 

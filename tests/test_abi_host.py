@@ -189,3 +189,23 @@ def test_backward_validates_before_launch():
     assert call(ws_bytes=1024) == kda.ERR_INVALID_ARG
     assert call(dq=FAKE) == kda.ERR_INVALID_ARG  # an output aliasing an input
     assert kda.last_error() != ""
+
+
+def test_mla_decode_validates_before_launch():
+    L = kda.lib
+    assert kda.mla_decode_workspace_size(64, 4096, 96, 128, 128, 512) > 0
+    assert kda.mla_decode_workspace_size(64, 4096, 96, 96, 128, 512) == 0
+    assert kda.mla_decode_workspace_size(64, 4096, 96, 128, 128, 1024) == 0
+
+    def call(**over):
+        a = dict(q=FAKE, o=FAKE * 5, dq=128, r=512, dtype=kda.BF16, ws=1 << 30, H=96)
+        a.update(over)
+        return L.kda_mla_decode(a["q"], FAKE * 2, FAKE * 3, FAKE * 4, None, 4, 64, a["H"], a["dq"], 128, a["r"], -1.0,
+                                a["dtype"], a["o"], FAKE * 6, a["ws"], None)
+    assert call(q=None) == kda.ERR_INVALID_ARG
+    assert call(dq=96) == kda.ERR_UNSUPPORTED
+    assert call(r=64) == kda.ERR_UNSUPPORTED
+    assert call(dtype=kda.F32) == kda.ERR_UNSUPPORTED
+    assert call(ws=16) == kda.ERR_INVALID_ARG
+    assert call(o=FAKE) == kda.ERR_INVALID_ARG
+    assert call(H=0) == kda.ERR_INVALID_ARG
