@@ -366,11 +366,63 @@ def measure_mla(dev, kda, hbm_peak, peak_kind, bf16_peak, steps=50, warmup=3):
             "kernels_per_call": 3}
 
 
+def backward_bytes(w) -> int:
+    """Reverse mode: the forward inputs and dO read (dtype), S0 if any; dq, dk, dv, dg, dbeta, dS0 written (fp32)."""
+    e = elt_bytes(w)
+    B, T, H, HV, K, V = w.B, w.T, w.H, w.HV, w.K, w.V
+    rd = 2 * B * T * H * K * e + 2 * B * T * HV * V * e + B * T * HV * K * e + B * T * HV * e + HV * 4 + HV * K * 4
+    if w.S0_std is not None:
+        rd += B * HV * K * V * 4
+    wr = 4 * (2 * B * T * H * K + B * T * HV * V + B * T * HV * K + B * T * HV + B * HV * K * V + HV + HV * K)
+    return rd + wr
+
+
+def measure_backward(dev, kda, hbm_peak, peak_kind, wid=2, steps=10, warmup=3):
+    """kda_backward on a prefill workload's shape (gradients of every input, gate included)."""
+    w = WORKLOADS[wid]
+    x = make_inputs(w, seed=rank_seed(w, 0), device=str(dev))
+    gen = torch.Generator(device=str(dev)).manual_seed(5)
+    dO = torch.randn(w.B, w.T, w.HV, w.V, generator=gen, device=dev).to(w.dtype)
+    out = {}
+    ws = torch.empty(kda.backward_workspace_size(w.B, w.T, w.H, w.HV, w.K, w.V), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, x["A_log"], x["dt_bias"], x["S0"], None,
+                     gate_mode=w.gate_mode, lower_bound=w.lower_bound, workspace=ws, out=out)
+    step(0)  # fills `out`; later calls reuse its buffers
+    for i in range(warmup):
+        step(i)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ms = _time_steps(step, steps, torch.cuda.current_stream(dev), dev, flush, 1)
+    sec = (sum(ms) / steps) / 1e3
+    roof = _roofline(backward_bytes(w), 0, sec, hbm_peak, peak_kind, "kimi_delta_attention_33_b200/csrc/kda_backward.cu",
+                     wid)
+    return {"workload": f"reverse mode on workload {wid}: {w.name}", "steps": steps, "ms_per_step": round(sec * 1e3, 4),
+            "tokens_per_s": round(w.B * w.T / sec, 1), "roofline": roof, "bound_note": "CUDA cores, latency of the "
+            "per-token reductions; the HBM roofline is given for reference"}
+
+
 EXTRA_STEPS = {1: 200, 2: 200, 3: 40, 4: 20}
+
+
+def run_mla_only(args, ws, rank, local):
+    """`--workload 6`: the absorbed MLA decode alone (profiler captures and quick looks; not the headline)."""
+    from kimi_delta_attention_33_b200 import kda
+    dev = torch.device("cuda", local)
+    hbm_peak, bf16_peak, peak_kind = measured_peaks()
+    r = measure_mla(dev, kda, hbm_peak, peak_kind, bf16_peak, steps=args.steps, warmup=args.warmup)
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": r["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["us_per_step"] / 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                          "data": "synthetic", "config": {"workload": r["workload"]}, "roofline": r["roofline"],
+                          "gpu_launches": args.steps * 3}), flush=True)
 
 
 def run_ours(args, ws, rank, local):
     from kimi_delta_attention_33_b200 import kda
+    if args.workload == 6:
+        return run_mla_only(args, ws, rank, local)
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
     if args.B is not None:
@@ -427,6 +479,8 @@ def run_ours(args, ws, rank, local):
                                 "state_GBps": r["achieved"], "frac": r["frac"], "roofline": r}
         torch.cuda.empty_cache()
         extras["mla_decode"] = measure_mla(dev, kda, hbm_peak, peak_kind, measured_peaks()[1])
+        torch.cuda.empty_cache()
+        extras["backward"] = measure_backward(dev, kda, hbm_peak, peak_kind)
         line.update(extras)
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(w) if (ws == 1 and not args.no_cpu_baseline) else None
@@ -570,8 +624,10 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
     ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.workload == 6:
+        return run_reference_mla(args, ws)
+    w = WORKLOADS[args.workload]
     run, desc, threads = _oracle_sample(w, budget_s=2.0)
     for _ in range(args.warmup):
         run()
@@ -587,6 +643,29 @@ def run_reference(args):
                       "note": "the float64 oracle on the host cores; the config's L2 note describes the GPU arm",
                       "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                        "sample": desc + " per step"},
+                      "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def run_reference_mla(args, ws):
+    """The MLA decode oracle on the host, one sequence of the decode workload per step."""
+    from oracle import mla
+    x = make_mla_inputs(**MLA_DECODE)
+    for _ in range(args.warmup):
+        mla.absorbed(x["q"][:1], x["W_UK"], x["W_UV"], x["c"][:1])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        b = i % MLA_DECODE["B"]
+        mla.absorbed(x["q"][b:b + 1], x["W_UK"], x["W_UV"], x["c"][b:b + 1])
+    el = time.perf_counter() - t0
+    v = round(args.steps / el, 2)
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic",
+                      "config": {"workload": "absorbed MLA decode B64 T4096 H96 d_q=d_v=128 r=512 (bf16)"},
+                      "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                                       "sample": "one sequence per step"},
                       "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
           flush=True)
 
@@ -626,7 +705,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6],
+                    help="1-5: the KDA workloads (4, the largest single-GPU prefill, is the headline); "
+                         "6: the absorbed MLA decode alone")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' extra keys")
@@ -641,7 +722,7 @@ def main():
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         sys.exit(relaunch_under_torchrun(args.gpus))
     if args.steps is None:
-        args.steps = {1: 200, 2: 200, 3: 40, 4: 20, 5: 128}[args.workload] if args.impl == "ours" else 10
+        args.steps = {1: 200, 2: 200, 3: 40, 4: 20, 5: 128, 6: 50}[args.workload] if args.impl == "ours" else 10
     if args.dry_plumbing:
         run_dry_plumbing(args)
         return

@@ -870,23 +870,27 @@ scan_chain_kernel(const float* __restrict__ S0, float* __restrict__ carry, int N
 }
 
 // ---------------------------------------------------------------------------------------------
-// Segments of the state pass.  Cost model, in chunk steps of one CTA per SM: the unsplit pass is a
-// chain of NC steps per wave of (pair, value block) CTAs (blocks of 16, 32 or 64 columns, as
-// launch_chunk_split picks them); the split one runs 2 x pairs x (NS - 1) carry CTAs, then pairs x NS output
-// CTAs, of L chunks each, in waves over the SMs, plus the segment chain at about 0.6 step per segment.
-// The number of SMs is a planning constant (a B200's 148), so that the workspace size does not depend
-// on the device; the split is taken only where the model gains at least a quarter.
+// Segments of the state pass.  Cost model, in thousands of cycles of one CTA per SM: the unsplit pass is
+// a chain of NC steps per wave of (pair, value block) CTAs, one step taking about 3.6K cycles with 16
+// columns, 4.8K with 32 and 6K with 64 (as launch_chunk_split picks the block width); the split one runs
+// 2 x pairs x (NS - 1) carry CTAs, then pairs x NS output CTAs, of L chunks each, in waves over the SMs,
+// one 128-column step taking about 10.3K cycles, plus the segment chain at about 3K cycles per segment
+// (measured on B200 with tf32 records).  The split therefore pays only where the unsplit pass leaves SMs
+// idle: few (sequence, head) pairs and long sequences.  The number of SMs is a planning constant (a
+// B200's 148), so that the workspace size does not depend on the device; the split is taken where the
+// model gains at least a fifth.
 ScanPlan chunk_scan_plan(long long pairs, int NC) {
     constexpr long long kPlanSMs = 148;
     const long long nvb = pairs * 8 <= kPlanSMs ? 8 : pairs * 4 <= kPlanSMs ? 4 : 2;
+    const double t_unsplit = nvb == 8 ? 3.6 : nvb == 4 ? 4.8 : 6.0, t_split = 10.3, t_chain = 3.0;
     ScanPlan plan{NC, 1};
-    double best = 0.75 * (double)NC * (double)((pairs * nvb + kPlanSMs - 1) / kPlanSMs);
+    double best = 0.8 * (double)NC * t_unsplit * (double)((pairs * nvb + kPlanSMs - 1) / kPlanSMs);
     for (int Lc : {8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256}) {
         if (Lc >= NC) break;
         const long long NS = (NC + Lc - 1) / Lc;
         const long long wa = (2 * pairs * (NS - 1) + kPlanSMs - 1) / kPlanSMs;
         const long long wc = (pairs * NS + kPlanSMs - 1) / kPlanSMs;
-        const double cost = (double)(wa + wc) * Lc + 0.6 * (double)NS;
+        const double cost = (double)(wa + wc) * Lc * t_split + t_chain * (double)NS;
         if (cost < best) {
             best = cost;
             plan = ScanPlan{Lc, (int)NS};

@@ -275,7 +275,7 @@ def backward(q, k, v, g, beta, dO, A_log=None, dt_bias=None, S0=None, dS_T=None,
     HV, V = v.shape[2], v.shape[3]
     dev = q.device
     f32 = dict(dtype=torch.float32, device=dev)
-    o = dict(out or {})
+    o = out if out is not None else {}
     o.setdefault("dq", torch.empty(B, T, H, K, **f32))
     o.setdefault("dk", torch.empty(B, T, H, K, **f32))
     o.setdefault("dv", torch.empty(B, T, HV, V, **f32))

@@ -46,9 +46,9 @@ def _check(w, x, o, S, n=3):
     assert eS <= TOL[w.dtype], f"S rel err {eS:.3e}"
 
 
-@pytest.mark.parametrize("B,H,HV,T,gate", [(1, 2, 4, 4096 + 37, GATE_SAFE),      # 65 chunks: a 1-chunk last segment
-                                           (2, 2, 2, 2560, GATE_STANDARD),       # 5 segments of 8
-                                           (1, 4, 16, 8192 - 5, GATE_SAFE),      # GVA, 16 pairs
+@pytest.mark.parametrize("B,H,HV,T,gate", [(1, 2, 4, 5000, GATE_SAFE),           # 79 chunks, ragged last chunk
+                                           (2, 2, 2, 9000, GATE_STANDARD),       # a short last segment
+                                           (1, 4, 8, 8192 - 5, GATE_SAFE),       # GVA
                                            (1, 1, 1, 64 * 300 + 63, GATE_STANDARD)])  # one pair, many segments
 def test_scan_ragged_and_segmented(B, H, HV, T, gate):
     w = _wl(B, T, H, HV, gate=gate, A_log=(-1.0, 0.5))
@@ -59,7 +59,7 @@ def test_scan_ragged_and_segmented(B, H, HV, T, gate):
 
 
 def test_scan_without_initial_state_and_bias():
-    w = _wl(1, 5000, 2, 4, S0=None)
+    w = _wl(1, 6000, 1, 1, S0=None)
     x = make_inputs(w)
     x["dt_bias"] = None
     o, S = _run(w, to_dev(x))
@@ -68,7 +68,7 @@ def test_scan_without_initial_state_and_bias():
 
 
 def test_scan_strong_decay_exact_path():
-    w = _wl(1, 3000, 2, 4, dt_mean=6.0)
+    w = _wl(1, 6000, 2, 4, dt_mean=6.0)
     x = make_inputs(w)
     o, S = _run(w, to_dev(x))
     torch.cuda.synchronize()
@@ -76,7 +76,7 @@ def test_scan_strong_decay_exact_path():
 
 
 def test_scan_in_place_state():
-    w = _wl(1, 4200, 2, 4)
+    w = _wl(1, 5000, 2, 2)
     x = make_inputs(w)
     xd = to_dev(x)
     S_buf = xd["S0"].clone()
@@ -88,7 +88,7 @@ def test_scan_in_place_state():
 
 
 def test_scan_agrees_with_single_pass_and_repeats_bit_exactly():
-    w = _wl(2, 6000, 2, 4)
+    w = _wl(2, 8187, 2, 4)
     xd = to_dev(make_inputs(w))
     o1, S1 = _run(w, xd)
     o1b, S1b = _run(w, xd)
