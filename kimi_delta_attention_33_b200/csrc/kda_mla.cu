@@ -35,7 +35,8 @@ struct MlaSmem {
     static constexpr size_t QA = 0;                                      // hi, lo: [48][PITCH] bf16 each
     static constexpr size_t CT = QA + 2 * (size_t)MLA_GH * PITCH * 2;    // latent tiles: 2 x [32][PITCH] bf16
     static constexpr size_t PB = CT + 2 * (size_t)MLA_TP * PITCH * 2;    // probabilities: 2 x [48][PP] bf16
-    static constexpr size_t ST = PB + 2 * (size_t)MLA_GH * PP * 2;       // row statistics (floats)
+    static constexpr size_t SP = PB + 2 * (size_t)MLA_GH * PP * 2;       // score partials: [4][48][32] fp32
+    static constexpr size_t ST = SP + 4 * (size_t)MLA_GH * MLA_TP * 4;   // row statistics (floats)
     // ST: max partials 2 x [4][48], sum partials 2 x [4][48], running max 2 x [48], running sum [48]
     static constexpr size_t BYTES = ST + (2 * 4 * MLA_GH + 2 * 4 * MLA_GH + 2 * MLA_GH + MLA_GH) * 4;
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -50,6 +51,14 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 b16 matrices, lane l giving the address of row l % 8 of matrix l / 8; thread t receives
+// (row t / 4, columns 2 (t % 4) and 2 (t % 4) + 1) of each matrix.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
 
 // Two 8x8 b16 matrices from rows k0 .. k0 + 15 of a row-major [K][N] shared tile (lanes 0-15 give the
@@ -98,10 +107,12 @@ mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B
 }
 
 // ---- steps 2-3: scores, online softmax, weighted latent sum -------------------------------------
-// Grid (B, ceil(H / 48), NSPLIT).  Warp w: head tile m = w / 4 (16 heads); for the scores it owns the 8
-// positions 8 (w % 4) of each 32-position tile, for the weighted sum the latent columns
-// (R / 4) (w % 4) .. + R / 4.  Writes the unnormalised o_lat, the running max and the running sum of
-// its split to the workspace.
+// Grid (B, ceil(H / 48), NSPLIT).  Warp w: head tile m = w / 4 (16 heads) and quarter w % 4.  For the scores
+// the quarter is a quarter of the latent columns: the warp computes partial scores of its 16 heads for all
+// 32 positions of the tile (four independent accumulators; every q_abs fragment is read from shared memory
+// once per tile), and the four partials meet in shared memory.  For the softmax the quarter is 8 positions,
+// for the weighted sum it is a quarter of the latent columns again.  Writes the unnormalised o_lat, the
+// running max and the running sum of its split to the workspace.
 template <int R>
 __global__ void __launch_bounds__(MLA_THREADS, 1)
 mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo, const bf16* __restrict__ c,
@@ -116,6 +127,7 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
     bf16* sQl = sQh + MLA_GH * P;
     bf16* sC = reinterpret_cast<bf16*>(msm + Sm::CT);
     bf16* sP = reinterpret_cast<bf16*>(msm + Sm::PB);
+    float* sSP = reinterpret_cast<float*>(msm + Sm::SP);    // [4][48][32] partial scores
     float* sMaxP = reinterpret_cast<float*>(msm + Sm::ST);  // 2 x [4][48]
     float* sSumP = sMaxP + 2 * 4 * MLA_GH;                   // 2 x [4][48]
     float* sM = sSumP + 2 * 4 * MLA_GH;                      // 2 x [48]
@@ -176,20 +188,57 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
         }
         __syncthreads();  // this tile has landed for every thread
         const bf16* cT = sC + buf * MLA_TP * P;
-        // ---- scores for 16 heads x 8 positions: (q_hi + q_lo) . c over the R latent columns ----
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- partial scores: 16 heads x 32 positions over this warp's quarter of the latent columns,
+        //      (q_hi + q_lo) . c with bf16 MMAs ----------------------------------------------------------
         {
-            const bf16* qh = sQh + (16 * m) * P;
-            const bf16* ql = sQl + (16 * m) * P;
-            const bf16* cn = cT + (8 * quarter + g) * P;  // B fragment: column n = position g
-#pragma unroll 4
-            for (int k = 0; k < R; k += 16) {
-                const uint32_t b0 = ld_u32(cn + k + 2 * t4), b1 = ld_u32(cn + k + 2 * t4 + 8);
-                mma_bf16(s, ld_u32(qh + g * P + k + 2 * t4), ld_u32(qh + (g + 8) * P + k + 2 * t4),
-                         ld_u32(qh + g * P + k + 2 * t4 + 8), ld_u32(qh + (g + 8) * P + k + 2 * t4 + 8), b0, b1);
-                mma_bf16(s, ld_u32(ql + g * P + k + 2 * t4), ld_u32(ql + (g + 8) * P + k + 2 * t4),
-                         ld_u32(ql + g * P + k + 2 * t4 + 8), ld_u32(ql + (g + 8) * P + k + 2 * t4 + 8), b0, b1);
+            float sp[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sp[j][0] = sp[j][1] = sp[j][2] = sp[j][3] = 0.f;
+            const uint32_t qh_base = (uint32_t)__cvta_generic_to_shared(sQh), ql_base = (uint32_t)__cvta_generic_to_shared(sQl);
+            const uint32_t ct_base = c_base + (uint32_t)(buf * MLA_TP * P * 2);
+            // A fragment addresses: lane l -> row 16 m + (l % 8) + 8 ((l / 8) % 2), column + 8 (l / 16)
+            const uint32_t a_off = (uint32_t)(((16 * m + (lane & 7) + 8 * ((lane >> 3) & 1)) * P + 8 * (lane >> 4)) * 2);
+            // B fragment addresses: lane l -> position 8 j + (l % 8), column + 8 (l / 8) (two k16 steps per load)
+            const uint32_t b_off = (uint32_t)(((lane & 7) * P + 8 * (lane >> 3)) * 2);
+            const int k_begin = quarter * (R / 4);
+#pragma unroll
+            for (int k = k_begin; k < k_begin + R / 4; k += 32) {
+                uint32_t ah[2][4], al[2][4];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    ldmatrix_x4(ah[h2][0], ah[h2][1], ah[h2][2], ah[h2][3], qh_base + a_off + (uint32_t)((k + 16 * h2) * 2));
+                    ldmatrix_x4(al[h2][0], al[h2][1], al[h2][2], al[h2][3], ql_base + a_off + (uint32_t)((k + 16 * h2) * 2));
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t b[4];
+                    ldmatrix_x4(b[0], b[1], b[2], b[3], ct_base + b_off + (uint32_t)((8 * j * P + k) * 2));
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        mma_bf16(sp[j], ah[h2][0], ah[h2][1], ah[h2][2], ah[h2][3], b[2 * h2], b[2 * h2 + 1]);
+                        mma_bf16(sp[j], al[h2][0], al[h2][1], al[h2][2], al[h2][3], b[2 * h2], b[2 * h2 + 1]);
+                    }
+                }
             }
+            float* dst = sSP + (size_t)quarter * MLA_GH * MLA_TP;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                *reinterpret_cast<float2*>(dst + (16 * m + g) * MLA_TP + 8 * j + 2 * t4) = make_float2(sp[j][0], sp[j][1]);
+                *reinterpret_cast<float2*>(dst + (16 * m + g + 8) * MLA_TP + 8 * j + 2 * t4) = make_float2(sp[j][2], sp[j][3]);
+            }
+        }
+        __syncthreads();
+        // the scores of 16 heads x this warp's 8 positions: the four partials summed
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+            const float* src = sSP + (size_t)kq * MLA_GH * MLA_TP;
+            const float2 x0 = *reinterpret_cast<const float2*>(src + (16 * m + g) * MLA_TP + 8 * quarter + 2 * t4);
+            const float2 x1 = *reinterpret_cast<const float2*>(src + (16 * m + g + 8) * MLA_TP + 8 * quarter + 2 * t4);
+            s[0] += x0.x;
+            s[1] += x0.y;
+            s[2] += x1.x;
+            s[3] += x1.y;
         }
         // scale into the log2 domain, mask positions past the split's end
         const int posc = p0 + tile * MLA_TP + 8 * quarter + 2 * t4;
