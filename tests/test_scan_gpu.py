@@ -87,15 +87,17 @@ def test_scan_in_place_state():
     _check(w, x, o, S_buf, n=4)
 
 
-def test_scan_agrees_with_single_pass_and_repeats_bit_exactly():
+def test_scan_repeats_bit_exactly_and_matches_single_pass_on_sampled_pairs():
     w = _wl(2, 8187, 2, 4)
-    xd = to_dev(make_inputs(w))
+    x = make_inputs(w)
+    xd = to_dev(x)
     o1, S1 = _run(w, xd)
     o1b, S1b = _run(w, xd)
+    assert torch.equal(o1, o1b) and torch.equal(S1, S1b)  # records and carries left by a call change nothing
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
     o2, S2 = kda.chunk_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"], xd["S0"],
                            chunk=64, gate_mode=w.gate_mode, lower_bound=w.lower_bound, workspace=ws)
     kda.read_status(ws)
-    assert torch.equal(o1, o1b) and torch.equal(S1, S1b)
-    assert rel_err(o1, o2.float().cpu().numpy().astype(np.float64)) <= TOL[w.dtype]
-    assert rel_err(S1, S2.cpu().numpy().astype(np.float64)) <= TOL[w.dtype]
+    torch.cuda.synchronize()
+    _check(w, x, o1, S1, n=3)
+    _check(w, x, o2, S2, n=3)

@@ -138,13 +138,16 @@ def test_short_last_chunk_decay_spans(schedule, c_last):
     assert rel_err(S, S_ref) <= TOL[w.dtype]
 
 
-def test_schedules_agree_with_each_other():
+def test_schedules_agree_on_the_same_call():
+    # both schedules on one set of device inputs, each against the oracle
     w = _wl(B=2, T=333, H=2, HV=6)
-    xd = to_dev(make_inputs(w))
-    o1, S1 = _run(w, xd, "two_pass")
-    o2, S2 = _run(w, xd, "single_pass")
-    assert rel_err(o1, o2.float().cpu().numpy().astype(np.float64)) <= TOL[w.dtype]
-    assert rel_err(S1, S2.cpu().numpy().astype(np.float64)) <= TOL[w.dtype]
+    x = make_inputs(w)
+    xd = to_dev(x)
+    o_ref, S_ref = _ref(w, x)
+    for schedule in SCHEDULES:
+        o, S = _run(w, xd, schedule)
+        assert rel_err(o, o_ref) <= TOL[w.dtype]
+        assert rel_err(S, S_ref) <= TOL[w.dtype]
 
 
 @pytest.mark.parametrize("wid", [2, 4])
