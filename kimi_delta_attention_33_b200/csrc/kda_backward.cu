@@ -110,6 +110,11 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
 
     auto tok_qk = [&](int t) { return ((size_t)b * T + t) * H + h; };      // row of q / k (times K)
     auto tok_v = [&](int t) { return ((size_t)b * T + t) * HV + hv; };     // row of v, g, dO (times V or K)
+    auto decay = [&](int t, float (&a)[R]) {
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            a[i] = expf(gate_value(to_f32(g[tok_v(t) * K + rg + RPP * i]), bias[i], rate, gate_mode, lower_bound));
+    };
     auto load4 = [&](const Elt* p) {  // 4 consecutive elements as float4
         return make_float4(to_f32(p[0]), to_f32(p[1]), to_f32(p[2]), to_f32(p[3]));
     };
@@ -118,45 +123,27 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
         red ^= 1;
         return s;
     };
-    // One token's inputs for this thread's rows and columns: decay factors, k (and q, dO in the reverse
-    // sweep), v, beta.  Loaded a token ahead of their use, so that each step's global loads and
-    // exponentials overlap the previous step.
-    struct TokIn {
-        float a[R], kd[R], qd[R];
-        float4 vv, dOc;
-        float bt;
-    };
-    auto load_tok = [&](int t, bool reverse) {
-        TokIn in;
-        const size_t rq = tok_qk(t) * K, rv = tok_v(t);
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int d = rg + RPP * i;
-            in.a[i] = expf(gate_value(to_f32(g[rv * K + d]), bias[i], rate, gate_mode, lower_bound));
-            in.kd[i] = to_f32(k[rq + d]);
-            in.qd[i] = reverse ? to_f32(q[rq + d]) : 0.f;
-        }
-        in.vv = load4(v + rv * V + c0 + 4 * cg);
-        in.dOc = reverse ? load4(dO + rv * V + c0 + 4 * cg) : make_float4(0.f, 0.f, 0.f, 0.f);
-        in.bt = to_f32(beta[rv]);
-        return in;
-    };
 
     // one forward step on this thread's state rows: decay, residual (returned), rank-1 write
     float4 S[R];
-    auto forward_step = [&](const TokIn& in) {
+    auto forward_step = [&](int t) {
+        float a[R];
+        decay(t, a);
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+        float kd[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            S[i] = make_float4(in.a[i] * S[i].x, in.a[i] * S[i].y, in.a[i] * S[i].z, in.a[i] * S[i].w);
-            p = make_float4(p.x + in.kd[i] * S[i].x, p.y + in.kd[i] * S[i].y, p.z + in.kd[i] * S[i].z,
-                            p.w + in.kd[i] * S[i].w);
+            kd[i] = to_f32(k[tok_qk(t) * K + rg + RPP * i]);
+            S[i] = make_float4(a[i] * S[i].x, a[i] * S[i].y, a[i] * S[i].z, a[i] * S[i].w);
+            p = make_float4(p.x + kd[i] * S[i].x, p.y + kd[i] * S[i].y, p.z + kd[i] * S[i].z, p.w + kd[i] * S[i].w);
         }
         p = reduce(p);
-        const float4 r = make_float4(in.vv.x - p.x, in.vv.y - p.y, in.vv.z - p.z, in.vv.w - p.w);
+        const float4 vv = load4(v + tok_v(t) * V + c0 + 4 * cg);
+        const float4 r = make_float4(vv.x - p.x, vv.y - p.y, vv.z - p.z, vv.w - p.w);
+        const float bt = to_f32(beta[tok_v(t)]);
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const float w = in.bt * in.kd[i];
+            const float w = bt * kd[i];
             S[i] = make_float4(S[i].x + w * r.x, S[i].y + w * r.y, S[i].z + w * r.z, S[i].w + w * r.w);
         }
         return r;
@@ -167,19 +154,13 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     for (int i = 0; i < R; ++i)
         S[i] = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * K + rg + RPP * i) * V + c0 + 4 * cg)
                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-        TokIn cur = load_tok(0, false);
-        for (int t = 0; t < T; ++t) {
-            TokIn nxt = cur;
-            if (t + 1 < T) nxt = load_tok(t + 1, false);
-            if (t % BWD_CK == 0) {
+    for (int t = 0; t < T; ++t) {
+        if (t % BWD_CK == 0) {
 #pragma unroll
-                for (int i = 0; i < R; ++i)
-                    *reinterpret_cast<float4*>(my_ckpt + ((size_t)(t / BWD_CK) * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-            }
-            forward_step(cur);
-            cur = nxt;
+            for (int i = 0; i < R; ++i)
+                *reinterpret_cast<float4*>(my_ckpt + ((size_t)(t / BWD_CK) * K + rg + RPP * i) * VB + 4 * cg) = S[i];
         }
+        forward_step(t);
     }
 
     // ---- 2. blocks in reverse ----------------------------------------------------------------------
@@ -195,45 +176,42 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
 #pragma unroll
         for (int i = 0; i < R; ++i)
             S[i] = *reinterpret_cast<const float4*>(my_ckpt + ((size_t)blk * K + rg + RPP * i) * VB + 4 * cg);
-        {
-            TokIn cur = load_tok(t0, false);
-            for (int j = 0; j < n; ++j) {
-                TokIn nxt = cur;
-                if (j + 1 < n) nxt = load_tok(t0 + j + 1, false);
+        for (int j = 0; j < n; ++j) {
 #pragma unroll
-                for (int i = 0; i < R; ++i)
-                    *reinterpret_cast<float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-                const float4 r = forward_step(cur);
-                *reinterpret_cast<float4*>(sR + j * VB + 4 * cg) = r;  // same values from every row group
-                cur = nxt;
-            }
+            for (int i = 0; i < R; ++i)
+                *reinterpret_cast<float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg) = S[i];
+            const float4 r = forward_step(t0 + j);
+            *reinterpret_cast<float4*>(sR + j * VB + 4 * cg) = r;  // same values from every row group
         }
         // reverse through the block; S holds the state after token t
-        TokIn cur = load_tok(t0 + n - 1, true);
         for (int j = n - 1; j >= 0; --j) {
             const int t = t0 + j;
             const size_t rq = tok_qk(t) * K, rv = tok_v(t);
-            TokIn nxt = cur;
-            if (j > 0) nxt = load_tok(t - 1, true);
-            const float4 dOc = cur.dOc;
+            const float4 dOc = load4(dO + rv * V + c0 + 4 * cg);
+            float qd[R], kd[R], a[R];
+            decay(t, a);
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                qd[i] = to_f32(q[rq + rg + RPP * i]);
+                kd[i] = to_f32(k[rq + rg + RPP * i]);
+            }
             // dq_t = s S_t dO_t ; dS += s q_t dO_t^T
 #pragma unroll
             for (int i = 0; i < R; ++i) {
                 const float part =
                     sum_over_cols<TPR>(make_float4(S[i].x * dOc.x, S[i].y * dOc.y, S[i].z * dOc.z, S[i].w * dOc.w));
                 if (cg == 0) atomicAdd(dq + rq + rg + RPP * i, scale * part);
-                const float w = scale * cur.qd[i];
+                const float w = scale * qd[i];
                 dS[i] = make_float4(dS[i].x + w * dOc.x, dS[i].y + w * dOc.y, dS[i].z + w * dOc.z, dS[i].w + w * dOc.w);
             }
             // u = dS^T k_t over the key rows
             float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < R; ++i)
-                u = make_float4(u.x + cur.kd[i] * dS[i].x, u.y + cur.kd[i] * dS[i].y, u.z + cur.kd[i] * dS[i].z,
-                                u.w + cur.kd[i] * dS[i].w);
+                u = make_float4(u.x + kd[i] * dS[i].x, u.y + kd[i] * dS[i].y, u.z + kd[i] * dS[i].z, u.w + kd[i] * dS[i].w);
             u = reduce(u);
             const float4 r = *reinterpret_cast<const float4*>(sR + j * VB + 4 * cg);
-            const float bt = cur.bt;
+            const float bt = to_f32(beta[rv]);
             const float4 dr = make_float4(bt * u.x, bt * u.y, bt * u.z, bt * u.w);
             if (rg == 0) {  // dbeta_t = u . r over this CTA's columns; dv_t = dr
                 float db = dot4(u, r);
@@ -244,22 +222,20 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
             }
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float ai = cur.a[i], kdi = cur.kd[i];
                 const float4 Sp = *reinterpret_cast<const float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg);
-                const float4 Sd = make_float4(ai * Sp.x, ai * Sp.y, ai * Sp.z, ai * Sp.w);
+                const float4 Sd = make_float4(a[i] * Sp.x, a[i] * Sp.y, a[i] * Sp.z, a[i] * Sp.w);
                 // dk_t = beta dS r - S_dec dr
                 const float pk = sum_over_cols<TPR>(make_float4(bt * dS[i].x * r.x - Sd.x * dr.x, bt * dS[i].y * r.y - Sd.y * dr.y,
                                                                 bt * dS[i].z * r.z - Sd.z * dr.z, bt * dS[i].w * r.w - Sd.w * dr.w));
                 if (cg == 0) atomicAdd(dk + rq + rg + RPP * i, pk);
                 // dS_dec = dS - k dr^T ; dg_t = a rowsum(dS_dec S_{t-1}) ; dS_{t-1} = a dS_dec
-                const float4 dSd = make_float4(dS[i].x - kdi * dr.x, dS[i].y - kdi * dr.y, dS[i].z - kdi * dr.z,
-                                               dS[i].w - kdi * dr.w);
+                const float4 dSd = make_float4(dS[i].x - kd[i] * dr.x, dS[i].y - kd[i] * dr.y, dS[i].z - kd[i] * dr.z,
+                                               dS[i].w - kd[i] * dr.w);
                 const float pg = sum_over_cols<TPR>(make_float4(dSd.x * Sp.x, dSd.y * Sp.y, dSd.z * Sp.z, dSd.w * Sp.w));
-                if (cg == 0) atomicAdd(dg + rv * K + rg + RPP * i, ai * pg);
-                dS[i] = make_float4(ai * dSd.x, ai * dSd.y, ai * dSd.z, ai * dSd.w);
+                if (cg == 0) atomicAdd(dg + rv * K + rg + RPP * i, a[i] * pg);
+                dS[i] = make_float4(a[i] * dSd.x, a[i] * dSd.y, a[i] * dSd.z, a[i] * dSd.w);
                 S[i] = Sp;
             }
-            cur = nxt;
         }
     }
     if (dS0) {

@@ -693,14 +693,6 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         if (tid == 0) {
             pending &= ~(2u << buf);
             if (c + 1 < c_end) load_wq(c + 1);  // M8 has read WQ
-            // the record parts two chunks ahead into L2, so that their copies into shared memory do not wait
-            // for HBM (the record of the next chunk is already on its way)
-            if (c + 2 < c_end) {
-                bulk_prefetch_l2(rec(c + 2) + Rec::WQ, 65536);
-                bulk_prefetch_l2(rec(c + 2) + Rec::KA, KA_LOAD);
-                if (use_u) bulk_prefetch_l2(rec(c + 2) + Rec::UT + vb0 * 256, VB * 256);
-                bulk_prefetch_l2(rec(c + 2) + Rec::VEC, 512);
-            }
         }
         // ---- E = U - Wtil S (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
         const uint32_t ka = s_base + Lay::ka(buf);

@@ -35,8 +35,9 @@ struct MlaSmem {
     static constexpr size_t QA = 0;                                      // hi, lo: [48][PITCH] bf16 each
     static constexpr size_t CT = QA + 2 * (size_t)MLA_GH * PITCH * 2;    // latent tiles: 2 x [32][PITCH] bf16
     static constexpr size_t PB = CT + 2 * (size_t)MLA_TP * PITCH * 2;    // probabilities: 2 x [48][PP] bf16
-    static constexpr size_t SP = PB + 2 * (size_t)MLA_GH * PP * 2;       // score partials: [4][48][32] fp32
-    static constexpr size_t ST = SP + 4 * (size_t)MLA_GH * MLA_TP * 4;   // row statistics (floats)
+    static constexpr int SPP = MLA_TP + 8;                                // score partial row pitch (floats)
+    static constexpr size_t SP = PB + 2 * (size_t)MLA_GH * PP * 2;       // score partials: [4][48][SPP] fp32
+    static constexpr size_t ST = SP + 4 * (size_t)MLA_GH * SPP * 4;      // row statistics (floats)
     // ST: max partials 2 x [4][48], sum partials 2 x [4][48], running max 2 x [48], running sum [48]
     static constexpr size_t BYTES = ST + (2 * 4 * MLA_GH + 2 * 4 * MLA_GH + 2 * MLA_GH + MLA_GH) * 4;
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -79,7 +80,7 @@ template <int DQ, int R>
 __global__ void __launch_bounds__(128)
 mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B, int H, bf16* __restrict__ qa_hi,
                 bf16* __restrict__ qa_lo) {
-    __shared__ float sq[16][DQ];
+    __shared__ __align__(16) float sq[16][DQ];
     const int h = blockIdx.x, col = blockIdx.y * 128 + threadIdx.x, b0 = blockIdx.z * 16;
     for (int i = threadIdx.x; i < 16 * DQ; i += 128) {
         const int bb = i / DQ, d = i - bb * DQ;
@@ -90,11 +91,15 @@ mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B
 #pragma unroll
     for (int bb = 0; bb < 16; ++bb) acc[bb] = 0.f;
     const bf16* w = W_UK + (size_t)h * DQ * R + col;
-#pragma unroll 4
-    for (int d = 0; d < DQ; ++d) {
-        const float wv = __bfloat162float(w[(size_t)d * R]);
+#pragma unroll 2
+    for (int d = 0; d < DQ; d += 4) {
+        const float w0 = __bfloat162float(w[(size_t)d * R]), w1 = __bfloat162float(w[(size_t)(d + 1) * R]);
+        const float w2 = __bfloat162float(w[(size_t)(d + 2) * R]), w3 = __bfloat162float(w[(size_t)(d + 3) * R]);
 #pragma unroll
-        for (int bb = 0; bb < 16; ++bb) acc[bb] = fmaf(sq[bb][d], wv, acc[bb]);
+        for (int bb = 0; bb < 16; ++bb) {
+            const float4 qv = *reinterpret_cast<const float4*>(&sq[bb][d]);
+            acc[bb] = fmaf(qv.x, w0, fmaf(qv.y, w1, fmaf(qv.z, w2, fmaf(qv.w, w3, acc[bb]))));
+        }
     }
 #pragma unroll
     for (int bb = 0; bb < 16; ++bb) {
@@ -119,7 +124,7 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
                   const int* __restrict__ lengths, int T, int H, int nsplit, int split_len, float scale_log2,
                   float* __restrict__ part_o, float* __restrict__ part_ml) {
     using Sm = MlaSmem<R>;
-    constexpr int P = Sm::PITCH, PP = Sm::PP;
+    constexpr int P = Sm::PITCH, PP = Sm::PP, SPP = Sm::SPP;
     constexpr int NC = R / 4;       // latent columns per warp in the weighted sum
     constexpr int NT8 = NC / 8;     // n8 tiles per warp
     extern __shared__ __align__(16) unsigned char msm[];
@@ -127,7 +132,7 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
     bf16* sQl = sQh + MLA_GH * P;
     bf16* sC = reinterpret_cast<bf16*>(msm + Sm::CT);
     bf16* sP = reinterpret_cast<bf16*>(msm + Sm::PB);
-    float* sSP = reinterpret_cast<float*>(msm + Sm::SP);    // [4][48][32] partial scores
+    float* sSP = reinterpret_cast<float*>(msm + Sm::SP);    // [4][48][SPP] partial scores
     float* sMaxP = reinterpret_cast<float*>(msm + Sm::ST);  // 2 x [4][48]
     float* sSumP = sMaxP + 2 * 4 * MLA_GH;                   // 2 x [4][48]
     float* sM = sSumP + 2 * 4 * MLA_GH;                      // 2 x [48]
@@ -220,11 +225,11 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
                     }
                 }
             }
-            float* dst = sSP + (size_t)quarter * MLA_GH * MLA_TP;
+            float* dst = sSP + (size_t)quarter * MLA_GH * SPP;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                *reinterpret_cast<float2*>(dst + (16 * m + g) * MLA_TP + 8 * j + 2 * t4) = make_float2(sp[j][0], sp[j][1]);
-                *reinterpret_cast<float2*>(dst + (16 * m + g + 8) * MLA_TP + 8 * j + 2 * t4) = make_float2(sp[j][2], sp[j][3]);
+                *reinterpret_cast<float2*>(dst + (16 * m + g) * SPP + 8 * j + 2 * t4) = make_float2(sp[j][0], sp[j][1]);
+                *reinterpret_cast<float2*>(dst + (16 * m + g + 8) * SPP + 8 * j + 2 * t4) = make_float2(sp[j][2], sp[j][3]);
             }
         }
         __syncthreads();
@@ -232,9 +237,9 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
         float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
-            const float* src = sSP + (size_t)kq * MLA_GH * MLA_TP;
-            const float2 x0 = *reinterpret_cast<const float2*>(src + (16 * m + g) * MLA_TP + 8 * quarter + 2 * t4);
-            const float2 x1 = *reinterpret_cast<const float2*>(src + (16 * m + g + 8) * MLA_TP + 8 * quarter + 2 * t4);
+            const float* src = sSP + (size_t)kq * MLA_GH * SPP;
+            const float2 x0 = *reinterpret_cast<const float2*>(src + (16 * m + g) * SPP + 8 * quarter + 2 * t4);
+            const float2 x1 = *reinterpret_cast<const float2*>(src + (16 * m + g + 8) * SPP + 8 * quarter + 2 * t4);
             s[0] += x0.x;
             s[1] += x0.y;
             s[2] += x1.x;
@@ -337,14 +342,17 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
 }
 
 // ---- merge the splits and step 4: o = (o_lat / l) W_UV^T ---------------------------------------
-// Grid (H, ceil(B / 8)); 256 threads.  The merged o_lat of 8 sequences goes to shared memory, then
-// thread v (of d_v) and batch row b accumulate over the latent columns, W_UV read in 32-column tiles.
+// Grid (H, ceil(B / 8)); 256 threads.  The merged o_lat of 8 sequences goes to shared memory; W_UV[h]
+// passes through shared memory in 32-column tiles.  Thread (v, part) accumulates the 8 sequences' outputs
+// for value column v over its part of each tile (float4 reads), and the parts are summed at the end.
 template <int DV, int R>
 __global__ void __launch_bounds__(256)
 mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, const bf16* __restrict__ W_UV,
                int B, int H, int nsplit, bf16* __restrict__ o) {
-    __shared__ float so[8][R];
-    __shared__ float sw[DV][33];
+    constexpr int PARTS = 256 / DV, KPT = 32 / PARTS;  // parts of each tile, columns per part
+    __shared__ __align__(16) float so[8][R];
+    __shared__ __align__(16) float sw[DV][36];           // pitch 36: conflict-free float4 reads by column v
+    __shared__ float sred[PARTS > 1 ? PARTS - 1 : 1][DV][8];
     const int h = blockIdx.x, b0 = blockIdx.y * 8, tid = threadIdx.x;
     // merge: o_lat = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s
     for (int i = tid; i < 8 * R; i += 256) {
@@ -365,12 +373,10 @@ mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_
         }
         so[bb][col] = val;
     }
-    // thread (v = tid % DV, batch rows bb = tid / DV + k * (256 / DV))
-    constexpr int BPT = 8 / (256 / DV);  // batch rows per thread
-    const int v = tid % DV, bq = tid / DV;
-    float acc[BPT];
+    const int v = tid % DV, part = tid / DV;
+    float acc[8];
 #pragma unroll
-    for (int i = 0; i < BPT; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     const bf16* w = W_UV + (size_t)h * DV * R;
     for (int k0 = 0; k0 < R; k0 += 32) {
         __syncthreads();  // previous W tile consumed (and o_lat merged, on the first pass)
@@ -379,17 +385,35 @@ mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_
             sw[vv][kk] = __bfloat162float(w[(size_t)vv * R + k0 + kk]);
         }
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            const float wv = sw[v][kk];
 #pragma unroll
-            for (int i = 0; i < BPT; ++i) acc[i] = fmaf(so[bq + i * (256 / DV)][k0 + kk], wv, acc[i]);
+        for (int kk = part * KPT; kk < part * KPT + KPT; kk += 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(&sw[v][kk]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = *reinterpret_cast<const float4*>(&so[i][k0 + kk]);
+                acc[i] = fmaf(x.x, wv.x, fmaf(x.y, wv.y, fmaf(x.z, wv.z, fmaf(x.w, wv.w, acc[i]))));
+            }
         }
     }
+    if (PARTS > 1) {
+        if (part > 0) {
 #pragma unroll
-    for (int i = 0; i < BPT; ++i) {
-        const int b = b0 + bq + i * (256 / DV);
-        if (b < B) o[((size_t)b * H + h) * DV + v] = __float2bfloat16_rn(acc[i]);
+            for (int i = 0; i < 8; ++i) sred[part - 1][v][i] = acc[i];
+        }
+        __syncthreads();
+        if (part == 0) {
+            for (int p2 = 0; p2 + 1 < PARTS; ++p2) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += sred[p2][v][i];
+            }
+        }
+    }
+    if (part == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int b = b0 + i;
+            if (b < B) o[((size_t)b * H + h) * DV + v] = __float2bfloat16_rn(acc[i]);
+        }
     }
 }
 

@@ -186,11 +186,6 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Bulk prefetch of global memory into L2 (no shared memory, no completion to wait for); the address is
-// 16-byte aligned and the size a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 // Wait until the committed bulk stores of this thread have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until the committed bulk stores of this thread are complete.
