@@ -12,7 +12,7 @@
 // dq and dk of a q/k head add up over the value heads that read it (GVA), and every row quantity adds
 // up over the value columns.
 //
-// Layout: one CTA per (b, hv, block of VB = min(V, 16) value columns); value columns are independent in
+// Layout: one CTA per (b, hv, block of VB = min(V, 8) value columns); value columns are independent in
 // the forward pass, so each CTA runs the recurrence on its columns alone.  Thread (row group rg, column
 // group cg) holds rows rg + RPP i (i < R) and columns 4 cg .. 4 cg + 3 of the state and of dS in
 // registers.  Reductions over key rows (the residual's prediction and u) go through warp shuffles and a
@@ -33,7 +33,7 @@ constexpr int BWD_CK = 8;  // tokens between saved states
 
 template <int K, int V>
 struct BwdShape {
-    static constexpr int VB = V < 16 ? V : 16;                         // value columns per CTA
+    static constexpr int VB = V < 8 ? V : 8;                           // value columns per CTA
     static constexpr int NT = (K * VB / 4 < 128) ? K * VB / 4 : 128;   // threads
     static constexpr int TPR = VB / 4;                                 // threads per state row
     static constexpr int RPP = NT / TPR;                               // row groups

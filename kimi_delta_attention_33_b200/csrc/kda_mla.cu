@@ -75,34 +75,37 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
 }  // namespace
 
 // ---- step 1: q_abs = q W_UK per head, as bf16 hi + lo ------------------------------------------
-// Grid (H, R / 128, ceil(B / 16)); thread = one latent column, 16 sequences per CTA.
+// Grid (H, R / 128, ceil(B / 32)); thread = one latent column, 32 sequences per CTA, so W_UK is read
+// ceil(B / 32) times; four key channels per step with the sequences' q values as float4.
+constexpr int QABS_B = 32;
+
 template <int DQ, int R>
 __global__ void __launch_bounds__(128)
 mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B, int H, bf16* __restrict__ qa_hi,
                 bf16* __restrict__ qa_lo) {
-    __shared__ __align__(16) float sq[16][DQ];
-    const int h = blockIdx.x, col = blockIdx.y * 128 + threadIdx.x, b0 = blockIdx.z * 16;
-    for (int i = threadIdx.x; i < 16 * DQ; i += 128) {
+    __shared__ __align__(16) float sq[QABS_B][DQ];
+    const int h = blockIdx.x, col = blockIdx.y * 128 + threadIdx.x, b0 = blockIdx.z * QABS_B;
+    for (int i = threadIdx.x; i < QABS_B * DQ; i += 128) {
         const int bb = i / DQ, d = i - bb * DQ;
         sq[bb][d] = (b0 + bb < B) ? __bfloat162float(q[((size_t)(b0 + bb) * H + h) * DQ + d]) : 0.f;
     }
     __syncthreads();
-    float acc[16];
+    float acc[QABS_B];
 #pragma unroll
-    for (int bb = 0; bb < 16; ++bb) acc[bb] = 0.f;
+    for (int bb = 0; bb < QABS_B; ++bb) acc[bb] = 0.f;
     const bf16* w = W_UK + (size_t)h * DQ * R + col;
-#pragma unroll 2
+#pragma unroll 1
     for (int d = 0; d < DQ; d += 4) {
         const float w0 = __bfloat162float(w[(size_t)d * R]), w1 = __bfloat162float(w[(size_t)(d + 1) * R]);
         const float w2 = __bfloat162float(w[(size_t)(d + 2) * R]), w3 = __bfloat162float(w[(size_t)(d + 3) * R]);
 #pragma unroll
-        for (int bb = 0; bb < 16; ++bb) {
+        for (int bb = 0; bb < QABS_B; ++bb) {
             const float4 qv = *reinterpret_cast<const float4*>(&sq[bb][d]);
             acc[bb] = fmaf(qv.x, w0, fmaf(qv.y, w1, fmaf(qv.z, w2, fmaf(qv.w, w3, acc[bb]))));
         }
     }
 #pragma unroll
-    for (int bb = 0; bb < 16; ++bb) {
+    for (int bb = 0; bb < QABS_B; ++bb) {
         if (b0 + bb >= B) break;
         const bf16 hi = __float2bfloat16_rn(acc[bb]);
         const size_t idx = ((size_t)(b0 + bb) * H + h) * R + col;
@@ -342,20 +345,34 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
 }
 
 // ---- merge the splits and step 4: o = (o_lat / l) W_UV^T ---------------------------------------
-// Grid (H, ceil(B / 8)); 256 threads.  The merged o_lat of 8 sequences goes to shared memory; W_UV[h]
-// passes through shared memory in 32-column tiles.  Thread (v, part) accumulates the 8 sequences' outputs
-// for value column v over its part of each tile (float4 reads), and the parts are summed at the end.
+// Grid (H, ceil(B / 32)); 256 threads.  The merged o_lat of 32 sequences goes to shared memory (dynamic);
+// W_UV[h] passes through shared memory in 32-column tiles loaded 16 bytes at a time, so it is read
+// ceil(B / 32) times.  Thread (v, part) accumulates the 32 sequences' outputs for value column v over its
+// part of each tile (float4 reads), and the parts are summed at the end.
+constexpr int OUT_B = 32;
+
+template <int DV, int R>
+struct MlaOutSmem {
+    static constexpr int PARTS = 256 / DV;
+    static constexpr size_t SO = 0;                                    // [32][R] fp32 merged o_lat
+    static constexpr size_t SW = SO + (size_t)OUT_B * R * 4;           // [DV][36] fp32 W tile
+    static constexpr size_t SR = SW + (size_t)DV * 36 * 4;             // [PARTS - 1][DV][32] partial sums
+    static constexpr size_t BYTES = SR + (size_t)(PARTS > 1 ? PARTS - 1 : 1) * DV * OUT_B * 4;
+};
+
 template <int DV, int R>
 __global__ void __launch_bounds__(256)
 mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, const bf16* __restrict__ W_UV,
                int B, int H, int nsplit, bf16* __restrict__ o) {
-    constexpr int PARTS = 256 / DV, KPT = 32 / PARTS;  // parts of each tile, columns per part
-    __shared__ __align__(16) float so[8][R];
-    __shared__ __align__(16) float sw[DV][36];           // pitch 36: conflict-free float4 reads by column v
-    __shared__ float sred[PARTS > 1 ? PARTS - 1 : 1][DV][8];
-    const int h = blockIdx.x, b0 = blockIdx.y * 8, tid = threadIdx.x;
+    using Sm = MlaOutSmem<DV, R>;
+    constexpr int PARTS = Sm::PARTS, KPT = 32 / PARTS;  // parts of each tile, columns per part
+    extern __shared__ __align__(16) unsigned char osm[];
+    float (*so)[R] = reinterpret_cast<float (*)[R]>(osm + Sm::SO);
+    float (*sw)[36] = reinterpret_cast<float (*)[36]>(osm + Sm::SW);  // pitch 36: conflict-free float4 reads
+    float* sred = reinterpret_cast<float*>(osm + Sm::SR);
+    const int h = blockIdx.x, b0 = blockIdx.y * OUT_B, tid = threadIdx.x;
     // merge: o_lat = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s
-    for (int i = tid; i < 8 * R; i += 256) {
+    for (int i = tid; i < OUT_B * R; i += 256) {
         const int bb = i / R, col = i - bb * R, b = b0 + bb;
         float val = 0.f;
         if (b < B) {
@@ -374,22 +391,27 @@ mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_
         so[bb][col] = val;
     }
     const int v = tid % DV, part = tid / DV;
-    float acc[8];
+    float acc[OUT_B];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < OUT_B; ++i) acc[i] = 0.f;
     const bf16* w = W_UV + (size_t)h * DV * R;
     for (int k0 = 0; k0 < R; k0 += 32) {
         __syncthreads();  // previous W tile consumed (and o_lat merged, on the first pass)
-        for (int i = tid; i < DV * 32; i += 256) {
-            const int vv = i / 32, kk = i - vv * 32;
-            sw[vv][kk] = __bfloat162float(w[(size_t)vv * R + k0 + kk]);
+        for (int i = tid; i < DV * 4; i += 256) {  // DV rows x 4 chunks of 8 bf16
+            const int vv = i >> 2, ch = i & 3;
+            const uint4 raw = *reinterpret_cast<const uint4*>(w + (size_t)vv * R + k0 + 8 * ch);
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+            const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+            *reinterpret_cast<float4*>(&sw[vv][8 * ch]) = make_float4(f0.x, f0.y, f1.x, f1.y);
+            *reinterpret_cast<float4*>(&sw[vv][8 * ch + 4]) = make_float4(f2.x, f2.y, f3.x, f3.y);
         }
         __syncthreads();
 #pragma unroll
         for (int kk = part * KPT; kk < part * KPT + KPT; kk += 4) {
             const float4 wv = *reinterpret_cast<const float4*>(&sw[v][kk]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < OUT_B; ++i) {
                 const float4 x = *reinterpret_cast<const float4*>(&so[i][k0 + kk]);
                 acc[i] = fmaf(x.x, wv.x, fmaf(x.y, wv.y, fmaf(x.z, wv.z, fmaf(x.w, wv.w, acc[i]))));
             }
@@ -398,19 +420,19 @@ mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_
     if (PARTS > 1) {
         if (part > 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sred[part - 1][v][i] = acc[i];
+            for (int i = 0; i < OUT_B; ++i) sred[((part - 1) * DV + v) * OUT_B + i] = acc[i];
         }
         __syncthreads();
         if (part == 0) {
             for (int p2 = 0; p2 + 1 < PARTS; ++p2) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] += sred[p2][v][i];
+                for (int i = 0; i < OUT_B; ++i) acc[i] += sred[(p2 * DV + v) * OUT_B + i];
             }
         }
     }
     if (part == 0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < OUT_B; ++i) {
             const int b = b0 + i;
             if (b < B) o[((size_t)b * H + h) * DV + v] = __float2bfloat16_rn(acc[i]);
         }
@@ -445,7 +467,7 @@ cudaError_t launch_mla_t(const MlaArgs& a) {
     float* part_o = reinterpret_cast<float*>(qa_lo + (size_t)a.B * a.H * R);
     float* part_ml = part_o + (size_t)a.B * ns * a.H * R;
     const bf16* q = static_cast<const bf16*>(a.q);
-    mla_qabs_kernel<DQ, R><<<dim3(a.H, R / 128, (a.B + 15) / 16), 128, 0, a.stream>>>(
+    mla_qabs_kernel<DQ, R><<<dim3(a.H, R / 128, (a.B + QABS_B - 1) / QABS_B), 128, 0, a.stream>>>(
         q, static_cast<const bf16*>(a.W_UK), a.B, a.H, qa_hi, qa_lo);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -456,9 +478,11 @@ cudaError_t launch_mla_t(const MlaArgs& a) {
     mla_attend_kernel<R><<<dim3(a.B, (a.H + MLA_GH - 1) / MLA_GH, ns), MLA_THREADS, Sm::BYTES, a.stream>>>(
         qa_hi, qa_lo, static_cast<const bf16*>(a.c), a.lengths, a.T, a.H, ns, split_len, scale_log2, part_o, part_ml);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    mla_out_kernel<DV, R><<<dim3(a.H, (a.B + 7) / 8), 256, 0, a.stream>>>(part_o, part_ml,
-                                                                          static_cast<const bf16*>(a.W_UV), a.B, a.H,
-                                                                          ns, static_cast<bf16*>(a.o));
+    using OSm = MlaOutSmem<DV, R>;
+    e = cudaFuncSetAttribute(mla_out_kernel<DV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OSm::BYTES);
+    if (e != cudaSuccess) return e;
+    mla_out_kernel<DV, R><<<dim3(a.H, (a.B + OUT_B - 1) / OUT_B), 256, OSm::BYTES, a.stream>>>(
+        part_o, part_ml, static_cast<const bf16*>(a.W_UV), a.B, a.H, ns, static_cast<bf16*>(a.o));
     return cudaGetLastError();
 }
 
