@@ -17,19 +17,28 @@
 //
 // Pass 1 (chunk_prep_kernel, persistent, one chunk per CTA iteration, all chunks in parallel):
 // gate, Gam, the operands, M1 = [-Khat; Qhat] Kchk^T -> R and A, the triangular inverse, and
-// M7 = [Tb; Tb] [Khat^T; V^T]^T -> W and U, written to a per-chunk record in the workspace:
-//   WQ  [Wtil; Qtil]  128 x 128 tf32 in the K-major tiling of kda_tc_ptx.cuh (the A operand of M8)
-//   KA  [Kend; A]     192 x 64 tf32, same tiling (A operands of M9 and M10)
-//   UT  U^T, fp32 rows of 64 (one per value column)
-//   VEC e^{Gam_end} (fp32, 128)
+// M7 = [Tb; A] [Khat^T; V^T]^T -> W and U (rows 0-63), and the products that fold the delta errors
+// into the record:
+//   S_c+1 = e^{Gam_end} S_c + Kend (U - Wtil S_c) = e^{Gam_end} S_c - G S_c + KU,  G = Kend Wtil, KU = Kend U
+//   O      = Qtil S_c + A (U - Wtil S_c)          = Q' S_c + A U,               Q' = Qtil - A Wtil
+// M11 = Kend [Wtil^T; U^T]^T -> [G | KU] and M12 = [Tb; A] [Wtil^T; U^T]^T -> [A Wtil | A U] (rows 64-127),
+// written to a per-chunk record in the workspace:
+//   WQ  [G; Q']   192 x 128 fp16 in the K-major tiling of kda_tc_ptx.cuh (A operands of the state pass)
+//   KU  128 x 128 fp16, AU 64 x 128 fp32, both by blocks of 16 value columns
+//   VEC e^{Gam_end} (fp32, 128), then the scale block
+// Every fp16 tile (G, Q', KU) is stored as tile * 2^-e with one power-of-two exponent e per tile, chosen
+// from the tile's largest magnitude so that the scaled tile uses fp16's range (kda_tc_ptx.cuh,
+// fp16_scale_exponent); the exponents sit in the scale block.  fp16 carries the same 10 fraction bits as
+// tf32, and the powers of two come off exactly on the fp32 accumulators.  The decay e^{Gam_end} S stays
+// an exact fp32 product: only the low-rank corrections G S and KU are rounded.
 // Pass 2 (chunk_state_kernel, one CTA per (pair, block of VB value columns), chunks in order):
 // the state slice S_c[:, block] lives in registers (thread d owns key row d, exact fp32);
-// per chunk, with tf32(S_c)^T staged in shared memory as a B operand:
-//   M8   D1 = [Wtil; Qtil] S_c           -> Wtil S_c (rows 0-63), Qtil S_c (rows 64-127)
-//   E    = U - Wtil S_c  on the CUDA cores, staged as a tf32 B operand
-//   M10  D2 = Kend E                      -> S_c+1 = e^{Gam_end} S_c + D2, in registers
-//   M9   D1[64:] += A E                   -> O  (issued after M10 with its own commit: off the
-//                                             chunk-to-chunk path)
+// per chunk, with fp16(S_c 2^-sig)^T staged in shared memory as a B operand:
+//   chain  D_S = G S_c                     -> S_c+1 = e^{Gam_end} S_c - D_S + KU, in registers
+//   out    D_O = [G rows 64-127; Q'] S_c   -> O = Q' S_c + A U (rows 64-127), read out while the next
+//                                             chunk's chain product runs
+// One tensor-core round trip per chunk is on the chunk-to-chunk path.  The state scale is not reduced over
+// the CTA on the chain: it comes from a bound that all threads compute alike (see chunk_state_kernel).
 // Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
 // where shared memory allows.
 #include <cuda.h>
@@ -44,16 +53,22 @@ using bf16 = __nv_bfloat16;
 namespace {
 using namespace c64;
 
-// Per-chunk record in the workspace (bytes).
+// Per-chunk record in the workspace (bytes).  Value-column blocks of 16 (KU, AU) let a state CTA read
+// its columns with one contiguous copy per block.
 struct Rec {
-    static constexpr uint32_t WQ = 0;        // [128][128] tf32 tiles
-    static constexpr uint32_t KA = 65536;    // [192][64] tf32 tiles
-    static constexpr uint32_t KA_BYTES = 49152;
-    static constexpr uint32_t UT = 114688;   // [128][64] fp32 rows
-    static constexpr uint32_t VEC = 147456;  // [128] fp32 e^{Gam_end}, then padding
-    static constexpr uint32_t BYTES = 149504;
-    static_assert(VEC + 512 <= BYTES && BYTES % 256 == 0, "record layout");
+    static constexpr uint32_t WQ = 0;          // [192][128] fp16 tiles: G 2^-eg (rows 0-127), Q' 2^-eq (rows 128-191)
+    static constexpr uint32_t WQ_BYTES = 49152;
+    static constexpr uint32_t QP_OFF = 32768;  // row 128 of WQ
+    static constexpr uint32_t KU = 49152;      // fp16 [8][128][16]: KU 2^-eu by blocks of 16 value columns
+    static constexpr uint32_t AU = 81920;      // fp32 [8][64][16]: A U by blocks of 16 value columns
+    static constexpr uint32_t VEC = 114688;    // [128] fp32 e^{Gam_end}, then the scale block at SCL
+    static constexpr uint32_t SCL = VEC + 512; // int eg, eq, eu; float max e^{Gam_end}
+    static constexpr uint32_t VEC_LOAD = 528;  // bytes of VEC the state pass reads
+    static constexpr uint32_t BYTES = 115712;
+    static_assert(SCL + 16 <= VEC + VEC_LOAD && VEC + 1024 <= BYTES && BYTES % 256 == 0, "record layout");
 };
+// slots of the per-chunk maxima in the prep kernel (PrepLayout::MX)
+enum : int { MX_QT = 0, MX_K = 1, MX_A = 2, MX_W = 3, MX_U = 4, MX_EG = 5, MX_SLOTS = 8 };
 
 struct PrepLayout {
     static constexpr uint32_t X1 = 0;        // [128][128] [-Khat; Qhat] (A of M1); once M1 is done X1 stages
@@ -63,50 +78,66 @@ struct PrepLayout {
     static constexpr uint32_t CK = 65536;    // [64][128] Kchk (B of M1); then R / T (pitch RP) + doubling
                                              //   scratch; then U^T [128][64] fp32 (record UT)
     static constexpr uint32_t XS = CK + 64 * RP * 4;
-    static constexpr uint32_t KA = 98304;    // [256][64]: Kend^T rows 0-127 (record KA, first part),
-                                             //   Tb twice in rows 128-255 (A of M7)
+    static constexpr uint32_t KA = 98304;    // [256][64]: Kend^T rows 0-127 (A of M11), Tb in rows 128-191 and
+                                             //   the masked A in rows 192-255 (A of M7 and M12)
     static constexpr uint32_t GM = 163840;   // Gam (fp32 [64][128]) -> Khat^T [128][64] (B rows 0-127 of M7)
-    static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7)
+    static constexpr uint32_t VT = 196608;   // V^T [128][64] (B rows 128-255 of M7); after M7 GM and VT hold
+                                             //   BT = [Wtil^T; U^T] [256][64], the B operand of M11 and M12
     static constexpr uint32_t VEC = 229376;
     static constexpr uint32_t RHO = VEC, SIG = VEC + 512, BETA = VEC + 1024, ERHO = VEC + 1280, FEND = VEC + 1792;
     static constexpr uint32_t MBAR = VEC + 2304, MBAR_IN = MBAR + 8, TBASE = MBAR_IN + 8;
     static constexpr uint32_t SQQ = VEC + 2336, SQK = VEC + 2592;  // [64] row sums of squares of q, k
+    static constexpr uint32_t MX = VEC + 2848;  // [MX_SLOTS] per-chunk maxima of the record tiles (float bits)
     static constexpr uint32_t QT = KA + 32768;    // record Qtil staging, in the Tb rows (free until the inverse)
-    static constexpr uint32_t PART = KA + 32768;  // gate: per-channel quarter totals and Gam_0 (5 x [128] fp32),
-                                                  //   in the Tb rows, which are free until the inverse
+    static constexpr uint32_t PART = KA + 49152;  // gate: per-channel quarter totals and Gam_0 (5 x [128] fp32),
+                                                  //   in KA rows 192-255, free until M1 is read out and not
+                                                  //   part of the record staging below
+    // record staging at the end of a chunk (bulk stores, done reading before the next chunk's V^T step):
+    // [G; Q'] fp16 in KA rows 0-191, KU in CK, AU in VT
     static constexpr uint32_t STG_G = X1, STG_V = X1 + 16384, STG_Q = X1 + 32768, STG_K = X1 + 49152;
-    static constexpr uint32_t BYTES = SQK + 256;
-    static constexpr uint32_t TMEM_COLS = 256;  // D1 [128][64] for M1, then [128][256] for M7
+    static constexpr uint32_t BYTES = MX + 4 * MX_SLOTS;
+    static constexpr uint32_t TMEM_COLS = 512;  // D [128][64] for M1, [128][256] for M7, then [128][512] for M11, M12
     static_assert(XS + 1024 * 4 <= KA, "doubling scratch");
     static_assert(GM + 32768 == VT, "M7's B operand spans GM and VT");
-    static_assert(BYTES <= 232448, "shared memory budget");
-};
-
-template <int VB>
-struct StateLayout {
-    static constexpr int NKA = VB <= 32 ? 2 : 1;              // KA / U buffers
-    // With 128 value columns the E^T operand takes the place of the U^T rows it is computed from.
-    static constexpr bool ALIAS_E = VB > 64;
-    static constexpr uint32_t WQ = 0;                          // [128][128]
-    static constexpr uint32_t KA0 = 65536;                     // per buffer: KA [192][64], U^T [VB][64], e^{Gam_end}
-    static constexpr uint32_t UT_OFF = Rec::KA_BYTES, VEC_OFF = Rec::KA_BYTES + VB * 256;
-    static constexpr uint32_t KA_STRIDE = VEC_OFF + 512;
-    static constexpr uint32_t SOP = KA0 + NKA * KA_STRIDE;     // tf32 S^T [VB][128]    (B of M8)
-    static constexpr uint32_t EOP = ALIAS_E ? KA0 + UT_OFF : SOP + VB * 128 * 4;  // tf32 E^T [VB][64] (B of M9, M10)
-    static constexpr uint32_t MBAR = ALIAS_E ? SOP + VB * 128 * 4 : EOP + VB * 64 * 4;  // wq, mma, ka[0], ka[1], out
-    static constexpr uint32_t TBASE = MBAR + 40;
-    static constexpr uint32_t BYTES = TBASE + 16;
-    static constexpr uint32_t TMEM_COLS = 2 * VB < 32 ? 32 : 2 * VB;
-    static constexpr int D1 = 0, D2 = VB;
-    static __device__ __forceinline__ uint32_t ka(int buf) { return KA0 + buf * KA_STRIDE; }
-    static_assert(!ALIAS_E || VB * 64 * 4 <= VB * 256, "E^T fits in the U^T rows");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
 // What one state-pass CTA computes over its chunks (see chunk_state_kernel).
 enum : int { STATE_OUT = 0, STATE_CARRY = 1 };
 
-constexpr int STATE_THREADS = 256;
+// Shared memory of one state-pass CTA.  Record slots hold, per chunk, [G; Q'] (G only without outputs), this
+// block's columns of KU and AU, and VEC.  With outputs a slot stays in use until the step after its own (the
+// outputs are read out then), so three slots keep the copies two chunks ahead; without, two.
+template <int VB, int MODE>
+struct StateLayout {
+    static constexpr bool OUTS = MODE == STATE_OUT;
+    static constexpr int NBUF = OUTS ? 3 : 2;
+    static constexpr int NSOP = OUTS ? 2 : 1;                  // S operands: by chunk parity when the output
+                                                               // product of a chunk may still read its own
+    static constexpr uint32_t WQ_LOAD = OUTS ? Rec::WQ_BYTES : Rec::QP_OFF;
+    static constexpr uint32_t KU_OFF = WQ_LOAD, AU_OFF = KU_OFF + VB * 256;
+    static constexpr uint32_t VEC_OFF = AU_OFF + (OUTS ? VB * 256 : 0);
+    static constexpr uint32_t SLOT = VEC_OFF + 1024;
+    // fp16 S^T [VB][128] per buffer (B operand), in the padded tiling: K-adjacent core matrices 144 bytes
+    // apart (SOP_LBO), 8-row groups 16 x 144 bytes apart (SOP_SBO)
+    static constexpr uint32_t SOP_LBO = 144, SOP_SBO = 16 * SOP_LBO, SOP_BYTES = VB / 8 * SOP_SBO;
+    static constexpr uint32_t SOP = NBUF * SLOT;
+    static constexpr uint32_t MBAR = SOP + NSOP * SOP_BYTES;   // rec[NBUF], chain, out[2]
+    static constexpr uint32_t TBASE = MBAR + 8 * (NBUF + 3);
+    static constexpr uint32_t SMX = TBASE + 16;                // [2][8] per-warp max |S|, by chunk parity
+    static constexpr uint32_t BYTES = SMX + 64;
+    // D_S = G S (chain); D_O[2] = [G; Q'] S rows 64-127 hold Q' S, by chunk parity
+    static constexpr int D_S = 0, D_O = VB;
+    static constexpr uint32_t NCOL = OUTS ? 3 * VB : VB;
+    static constexpr uint32_t TMEM_COLS = NCOL <= 32 ? 32 : NCOL <= 64 ? 64 : NCOL <= 128 ? 128 : NCOL <= 256 ? 256 : 512;
+    static __device__ __forceinline__ uint32_t slot(int k) { return k * SLOT; }
+    static_assert(SLOT % 1024 == 0 && BYTES <= 232448, "shared memory budget");
+};
+
+
+constexpr int STATE_WARPS = 8;                         // warps that own the state slice
+constexpr int STATE_THREADS = 32 * (STATE_WARPS + 1);  // and one that issues the copies and the products
+constexpr int ISSUER = 32 * STATE_WARPS;
 constexpr int PREP_THREADS = 512;
 static_assert(PREP_THREADS == INV_THREADS, "the triangular inverse assumes 512 threads");
 
@@ -125,6 +156,16 @@ __device__ __forceinline__ Task make_task(int task, int T, int H, int HV, int NC
     t.nn = min(CH, T - t.c * CH);
     t.tk0 = (size_t)t.b * T + (size_t)t.c * CH;
     return t;
+}
+
+// Folds this thread's maximum magnitude into a shared slot (float bits; every lane of the warp calls).
+__device__ __forceinline__ void max_into_slot(float m, unsigned int* slot, int lane) {
+    m = warp_max_nonneg(m);
+    if (lane == 0) atomicMax(slot, __float_as_uint(m));
+}
+
+__device__ __forceinline__ float slot_value(const unsigned int* slot) {
+    return __uint_as_float(*reinterpret_cast<const volatile unsigned int*>(slot));
 }
 
 }  // namespace
@@ -152,6 +193,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     float* sFend = reinterpret_cast<float*>(smem + L::FEND);
     float* sSqQ = reinterpret_cast<float*>(smem + L::SQQ);
     float* sSqK = reinterpret_cast<float*>(smem + L::SQK);
+    unsigned int* sMx = reinterpret_cast<unsigned int*>(smem + L::MX);
     const bool norm_qk = (flags & KDA_INPUT_L2NORM_QK) != 0;
     float* sGam = reinterpret_cast<float*>(smem + L::GM);
     float* sRT = reinterpret_cast<float*>(smem + L::CK);  // R, overwritten in place by T
@@ -171,6 +213,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
     }
     if (warp == 0) tmem_alloc(s_base + L::TBASE, L::TMEM_COLS);
     if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;
+    if (tid < MX_SLOTS) sMx[tid] = 0u;
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TBASE);
     uint32_t phase = 0, phase_in = 0;
@@ -178,14 +221,12 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
 
     // Inputs of one chunk: the q, k, g and v tiles into X1 by six tensor-map copies issued by thread 32
     // (rows past T read as zero), completing on mbar_in; beta, this head's A_log and this thread's
-    // dt_bias entry into registers.  Thread 32 first lets the record stores it issued finish reading
-    // X1.  q / k are read back in the operand pass as units u = tid + NT * it: row
+    // dt_bias entry into registers.  q / k are read back in the operand pass as units u = tid + NT * it: row
     // i = 8 (u / 128) + u % 8, key group d8 = (u / 8) % 16.
     uint32_t beta_bits = 0;  // raw bf16 bits of beta for row tid (tid < 64), converted where used
     float alog_in = 0.f, bias_in = 0.f;
     auto load_inputs = [&](const Task& tk) {
         if (tid == 32) {
-            bulk_wait_read();
             mbar_expect_tx(mbar_in, 4u * 16384u);
             const int t0 = tk.c * CH;
             tma_load_4d(s_base + L::STG_G, &tm_g, 0, tk.hv, t0, tk.b, mbar_in);
@@ -251,7 +292,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 sSig[gd] = sig;
                 sERho[gd] = __expf(rho);
                 sFend[gd] = __expf(gend - sig);
-                reinterpret_cast<float*>(rec + Rec::VEC)[gd] = __expf(gend);
+                const float eg = __expf(gend);
+                reinterpret_cast<float*>(rec + Rec::VEC)[gd] = eg;
+                max_into_slot(eg, sMx + MX_EG, lane);  // warps 0-3 are exactly the gq = 0 threads
             }
         }
 
@@ -278,8 +321,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 kr[it] = *reinterpret_cast<const uint4*>(smem + L::STG_K + off);
             }
             if (norm_qk) add_row_sumsq(qr, kr, sSqQ, sSqK, tid, lane);  // totals complete after the barrier
-            // the previous chunk's record stores must be done reading CK before P3 rewrites it, and
-            // the staged tiles in X1 must all be read
+            // the previous chunk's record stores must be done reading KA, CK and VT (their staging) before this
+            // chunk rewrites them, and the staged tiles in X1 must all be read
             if (tid == 32) bulk_wait_read();
             __syncthreads();
 #pragma unroll
@@ -292,8 +335,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
         }
 
-        // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK; record parts Kend -> KA rows 0-127, Qtil -> QT -----
+        // ---- P3: [-Khat; Qhat] -> X1, Kchk -> CK, Kend^T -> KA rows 0-127 (A of M11); Qtil (fp32) -> QT;
+        //      the largest magnitudes of Qtil and Kend ----------------------------------------------------
         uint32_t kh[2][8];  // tf32 bits of -Khat (rotated), kept for Khat^T once Gam is no longer needed
+        float mq = 0.f, mk = 0.f;
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
             const int u = tid + NT * it;
@@ -317,11 +362,14 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             for (int t = 0; t < 8; ++t) {
                 const float e1 = __expf(gf[t] - rf[t]), e2 = __expf(sf[t] - gf[t]);
                 const float qh = scale * qf[t] * e1, kc = kf[t] * e2;
+                const float qtil = qh * ef[t], kend = kc * ff[t];
+                mq = fmaxf(mq, fabsf(qtil));
+                mk = fmaxf(mk, fabsf(kend));
                 wq_[t] = to_tf32(qh);
-                qt[t] = to_tf32(qh * ef[t]);
+                qt[t] = __float_as_uint(qtil);
                 kh[it][t] = to_tf32(-kf[t] * e1);
                 wc_[t] = to_tf32(kc);
-                ke[t] = to_tf32(kc * ff[t]);
+                ke[t] = to_tf32(kend);
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -342,12 +390,29 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 *reinterpret_cast<uint32_t*>(smem + L::KA + cm_off(8 * d8 + ((t + rot) & 7), i, CH)) = ke[t];
             rotate_groups8(kh[it], rot);  // stored transposed the same way below
         }
+        max_into_slot(mq, sMx + MX_QT, lane);
+        max_into_slot(mk, sMx + MX_K, lane);
         fence_proxy_async();
         cta_sync_tc();
-        if (tid == 32) {  // Qtil and Kend are final: their record stores run while M1 does
-            bulk_store(rec + Rec::WQ + 32768, s_base + L::QT, 32768);  // Wtil goes straight out later
-            bulk_store(rec + Rec::KA, s_base + L::KA, 32768);         // A goes straight to the record later
-            bulk_commit();
+        if (!slow && tid == 0) {
+            gemm_tf32(tmem, s_base + L::X1, KD / 4 * 128, s_base + L::CK, KD / 4 * 128, idesc_tf32(128, 64), KD / 8,
+                      false);
+            mma_commit(mbar);
+        }
+        // Qtil (fp32) into TMEM rows 64-127, columns 256-383, while M1 runs: M12 accumulates -A Wtil onto it
+        if (wq >= 2) {
+            const int i = 32 * (wq - 2) + lane;
+            uint32_t x[32];
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const uint4 v4 = *reinterpret_cast<const uint4*>(smem + L::QT + cm_off(i, 32 * wc + 4 * c4, KD));
+                x[4 * c4] = v4.x;
+                x[4 * c4 + 1] = v4.y;
+                x[4 * c4 + 2] = v4.z;
+                x[4 * c4 + 3] = v4.w;
+            }
+            tmem_st32(taddr(tmem, 32 * wq, 256 + 32 * wc), x);
+            tmem_wait_st();
         }
 
         // Khat^T into GM (B rows 0-127 of M7) once Gam is no longer read
@@ -365,11 +430,6 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
 
         // ---- A -> record (KA rows 128-191), R -> CK region (pitch RP) ----------------------------
         if (!slow) {
-            if (tid == 0) {
-                gemm_tf32(tmem, s_base + L::X1, KD / 4 * 128, s_base + L::CK, KD / 4 * 128, idesc_tf32(128, 64), KD / 8,
-                          false);
-                mma_commit(mbar);
-            }
             write_khat_t();
             const bool ok = mbar_wait(mbar, phase, WAIT_POLLS);
             fence_after_sync();
@@ -392,19 +452,22 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                                     j + 2 < i ? bi * __uint_as_float(raw[jj + 2]) : 0.f,
                                     j + 3 < i ? bi * __uint_as_float(raw[jj + 3]) : 0.f);
                 }
-            } else {  // rows 64-127 hold A (unmasked): masked, tf32, straight into the record
+            } else {  // rows 64-127 hold A (unmasked): masked, negated, tf32, into KA rows 192-255 (A of M12)
                 const int i = 32 * (wq - 2) + lane;
-                unsigned char* ra = rec + Rec::KA + 32768;
+                float m = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < 16; jj += 4) {
                     const int j = 16 * wc + jj;
-                    uint4 w4;
-                    w4.x = to_tf32(j + 0 <= i ? __uint_as_float(raw[jj + 0]) : 0.f);
-                    w4.y = to_tf32(j + 1 <= i ? __uint_as_float(raw[jj + 1]) : 0.f);
-                    w4.z = to_tf32(j + 2 <= i ? __uint_as_float(raw[jj + 2]) : 0.f);
-                    w4.w = to_tf32(j + 3 <= i ? __uint_as_float(raw[jj + 3]) : 0.f);
-                    *reinterpret_cast<uint4*>(ra + cm_off(i, j, CH)) = w4;
+                    float a4[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        a4[t] = j + t <= i ? __uint_as_float(raw[jj + t]) : 0.f;
+                        m = fmaxf(m, fabsf(a4[t]));
+                    }
+                    *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, j, CH)) =
+                        make_uint4(to_tf32(-a4[0]), to_tf32(-a4[1]), to_tf32(-a4[2]), to_tf32(-a4[3]));
                 }
+                max_into_slot(m, sMx + MX_A, lane);
             }
         } else {
             if (task + gridDim.x < ntasks) load_inputs(make_task(task + gridDim.x, T, H, HV, NC));
@@ -434,22 +497,27 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 av[x] = (j <= i) ? scale * a : 0.f;
                 rr[x] = (j < i) ? sBeta[i] * r : 0.f;
             }
+            {
+                float m = 0.f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) m = fmaxf(m, fabsf(av[x]));
+                max_into_slot(m, sMx + MX_A, lane);
+            }
             __syncthreads();  // Gam fully read: GM becomes Khat^T
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
                 const int p = tid + NT * x;
                 const int i = p >> 6, j = p & 63;
-                *reinterpret_cast<uint32_t*>(rec + Rec::KA + 32768 + cm_off(i, j, CH)) = to_tf32(av[x]);
+                *reinterpret_cast<uint32_t*>(smem + L::KA + 49152 + cm_off(i, j, CH)) = to_tf32(-av[x]);
                 sRT[i * RP + j] = rr[x];
             }
             write_khat_t();
         }
         __syncthreads();
 
-        // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 and 192-255 ----------
+        // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 --------------------------
         tri_inverse_diag16(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
-        if (tid == 32) bulk_wait_read();  // the Qtil store has read QT before Tb overwrites it
         tri_inverse_step32(sRT, sX, tid);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
@@ -466,15 +534,16 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             }
             const uint4 w4 = make_uint4(w[0], w[1], w[2], w[3]);
             *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, 4 * j4, CH)) = w4;
-            *reinterpret_cast<uint4*>(smem + L::KA + 49152 + cm_off(i, 4 * j4, CH)) = w4;
         }
         if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;  // read for the last time above; the next chunk's sums follow
         fence_proxy_async();
         cta_sync_tc();
 
-        // ---- M7: D[128][256] = [Tb; Tb] [Khat^T; V^T]^T; rows 0-63 and 64-127 both hold W | U ------
+        // ---- M7: D[:, 0:64] = Khat^T Tb^T = W^T and D[:, 64:128] = V^T Tb^T = U^T (rows d / v, columns i) ----
         if (tid == 0) {
-            gemm_tf32(tmem, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::GM, CH / 4 * 128, idesc_tf32(128, 256),
+            gemm_tf32(tmem, s_base + L::GM, CH / 4 * 128, s_base + L::KA + 32768, CH / 4 * 128, idesc_tf32(128, 64),
+                      CH / 8, false);
+            gemm_tf32(tmem + 64, s_base + L::VT, CH / 4 * 128, s_base + L::KA + 32768, CH / 4 * 128, idesc_tf32(128, 64),
                       CH / 8, false);
             mma_commit(mbar);
         }
@@ -484,34 +553,133 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             if (!__syncthreads_and(ok)) { aborted = true; break; }
             phase ^= 1u;
         }
+        // BT = [Wtil^T; U^T] (tf32 [256][64] over GM and VT, which M7 has read), Wtil^T = diag(e^rho) W^T: warp
+        // (wq, wc) stores 32 columns i of row 32 wq + lane of W^T (wc < 2) or of U^T (wc >= 2)
         {
-            // lane quarters 0-1 read W (rows 0-63), quarters 2-3 read U (rows 64-127); wc picks 32 columns
-            const int i = 32 * (wq & 1) + lane;
-            uint32_t r0[32];
-            tmem_ld32(taddr(tmem, 32 * wq, (wq < 2 ? 0 : 128) + 32 * wc), r0);
+            const int r = 32 * wq + lane;
+            const bool isW = wc < 2;
+            uint32_t x[32];
+            tmem_ld32(taddr(tmem, 32 * wq, (isW ? 0 : 64) + 32 * (wc & 1)), x);
             tmem_wait_ld();
-            if (wq < 2) {  // Wtil = W diag(e^rho) -> record WQ rows 0-63 (tf32, operand tiling)
-                unsigned char* rw = rec + Rec::WQ;
+            const float sc = isW ? sERho[r] : 1.f;
+            float m = 0.f;
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const float4 er = *reinterpret_cast<const float4*>(sERho + 32 * wc + 4 * c4);
-                    *reinterpret_cast<uint4*>(rw + cm_off(i, 32 * wc + 4 * c4, KD)) =
-                        make_uint4(to_tf32(er.x * __uint_as_float(r0[4 * c4])),
-                                   to_tf32(er.y * __uint_as_float(r0[4 * c4 + 1])),
-                                   to_tf32(er.z * __uint_as_float(r0[4 * c4 + 2])),
-                                   to_tf32(er.w * __uint_as_float(r0[4 * c4 + 3])));
-                }
-            } else {  // U^T (fp32, row = value column) -> CK region, free once Tb was built
-                float* ut = reinterpret_cast<float*>(smem + L::CK);
-#pragma unroll
-                for (int cc = 0; cc < 32; ++cc) ut[(32 * wc + cc) * CH + i] = __uint_as_float(r0[cc]);
+            for (int t = 0; t < 32; ++t) {
+                const float v = __uint_as_float(x[t]) * sc;
+                m = fmaxf(m, fabsf(v));
+                x[t] = to_tf32(v);
             }
+            max_into_slot(m, sMx + (isW ? MX_W : MX_U), lane);
+            const int n = (isW ? 0 : 128) + r;
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+                *reinterpret_cast<uint4*>(smem + L::GM + cm_off(n, 32 * (wc & 1) + 4 * c4, CH)) =
+                    make_uint4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
         }
         fence_proxy_async();
         cta_sync_tc();
+
+        // ---- M11: D[:, 0:256] = Kend^T BT^T = [G | KU];  M12: D[:, 256:512] = [Tb; -A] BT^T, rows 64-127:
+        //      Qtil - A Wtil = Q' (accumulated onto Qtil) and -A U -------------------------------------------
+        if (tid == 0) {
+            gemm_tf32(tmem, s_base + L::KA, CH / 4 * 128, s_base + L::GM, CH / 4 * 128, idesc_tf32(128, 256), CH / 8,
+                      false);
+            gemm_tf32(tmem + 256, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::GM, CH / 4 * 128,
+                      idesc_tf32(128, 128), CH / 8, true);
+            gemm_tf32(tmem + 384, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::VT, CH / 4 * 128,
+                      idesc_tf32(128, 128), CH / 8, false);
+            mma_commit(mbar);
+        }
+        {
+            const bool ok = mbar_wait(mbar, phase, WAIT_POLLS);
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) { aborted = true; break; }
+            phase ^= 1u;
+        }
+        // ---- read-out to the record, staged in shared memory that M11 and M12 have read (KA, VT) or that is
+        //      free since Tb (CK), then three bulk stores.  Every warp: 64 columns of [G | KU] (rows d = lane
+        //      quarter); the warps of lane quarters 2, 3 also 64 columns of [Q' | -A U] (rows i = d - 64).  The
+        //      fp16 exponents come from bounds on the tiles (64 products per entry, a factor 2 for the tf32
+        //      operands), so that one pass converts. --------------------------------------------------------
+        const float kmax = slot_value(sMx + MX_K), wmax = slot_value(sMx + MX_W);
+        const int e_g = fp16_scale_exponent(128.f * kmax * wmax);
+        const int e_u = fp16_scale_exponent(128.f * kmax * slot_value(sMx + MX_U));
+        const int e_q = fp16_scale_exponent(slot_value(sMx + MX_QT) + 128.f * slot_value(sMx + MX_A) * wmax);
+        {
+            const int d = 32 * wq + lane;
+            const bool isG = wc < 2;
+            const float f = exp2i(-(isG ? e_g : e_u));
+            uint32_t r[32];
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                tmem_ld32(taddr(tmem, 32 * wq, 64 * wc + 32 * h), r);
+                tmem_wait_ld();
+                uint4 w[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    w[c] = make_uint4(pack_f16x2(__uint_as_float(r[8 * c]) * f, __uint_as_float(r[8 * c + 1]) * f),
+                                      pack_f16x2(__uint_as_float(r[8 * c + 2]) * f, __uint_as_float(r[8 * c + 3]) * f),
+                                      pack_f16x2(__uint_as_float(r[8 * c + 4]) * f, __uint_as_float(r[8 * c + 5]) * f),
+                                      pack_f16x2(__uint_as_float(r[8 * c + 6]) * f, __uint_as_float(r[8 * c + 7]) * f));
+                if (isG) {  // G row d, columns 64 wc + 32 h + 8 c: operand tiling
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(smem + L::KA + cm_off16(d, 64 * wc + 32 * h + 8 * c, KD)) = w[c];
+                } else {    // KU row d, value columns v = 64 (wc - 2) + 32 h + 8 c: blocks of 16 columns
+                    const int v0 = 64 * (wc - 2) + 32 * h;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int v = v0 + 8 * c;
+                        *reinterpret_cast<uint4*>(smem + L::CK + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2) = w[c];
+                    }
+                }
+            }
+            if (wq >= 2) {
+                const int i = d - 64;
+                const float fq = exp2i(-e_q);
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    tmem_ld32(taddr(tmem, 32 * wq, 256 + 64 * wc + 32 * h), r);
+                    tmem_wait_ld();
+                    if (isG) {  // Q' row i, columns 64 wc + 32 h + 8 c: operand tiling, rows 128-191 of [G; Q']
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(smem + L::KA + Rec::QP_OFF + cm_off16(i, 64 * wc + 32 * h + 8 * c, KD)) =
+                                make_uint4(pack_f16x2(__uint_as_float(r[8 * c]) * fq, __uint_as_float(r[8 * c + 1]) * fq),
+                                           pack_f16x2(__uint_as_float(r[8 * c + 2]) * fq, __uint_as_float(r[8 * c + 3]) * fq),
+                                           pack_f16x2(__uint_as_float(r[8 * c + 4]) * fq, __uint_as_float(r[8 * c + 5]) * fq),
+                                           pack_f16x2(__uint_as_float(r[8 * c + 6]) * fq, __uint_as_float(r[8 * c + 7]) * fq));
+                    } else {    // A U row i (negated back), value columns 64 (wc - 2) + 32 h + 4 c: fp32
+                        const int v0 = 64 * (wc - 2) + 32 * h;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int v = v0 + 4 * c;
+                            *reinterpret_cast<uint4*>(smem + L::VT + (((v >> 4) * 64 + i) * 16 + (v & 15)) * 4) =
+                                make_uint4(r[4 * c] ^ 0x80000000u, r[4 * c + 1] ^ 0x80000000u, r[4 * c + 2] ^ 0x80000000u,
+                                           r[4 * c + 3] ^ 0x80000000u);
+                        }
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
         if (tid == 32) {
-            bulk_store(rec + Rec::UT, s_base + L::CK, 32768);
+            bulk_store(rec + Rec::WQ, s_base + L::KA, Rec::WQ_BYTES);
+            bulk_store(rec + Rec::KU, s_base + L::CK, 32768);
+            bulk_store(rec + Rec::AU, s_base + L::VT, 32768);
             bulk_commit();
+        }
+        if (tid == 0) {  // the scale block; then the maxima start over for the next chunk
+            int* sc = reinterpret_cast<int*>(rec + Rec::SCL);
+            sc[0] = e_g;
+            sc[1] = e_q;
+            sc[2] = e_u;
+            sc[3] = (int)sMx[MX_EG];
+#pragma unroll
+            for (int x = 0; x < MX_SLOTS; ++x) sMx[x] = 0u;
         }
     }
 
@@ -545,34 +713,48 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
     }
 }
 
-// Thread layout: warp w serves TMEM lane quarter w % 4 (rows 32 (w % 4) + lane of every
-// accumulator) and column half w / 4 of the value block (HALF = VB / 2 columns).
+// Thread layout: warp w < 8 serves TMEM lane quarter w % 4 (rows 32 (w % 4) + lane of every
+// accumulator) and column half w / 4 of the value block (HALF = VB / 2 columns); warp 8 issues the record
+// copies and the tensor-core products (one thread), so that no state row waits while the products issue.
 //
 // One CTA runs chunks [seg L, min(NC, seg L + L)) of one (sequence, value head) pair for one block of
 // VB state columns.  With NS = 1 that is the whole sequence.  For long sequences the chunks are split
-// into NS segments: the chunk map S -> e^{Gam_end} S + Kend (U - Wtil S) is affine in S, so a segment
-// maps its entering state by S -> M S + b, and the segments can run in parallel (DeltaNet-family digest,
+// into NS segments: the chunk map S -> e^{Gam_end} S - G S + KU is affine in S, so a segment maps its
+// entering state by S -> M S + b, and the segments can run in parallel (DeltaNet-family digest,
 // "Chunkwise Triton pipeline": the state pass is the only traversal between chunks).
 //   STATE_CARRY  two CTA halves per (pair, segment but the last) carry X = [M | b] through the segment
-//                from [I | 0]:
-//                half 0 the M columns (identity start, no U: E = -Wtil X), half 1 the b columns (zero
+//                from [I | 0]: half 0 the M columns (identity start, no KU), half 1 the b columns (zero
 //                start); X is written to `carry` at the end.  No outputs.
 //   STATE_OUT    the chunks from the state entering the segment, with the outputs; the last segment
 //                writes S_T.  Unsplit (NS = 1) the entering state is S0; split, every segment reads it
 //                from `carry`, where scan_chain_kernel left it (so S_T may alias S0 in both cases).
+//
+// Per chunk c, one tensor-core round trip is on the chain: the issuer issues D_S = G S_c (and, with outputs,
+// D_O = [G; Q'] S_c into the buffer of c's parity) on the S operand of c; every thread waits for D_S and
+// updates its part of the state, S_c+1 = e^{Gam_end} S_c - D_S + KU, writes the next S operand, and meets
+// the others at one barrier.  The outputs of chunk c are read out by lane quarters 2, 3 in step c + 1,
+// before they wait for that step's D_S.
+//
+// The state operand is fp16(S_c 2^-sig_c).  sig_c comes from a bound on |S_c| that every thread computes
+// alike, with no reduction on the chain: at the start the exact maximum, then
+//   bound_c+1 = max e^{Gam_end} max|S_c| + 256 * 2^(14+eg) max|S_c| + 2 * 2^(14+eu),
+// where |G| <= 2^(14+eg) and |KU| <= 2^(14+eu) (128 terms in G S; a factor 2 for the fp16 roundings) and
+// max|S_c| is the exact CTA maximum, reduced one step late through per-warp slots.
 template <int VB, int MODE>
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __restrict__ S0, int T, int HV, int NC,
                    int L, int NS, bf16* __restrict__ o, float* __restrict__ S_T, float* __restrict__ carry,
                    unsigned int* __restrict__ status) {
-    using Lay = StateLayout<VB>;
+    using Lay = StateLayout<VB, MODE>;
     constexpr bool OUTS = MODE == STATE_OUT;
     constexpr int NVB = VD / VB;
     constexpr int NH = OUTS ? 1 : 2;
     constexpr int HALF = VB / 2;
+    constexpr int NBUF = Lay::NBUF;
     extern __shared__ __align__(1024) unsigned char smem[];
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t bar_wq = s_base + Lay::MBAR, bar_mma = bar_wq + 8, bar_ka0 = bar_wq + 16, bar_out = bar_wq + 32;
+    const uint32_t bar_rec0 = s_base + Lay::MBAR, bar_chain = bar_rec0 + 8 * NBUF, bar_out0 = bar_chain + 8;
+    volatile unsigned int* sMaxS = reinterpret_cast<volatile unsigned int*>(smem + Lay::SMX);  // [2][8]
     int rest = blockIdx.x;
     const int vbi = rest % NVB;
     rest /= NVB;
@@ -586,52 +768,45 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     const int b = pair / HV, hv = pair - b * HV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, c0 = (warp >> 2) * HALF;  // lane quarter, first column of this half
-    const int rot = lane >> 2;                          // store rotation (see rotate_groups8)
     const size_t v_row = (size_t)HV * VD;
     const unsigned char* rec0 = rec_base + (size_t)pair * NC * Rec::BYTES;
     auto rec = [&](int c) { return rec0 + (size_t)c * Rec::BYTES; };
     // carry slots of (pair, segment): [2][KD][VD] fp32, M then b
     auto carry_slot = [&](int sg, int hf) { return carry + (((size_t)pair * NS + sg) * 2 + hf) * KD * VD; };
+    auto slot_of = [&](int c) { return (c - c_begin) % NBUF; };
 
     if (tid == 0) {
-        mbar_init(bar_wq, 1);
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_ka0, 1);
-        mbar_init(bar_ka0 + 8, 1);
-        mbar_init(bar_out, 1);
+        for (int k = 0; k < NBUF + 3; ++k) mbar_init(bar_rec0 + 8 * k, 1);
     }
     if (warp == 0) tmem_alloc(s_base + Lay::TBASE, Lay::TMEM_COLS);
     cta_sync_tc();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::TBASE);
 
-    // loads in flight, for the bounded drain on abort: bit 0 wq, bit 1 + buf ka
-    uint32_t pending = 0;
-    auto load_wq = [&](int c) {
-        mbar_expect_tx(bar_wq, 65536);
-        bulk_load(s_base + Lay::WQ, rec(c) + Rec::WQ, 65536, bar_wq);
-        pending |= 1u;
+    // record copies in flight (bit k: slot k), for the bounded drain on abort; per-slot phases
+    uint32_t pending = 0, ph_rec = 0;
+    auto load_rec = [&](int c) {
+        const int k = slot_of(c);
+        const uint32_t bar = bar_rec0 + 8 * k, dst = s_base + Lay::slot(k);
+        mbar_expect_tx(bar, Lay::WQ_LOAD + (use_u ? VB * 256u : 0u) + (OUTS ? VB * 256u : 0u) + Rec::VEC_LOAD);
+        bulk_load(dst, rec(c) + Rec::WQ, Lay::WQ_LOAD, bar);
+        if (use_u) bulk_load(dst + Lay::KU_OFF, rec(c) + Rec::KU + (vb0 / 16) * 4096, VB * 256, bar);
+        if (OUTS) bulk_load(dst + Lay::AU_OFF, rec(c) + Rec::AU + (vb0 / 16) * 4096, VB * 256, bar);
+        bulk_load(dst + Lay::VEC_OFF, rec(c) + Rec::VEC, Rec::VEC_LOAD, bar);
+        pending |= 1u << k;
     };
-    // the carry pass reads Kend only (no A) and, for the M columns, no U
-    constexpr uint32_t KA_LOAD = OUTS ? Rec::KA_BYTES : 32768u;
-    auto load_ka = [&](int c, int buf) {
-        const uint32_t bar = bar_ka0 + 8 * buf;
-        mbar_expect_tx(bar, KA_LOAD + (use_u ? VB * 256u : 0u) + 512u);
-        bulk_load(s_base + Lay::ka(buf), rec(c) + Rec::KA, KA_LOAD, bar);
-        if (use_u) bulk_load(s_base + Lay::ka(buf) + Lay::UT_OFF, rec(c) + Rec::UT + vb0 * 256, VB * 256, bar);
-        bulk_load(s_base + Lay::ka(buf) + Lay::VEC_OFF, rec(c) + Rec::VEC, 512, bar);
-        pending |= 2u << buf;
-    };
-    // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32
+    // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32 (state warps)
+    const bool issuer = tid == ISSUER, state_warp = warp < STATE_WARPS;
+    const bool loader = tid == 0;  // issues the record copies (its warp waits for D_S with time to spare)
     const int d = 32 * wq + lane;
     float s[HALF];
     {
         const float* src = nullptr;  // row-major [KD][VD] source of the entering state, or none (zeros)
-        if (OUTS) src = NS == 1 ? (S0 ? S0 + (size_t)pair * KD * VD : nullptr) : carry_slot(seg == 0 ? NS - 1 : seg - 1, seg == 0 ? 0 : 1);
+        if (OUTS && state_warp) src = NS == 1 ? (S0 ? S0 + (size_t)pair * KD * VD : nullptr) : carry_slot(seg == 0 ? NS - 1 : seg - 1, seg == 0 ? 0 : 1);
 #pragma unroll
         for (int j = 0; j < HALF; j += 4) {
             float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)d * VD + vb0 + c0 + j)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (!OUTS && half == 0) {  // identity: row d has its 1 in column d
+            if (!OUTS && half == 0 && state_warp) {  // identity: row d has its 1 in column d
                 const int col = vb0 + c0 + j;
                 x = make_float4(col == d ? 1.f : 0.f, col + 1 == d ? 1.f : 0.f, col + 2 == d ? 1.f : 0.f,
                                 col + 3 == d ? 1.f : 0.f);
@@ -646,156 +821,173 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
     // grid was launched as its programmatic dependent; the prep CTAs release it once their records
     // are complete, so only the launch itself overlaps their tail)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 0) {
-        load_wq(c_begin);
-        load_ka(c_begin, 0);
-        if (Lay::NKA == 2 && c_begin + 1 < c_end) load_ka(c_begin + 1, 1);
+    if (loader) {  // two chunks ahead
+        load_rec(c_begin);
+        if (c_begin + 1 < c_end) load_rec(c_begin + 1);
     }
-    // tf32(S)^T into the B operand of M8; lanes sharing a bank store different columns
-    auto write_sop = [&]() {
-        uint32_t w[HALF];
+    // this warp's largest |S| into slot `par`
+    auto warp_max_s = [&](int par) {
+        float m = 0.f;
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) w[j] = to_tf32(s[j]);
-        rotate_groups8(w, rot);
+        for (int j = 0; j < HALF; ++j) m = fmaxf(m, fabsf(s[j]));
+        m = warp_max_nonneg(m);
+        if (lane == 0) sMaxS[8 * par + warp] = __float_as_uint(m);
+    };
+    auto cta_max_s = [&](int par) {
+        float m = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) m = fmaxf(m, __uint_as_float(sMaxS[8 * par + w]));
+        return m;
+    };
+    // fp16(S 2^-sig)^T into S operand `buf`: element (v, d) of the padded tiling; the 32 lanes (d) of a
+    // warp store one column v into 16 different banks
+    const uint32_t sop_thread = (uint32_t)(c0 >> 3) * Lay::SOP_SBO + (uint32_t)(d >> 3) * Lay::SOP_LBO + (uint32_t)(d & 7) * 2;
+    auto write_sop = [&](int buf, int sig) {
+        const float f = exp2i(-sig);
+        unsigned char* sop = smem + Lay::SOP + buf * Lay::SOP_BYTES + sop_thread;
 #pragma unroll
         for (int j = 0; j < HALF; ++j)
-            *reinterpret_cast<uint32_t*>(smem + Lay::SOP + cm_off(c0 + (j & ~7) + ((j + rot) & 7), d, KD)) = w[j];
+            *reinterpret_cast<uint16_t*>(sop + (j >> 3) * Lay::SOP_SBO + (j & 7) * 16) = to_f16_bits(s[j] * f);
     };
-    uint32_t ph_wq = 0, ph_mma = 0, ph_ka = 0, ph_out = 0;
-    bool aborted = false;
-    write_sop();
-    fence_proxy_async();
-    cta_sync_tc();
-    for (int c = c_begin; c < c_end && !aborted; ++c) {
-        const int buf = (Lay::NKA == 2) ? ((c - c_begin) & 1) : 0;
-        const int n = min(CH, T - c * CH);
-        // ---- M8: D1 = [Wtil; Qtil] S ------------------------------------------------------------
-        bool ok = true;
-        if (tid == 0) {
-            ok = mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
-            if (ok) {
-                pending &= ~1u;
-                gemm_tf32(tmem + Lay::D1, s_base + Lay::WQ, KD / 4 * 128, s_base + Lay::SOP, KD / 4 * 128,
-                          idesc_tf32(128, VB), KD / 8, false);
-                mma_commit(bar_mma);
-            }
-        }
-        ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS) && ok;
-        ok = mbar_wait(bar_ka0 + 8 * buf, (ph_ka >> buf) & 1u, WAIT_POLLS) && ok;
+    // outputs of chunk c (lane quarters 2, 3: rows i = d - 64 of D_O), O = Q' S_c 2^(eq + sig_c) + A U
+    uint32_t ph_out = 0;
+    auto outputs = [&](int c, float f_q) -> bool {
+        const int par = (c - c_begin) & 1;
+        const bool ok = mbar_wait(bar_out0 + 8 * par, (ph_out >> par) & 1u, WAIT_POLLS);
         fence_after_sync();
-        if (!__syncthreads_and(ok)) { aborted = true; break; }
-        // phases advance only on success, so that on abort they name the operations still pending
-        ph_wq ^= 1u;
-        ph_mma ^= 1u;
-        ph_ka ^= 1u << buf;
-        // this chunk's e^{Gam_end}, read before a single KA buffer is refilled below
-        const float eg = reinterpret_cast<const float*>(smem + Lay::ka(buf) + Lay::VEC_OFF)[d];
-        if (tid == 0) {
-            pending &= ~(2u << buf);
-            if (c + 1 < c_end) load_wq(c + 1);  // M8 has read WQ
-        }
-        // ---- E = U - Wtil S (rows 0-63: lane quarters 0, 1) -> E^T tf32 operand ------------------
-        const uint32_t ka = s_base + Lay::ka(buf);
-        {
-            uint32_t r[HALF];
-            if (wq < 2) {
-                const float* sU = reinterpret_cast<const float*>(smem + Lay::ka(buf) + Lay::UT_OFF);
-                tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D1 + c0), r);
-                tmem_wait_ld();
+        if (!ok) return false;
+        ph_out ^= 1u << par;
+        const int i = d - 64, n = min(CH, T - c * CH);
+        const float* sAU = reinterpret_cast<const float*>(smem + Lay::slot(slot_of(c)) + Lay::AU_OFF);
+        constexpr int SUB = HALF < 16 ? HALF : 16;
 #pragma unroll
-                for (int vv = 0; vv < HALF; ++vv)
-                    r[vv] = to_tf32((use_u ? sU[(c0 + vv) * CH + d] : 0.f) - __uint_as_float(r[vv]));
-                rotate_groups8(r, rot);
-            }
-            if constexpr (Lay::ALIAS_E) __syncthreads();  // every U^T read done before E^T overwrites them
-            if (wq < 2) {
-#pragma unroll
-                for (int vv = 0; vv < HALF; ++vv)
-                    *reinterpret_cast<uint32_t*>(smem + Lay::EOP + cm_off(c0 + (vv & ~7) + ((vv + rot) & 7), d, CH)) =
-                        r[vv];
-            }
-        }
-        fence_proxy_async();
-        cta_sync_tc();
-        // ---- M10: D2 = Kend E (the state side), then M9: D1[64:] += A E (the outputs), each with its
-        //      own commit, so that the state update starts after M10 while M9 still runs -------------
-        if (tid == 0) {
-            gemm_tf32(tmem + Lay::D2, ka, CH / 4 * 128, s_base + Lay::EOP, CH / 4 * 128, idesc_tf32(128, VB), CH / 8,
-                      false);
-            mma_commit(bar_mma);
-            if (OUTS) {
-                gemm_tf32(tmem + Lay::D1, ka + 16384, CH / 4 * 128, s_base + Lay::EOP, CH / 4 * 128,
-                          idesc_tf32(128, VB), CH / 8, true);
-                mma_commit(bar_out);
-            }
-        }
-        ok = mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
-        fence_after_sync();
-        if (!__syncthreads_and(ok)) { aborted = true; break; }
-        ph_mma ^= 1u;
-        // ---- state: S = e^{Gam_end} S + D2 --------------------------------------------------------
-        {
-            uint32_t r[HALF];
-            tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D2 + c0), r);
+        for (int j0 = 0; j0 < HALF; j0 += SUB) {
+            uint32_t r[SUB];
+            tmem_ld_row<SUB>(taddr(tmem, 32 * wq, Lay::D_O + par * VB + c0 + j0), r);
             tmem_wait_ld();
+            if (i < n) {
+                bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0 + c0 + j0;
 #pragma unroll
-            for (int j = 0; j < HALF; ++j) s[j] = fmaf(eg, s[j], __uint_as_float(r[j]));
-        }
-        bool ok_out = true;
-        if constexpr (OUTS) {
-            // ---- outputs (rows 64-127 of D1: lane quarters 2, 3), once M9 is done; thread 0 waits for
-            //      it too before a KA buffer M9 reads is refilled -------------------------------------
-            if (wq >= 2 || tid == 0) {
-                ok_out = mbar_wait(bar_out, ph_out, WAIT_POLLS);
-                fence_after_sync();
-            }
-            if (wq >= 2 && ok_out) {
-                const int i = d - 64;
-                uint32_t r[HALF];
-                tmem_ld_row<HALF>(taddr(tmem, 32 * wq, Lay::D1 + c0), r);
-                tmem_wait_ld();
-                if (i < n) {
-                    bf16* op = o + ((size_t)b * T + (size_t)c * CH + i) * v_row + (size_t)hv * VD + vb0 + c0;
+                for (int j = 0; j < SUB; j += 8) {
+                    const int v = c0 + j0 + j;  // column within the block; AU by blocks of 16 columns
+                    const float4 a0 = *reinterpret_cast<const float4*>(sAU + ((v >> 4) * 64 + i) * 16 + (v & 15));
+                    const float4 a1 = *reinterpret_cast<const float4*>(sAU + ((v >> 4) * 64 + i) * 16 + (v & 15) + 4);
+                    const float au[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                    uint32_t w[4];
 #pragma unroll
-                    for (int j = 0; j < HALF; j += 8) {
-                        uint4 w;
-                        __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
-                        __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                        __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
-                        __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                        w.x = *reinterpret_cast<uint32_t*>(&p0);
-                        w.y = *reinterpret_cast<uint32_t*>(&p1);
-                        w.z = *reinterpret_cast<uint32_t*>(&p2);
-                        w.w = *reinterpret_cast<uint32_t*>(&p3);
-                        *reinterpret_cast<uint4*>(op + j) = w;
+                    for (int t = 0; t < 4; ++t) {
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(__uint_as_float(r[j + 2 * t]), f_q, au[2 * t]),
+                                                                  fmaf(__uint_as_float(r[j + 2 * t + 1]), f_q, au[2 * t + 1]));
+                        w[t] = *reinterpret_cast<uint32_t*>(&pr);
                     }
+                    *reinterpret_cast<uint4*>(op + j) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
         }
-        // a single KA buffer (and, with 128 columns, the E^T operand over its U^T rows) is refilled once
-        // the products that read it (M10, and M9 when there are outputs) are done
-        if (Lay::NKA == 1 && tid == 0 && ok_out && c + 1 < c_end) load_ka(c + 1, 0);
-        // ---- the next chunk's S operand --------------------------------------------------------
-        if (c + 1 < c_end) write_sop();
+        return true;
+    };
+    uint32_t ph_chain = 0;
+    bool aborted = false;
+    if (state_warp) warp_max_s(0);
+    __syncthreads();
+    int sig = fp16_scale_exponent(cta_max_s(0));  // exact max |S| of the entering state
+    float fq_prev = 0.f;      // output scale of the previous chunk
+    if (state_warp) write_sop(0, sig);
+    fence_proxy_async();
+    cta_sync_tc();
+    for (int c = c_begin; c < c_end && !aborted; ++c) {
+        const int par = (c - c_begin) & 1, k = slot_of(c);
+        const uint32_t sl = s_base + Lay::slot(k);
+        const uint32_t sop = s_base + Lay::SOP + (Lay::NSOP == 2 ? par : 0) * Lay::SOP_BYTES;
+        // ---- chain (and output) products on the S operand of chunk c ---------------------------------
+        bool ok = mbar_wait(bar_rec0 + 8 * k, (ph_rec >> k) & 1u, WAIT_POLLS);
+        ph_rec ^= 1u << k;
+        if (loader && ok) pending &= ~(1u << k);
+        if (issuer && ok) {
+            gemm_f16_bpad(tmem + Lay::D_S, sl, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO, idesc_f16(128, VB),
+                          KD / 16, false);
+            mma_commit(bar_chain);  // before the output product: the chain waits for G S alone
+            if (OUTS) {  // rows 64-191 of [G; Q']: D_O rows 64-127 hold Q' S
+                gemm_f16_bpad(tmem + Lay::D_O + par * VB, sl + 16384, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO,
+                              idesc_f16(128, VB), KD / 16, false);
+                mma_commit(bar_out0 + 8 * par);
+            }
+        }
+        fence_after_sync();
+        const unsigned char* vec = smem + Lay::slot(k) + Lay::VEC_OFF;
+        const float eg = reinterpret_cast<const float*>(vec)[d];
+        const int* scl = reinterpret_cast<const int*>(vec + (Rec::SCL - Rec::VEC));
+        const int e_g = scl[0], e_q = scl[1], e_u = scl[2];
+        const float egmax = __int_as_float(scl[3]);
+        // scales: this chunk's outputs (sig_c), and the bound on S_c+1 that sets sig_c+1 (max |S_c| exact)
+        const float mS = cta_max_s(par);
+        const float fq = exp2i(e_q) * exp2i(sig);
+        const float f_g = exp2i(e_g) * exp2i(sig), f_u = exp2i(e_u);
+        const int sig_next = fp16_scale_exponent(egmax * mS + 256.f * exp2i(14 + e_g) * mS +
+                                                 (use_u ? 2.f * exp2i(14 + e_u) : 0.f));
+        // ---- the previous chunk's outputs, while D_S runs -------------------------------------------
+        if (OUTS && state_warp && wq >= 2 && c > c_begin) ok = outputs(c - 1, fq_prev) && ok;
+        // ---- state: S = e^{Gam_end} S - G S + KU ------------------------------------------------------
+        const unsigned char* sKU = smem + Lay::slot(k) + Lay::KU_OFF;
+        constexpr int PIECE = HALF < 32 ? HALF : 32;
+        uint4 ku_first[PIECE / 8];  // this thread's KU of the first piece, read while D_S runs
+#pragma unroll
+        for (int j = 0; j < PIECE; j += 8) {
+            const int v = c0 + j;
+            ku_first[j / 8] = use_u && state_warp ? *reinterpret_cast<const uint4*>(sKU + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (state_warp) ok = mbar_wait(bar_chain, ph_chain, WAIT_POLLS) && ok;
+        ph_chain ^= 1u;
+        fence_after_sync();
+        if (ok && state_warp) {
+#pragma unroll
+            for (int j0 = 0; j0 < HALF; j0 += PIECE) {
+                uint32_t r[PIECE];
+                tmem_ld_row<PIECE>(taddr(tmem, 32 * wq, Lay::D_S + c0 + j0), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < PIECE; j += 8) {
+                    float ku[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (use_u) {
+                        const int v = c0 + j0 + j;
+                        const uint4 u4 = j0 == 0 ? ku_first[j / 8]
+                                                 : *reinterpret_cast<const uint4*>(sKU + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2);
+                        f16x2_to_f32(u4.x, ku[0], ku[1]);
+                        f16x2_to_f32(u4.y, ku[2], ku[3]);
+                        f16x2_to_f32(u4.z, ku[4], ku[5]);
+                        f16x2_to_f32(u4.w, ku[6], ku[7]);
+                    }
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        s[j0 + j + t] = fmaf(ku[t], f_u, fmaf(eg, s[j0 + j + t], -__uint_as_float(r[j + t]) * f_g));
+                }
+            }
+            // ---- the next chunk's S operand (its buffer is free: the products of chunk c - 1 that read it
+            //      are complete, since D_S of chunk c completes after them); max |S_c+1| for the next bound --
+            if (c + 1 < c_end) write_sop(Lay::NSOP == 2 ? par ^ 1 : 0, sig_next);
+            warp_max_s(par ^ 1);
+        }
+        sig = sig_next;
         fence_proxy_async();
         fence_before_sync();
-        if (!__syncthreads_and(ok_out)) { aborted = true; break; }
+        if (!__syncthreads_and(ok)) { aborted = true; break; }
         fence_after_sync();
-        if (OUTS) ph_out ^= 1u;
-        if (Lay::NKA == 2 && tid == 0 && c + 2 < c_end) load_ka(c + 2, buf);
+        if (loader && c + 2 < c_end) load_rec(c + 2);  // into the slot of chunk c - 1 (outputs) or c (no outputs)
+        fq_prev = fq;
     }
+    if (OUTS && !aborted && state_warp && wq >= 2 && c_end > c_begin) aborted = !outputs(c_end - 1, fq_prev);
+    aborted = __syncthreads_or(aborted) != 0;
 
     if (aborted) {
-        if (tid == 0) {
+        // bounded drain of copies and MMAs still in flight before shared memory and TMEM go away
+        if (loader) {
             atomicOr(status, STATUS_TIMEOUT);
-            // bounded drain of copies and MMAs still in flight before shared memory and TMEM go away
-            if (pending & 1u) mbar_wait(bar_wq, ph_wq, WAIT_POLLS);
-            for (int bb = 0; bb < Lay::NKA; ++bb)
-                if (pending & (2u << bb)) mbar_wait(bar_ka0 + 8 * bb, (ph_ka >> bb) & 1u, WAIT_POLLS);
-            mbar_wait(bar_mma, ph_mma, WAIT_POLLS);
-            if (OUTS) mbar_wait(bar_out, ph_out, WAIT_POLLS);
+            for (int bb = 0; bb < NBUF; ++bb)
+                if (pending & (1u << bb)) mbar_wait(bar_rec0 + 8 * bb, (ph_rec >> bb) & 1u, WAIT_POLLS);
         }
-    } else {
+        if (issuer) mbar_wait(bar_chain, ph_chain, WAIT_POLLS);
+    } else if (state_warp) {
         float* dst = nullptr;
         if (!OUTS) dst = carry_slot(seg, half);
         else if (S_T && seg == NS - 1) dst = S_T + (size_t)pair * KD * VD;
@@ -871,26 +1063,28 @@ scan_chain_kernel(const float* __restrict__ S0, float* __restrict__ carry, int N
 
 // ---------------------------------------------------------------------------------------------
 // Segments of the state pass.  Cost model, in thousands of cycles of one CTA per SM: the unsplit pass is
-// a chain of NC steps per wave of (pair, value block) CTAs, one step taking about 3.6K cycles with 16
-// columns, 4.8K with 32 and 6K with 64 (as launch_chunk_split picks the block width); the split one runs
-// 2 x pairs x (NS - 1) carry CTAs, then pairs x NS output CTAs, of L chunks each, in waves over the SMs,
-// one 128-column step taking about 10.3K cycles, plus the segment chain at about 3K cycles per segment
-// (measured on B200 with tf32 records).  The split therefore pays only where the unsplit pass leaves SMs
-// idle: few (sequence, head) pairs and long sequences.  The number of SMs is a planning constant (a
-// B200's 148), so that the workspace size does not depend on the device; the split is taken where the
-// model gains at least a fifth.
+// a chain of NC steps per wave of (pair, value block) CTAs, T_UNSPLIT16 / T_UNSPLIT32 per step with 16 / 32
+// columns (as launch_chunk_split picks the block width); the split one runs 4 x pairs x (NS - 1) carry
+// CTAs (64 columns, T_CARRY per step), then 4 x pairs x NS output CTAs (32 columns), of L chunks each, in
+// waves over the SMs, plus the segment chain at T_CHAIN per segment.  The split therefore pays only where
+// the unsplit pass leaves SMs idle: few (sequence, head) pairs and long sequences.  The number of SMs is a
+// planning constant (a B200's 148), so that the workspace size does not depend on the device; the split is
+// taken where the model gains at least a fifth.
+constexpr double T_UNSPLIT16 = 1.3, T_UNSPLIT32 = 1.4, T_CARRY = 1.5, T_CHAIN = 3.0;
+
 ScanPlan chunk_scan_plan(long long pairs, int NC) {
     constexpr long long kPlanSMs = 148;
-    const long long nvb = pairs * 8 <= kPlanSMs ? 8 : pairs * 4 <= kPlanSMs ? 4 : 2;
-    const double t_unsplit = nvb == 8 ? 3.6 : nvb == 4 ? 4.8 : 6.0, t_split = 10.3, t_chain = 3.0;
+    const bool narrow = pairs * 8 <= kPlanSMs;
+    const long long nvb = narrow ? 8 : 4;
     ScanPlan plan{NC, 1};
-    double best = 0.8 * (double)NC * t_unsplit * (double)((pairs * nvb + kPlanSMs - 1) / kPlanSMs);
+    double best = 0.8 * (double)NC * (narrow ? T_UNSPLIT16 : T_UNSPLIT32) *
+                  (double)((pairs * nvb + kPlanSMs - 1) / kPlanSMs);
     for (int Lc : {8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256}) {
         if (Lc >= NC) break;
         const long long NS = (NC + Lc - 1) / Lc;
-        const long long wa = (2 * pairs * (NS - 1) + kPlanSMs - 1) / kPlanSMs;
-        const long long wc = (pairs * NS + kPlanSMs - 1) / kPlanSMs;
-        const double cost = (double)(wa + wc) * Lc * t_split + t_chain * (double)NS;
+        const long long wa = (4 * pairs * (NS - 1) + kPlanSMs - 1) / kPlanSMs;
+        const long long wc = (4 * pairs * NS + kPlanSMs - 1) / kPlanSMs;
+        const double cost = (double)wa * Lc * T_CARRY + (double)wc * Lc * T_UNSPLIT32 + T_CHAIN * (double)NS;
         if (cost < best) {
             best = cost;
             plan = ScanPlan{Lc, (int)NS};
@@ -956,7 +1150,7 @@ cudaError_t launch_prep(const ChunkArgs& a, int NC, int ntasks, int grid) {
 
 template <int VB, int MODE>
 cudaError_t launch_state(const ChunkArgs& a, int NC, ScanPlan plan, float* carry, bool dependent) {
-    using L = StateLayout<VB>;
+    using L = StateLayout<VB, MODE>;
     auto kern = chunk_state_kernel<VB, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
     if (e != cudaSuccess) return e;
@@ -994,17 +1188,16 @@ cudaError_t launch_chunk_split(const ChunkArgs& a) {
     const long long pairs = (long long)a.B * a.HV;
     const ScanPlan plan = chunk_scan_plan(pairs, NC);
     if (plan.NS == 1) {
-        // value-block width: enough (pair, block) CTAs to cover the SMs, blocks as wide as that allows
+        // value-block width: 16 columns while the (pair, block) CTAs still fit on the SMs, else 32
         if (pairs * 8 <= nsm) return launch_state<16, STATE_OUT>(a, NC, plan, nullptr, true);
-        if (pairs * 4 <= nsm) return launch_state<32, STATE_OUT>(a, NC, plan, nullptr, true);
-        return launch_state<64, STATE_OUT>(a, NC, plan, nullptr, true);
+        return launch_state<32, STATE_OUT>(a, NC, plan, nullptr, true);
     }
     // long sequences: carry [M | b] through every segment, chain the segments, then the outputs
     float* carry = reinterpret_cast<float*>(static_cast<unsigned char*>(a.scratch) + (size_t)pairs * NC * Rec::BYTES);
-    if ((e = launch_state<128, STATE_CARRY>(a, NC, plan, carry, true)) != cudaSuccess) return e;
+    if ((e = launch_state<64, STATE_CARRY>(a, NC, plan, carry, true)) != cudaSuccess) return e;
     scan_chain_kernel<<<(unsigned)(pairs * (VD / CHAIN_COLS)), CHAIN_THREADS, 0, a.stream>>>(a.S0, carry, plan.NS);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_state<128, STATE_OUT>(a, NC, plan, carry, false);
+    return launch_state<32, STATE_OUT>(a, NC, plan, carry, false);
 }
 
 }  // namespace kda

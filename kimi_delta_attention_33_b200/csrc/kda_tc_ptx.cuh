@@ -69,6 +69,96 @@ __device__ __forceinline__ void gemm_tf32(uint32_t d_tmem, uint32_t a_addr, uint
                  (ks > 0 || accumulate) ? 1u : 0u);
 }
 
+// ---- kind::f16 with fp16 operands (both A and B fp16), fp32 accumulation ----------------------------
+// Operand tiling for 16-bit elements: 8-row x 16-byte core matrices hold 8 x 8 elements; core matrix
+// (row/8, k/8) sits at ((row/8) * KD/8 + k/8) * 128 bytes, so one K = 16 MMA step reads 256 bytes of it
+// (leading byte offset 128) and 8-row groups are KD/8 * 128 bytes apart (stride byte offset).
+__device__ __forceinline__ uint32_t cm_off16(int r, int k, int KD) {
+    return ((uint32_t)((r >> 3) * (KD >> 3) + (k >> 3)) << 7) + ((uint32_t)(r & 7) << 4) + ((uint32_t)(k & 7) << 1);
+}
+
+// Shared-memory matrix descriptor with a leading byte offset `lbo` (the distance between K-adjacent
+// core matrices; a multiple of 16), stride byte offset `sbo`, descriptor version 1, no swizzle.
+__device__ __forceinline__ uint64_t smem_desc_lbo(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B, fp32 accumulation, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// D[M x N] (+)= A[M x 16*ksteps] * B[N x 16*ksteps]^T, fp16 operands in the tiling of cm_off16.
+__device__ __forceinline__ void gemm_f16(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
+                                         uint32_t b_sbo, uint32_t idesc, int ksteps, bool accumulate) {
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_f16(d_tmem, smem_desc(a_addr + ks * 256u, a_sbo), smem_desc(b_addr + ks * 256u, b_sbo), idesc,
+                (ks > 0 || accumulate) ? 1u : 0u);
+}
+
+// gemm_f16 with a B operand whose K-adjacent core matrices are `b_lbo` bytes apart (a padded tiling:
+// with b_lbo = 144 the eight rows of a core matrix and the next core matrix along K fall in different
+// banks, so stores of one column by 32 consecutive K indices do not conflict).
+__device__ __forceinline__ void gemm_f16_bpad(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
+                                              uint32_t b_lbo, uint32_t b_sbo, uint32_t idesc, int ksteps,
+                                              bool accumulate) {
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_f16(d_tmem, smem_desc(a_addr + ks * 256u, a_sbo), smem_desc_lbo(b_addr + ks * 2u * b_lbo, b_lbo, b_sbo),
+                idesc, (ks > 0 || accumulate) ? 1u : 0u);
+}
+
+// 2^e as a float, for -126 <= e <= 127 (exact).
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// The power-of-two exponent e with max_abs * 2^-e in [2^13, 2^14): operands scaled by 2^-e keep fp16's
+// 10 mantissa bits and stay four times below its largest finite value.  0 for a zero or NaN bound, the
+// upper clamp for an infinite one; the result is clamped to [-100, 100] so that 2^e, 2^-e and the
+// product of two such factors with a small power of two are normal floats.
+__device__ __forceinline__ int fp16_scale_exponent(float max_abs) {
+    if (!(max_abs > 0.f)) return 0;
+    if (!(max_abs < 3.0e38f)) return 100;
+    // IEEE single: a normal value with biased exponent b lies in [2^(b-127), 2^(b-126))
+    const int b = (int)((__float_as_uint(max_abs) >> 23) & 0xFFu);
+    const int e = (b == 0 ? -126 : b - 126) - 14;
+    return e < -100 ? -100 : (e > 100 ? 100 : e);
+}
+
+// Round two floats to fp16 (nearest, ties to even) and pack them, the first in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Unpack two fp16 values (low half first) to floats.
+__device__ __forceinline__ void f16x2_to_f32(uint32_t x, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}" : "=f"(lo), "=f"(hi) : "r"(x));
+}
+
+__device__ __forceinline__ uint16_t to_f16_bits(float x) {
+    uint16_t r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+
+// Warp-wide maximum of non-negative floats (their bit patterns order like unsigned integers).
+__device__ __forceinline__ float warp_max_nonneg(float x) {
+    return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(x)));
+}
+
+// Barrier over `nthreads` threads (whole warps) that use the same id; id 0 is __syncthreads.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
 }

@@ -113,13 +113,13 @@ def test_read_status_rejects_null():
 
 
 def test_workspace_size_two_pass_records():
-    # K = V = 128, chunk 64: the status block plus one 149504-byte record per chunk per (b, hv)
+    # K = V = 128, chunk 64: the status block plus one 115712-byte record per chunk per (b, hv)
     B, T, HV = 2, 1000, 8
     nc = (T + 63) // 64
-    assert kda.workspace_size(B, T, 4, HV, 128, 128, 64) == 256 + B * HV * nc * 149504
+    assert kda.workspace_size(B, T, 4, HV, 128, 128, 64) == 256 + B * HV * nc * 115712
     assert kda.workspace_size(B, T, 4, HV, 128, 64, 64) == 256
     assert kda.workspace_size(B, T, 4, HV, 128, 128, 16) == 256
-    assert kda.workspace_size(12, T, 8, 8, 128, 128, 64) == 256 + 12 * 8 * nc * 149504  # 96 pairs
+    assert kda.workspace_size(12, T, 8, 8, 128, 128, 64) == 256 + 12 * 8 * nc * 115712  # 96 pairs
     assert kda.workspace_size(13, T, 8, 8, 128, 128, 64) == 256                          # 104 pairs
 
 
