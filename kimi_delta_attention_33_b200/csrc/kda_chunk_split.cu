@@ -35,8 +35,8 @@
 // the state slice S_c[:, block] lives in registers (thread d owns key row d, exact fp32);
 // per chunk, with fp16(S_c 2^-sig)^T staged in shared memory as a B operand:
 //   chain  D_S = G S_c                     -> S_c+1 = e^{Gam_end} S_c - D_S + KU, in registers
-//   out    D_O = [G rows 64-127; Q'] S_c   -> O = Q' S_c + A U (rows 64-127), read out while the next
-//                                             chunk's chain product runs
+//   out    D_O = Q' S_c (M = 64)           -> O = Q' S_c + A U, read out while the next chunk's chain
+//                                             product runs
 // One tensor-core round trip per chunk is on the chunk-to-chunk path.  The state scale is not reduced over
 // the CTA on the chain: it comes from a bound that all threads compute alike (see chunk_state_kernel).
 // Chunk records stream in by bulk asynchronous copies (mbarrier completion), double-buffered
@@ -126,7 +126,7 @@ struct StateLayout {
     static constexpr uint32_t TBASE = MBAR + 8 * (NBUF + 3);
     static constexpr uint32_t SMX = TBASE + 16;                // [2][8] per-warp max |S|, by chunk parity
     static constexpr uint32_t BYTES = SMX + 64;
-    // D_S = G S (chain); D_O[2] = [G; Q'] S rows 64-127 hold Q' S, by chunk parity
+    // D_S = G S (chain); D_O[2] = Q' S (M = 64, lanes 32 q + 0..15), by chunk parity
     static constexpr int D_S = 0, D_O = VB;
     static constexpr uint32_t NCOL = OUTS ? 3 * VB : VB;
     static constexpr uint32_t TMEM_COLS = NCOL <= 32 ? 32 : NCOL <= 64 ? 64 : NCOL <= 128 ? 128 : NCOL <= 256 ? 256 : 512;
@@ -730,10 +730,10 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t a, uint32_t (&r)[N]) {
 //                from `carry`, where scan_chain_kernel left it (so S_T may alias S0 in both cases).
 //
 // Per chunk c, one tensor-core round trip is on the chain: the issuer issues D_S = G S_c (and, with outputs,
-// D_O = [G; Q'] S_c into the buffer of c's parity) on the S operand of c; every thread waits for D_S and
+// D_O = Q' S_c into the buffer of c's parity) on the S operand of c; every thread waits for D_S and
 // updates its part of the state, S_c+1 = e^{Gam_end} S_c - D_S + KU, writes the next S operand, and meets
-// the others at one barrier.  The outputs of chunk c are read out by lane quarters 2, 3 in step c + 1,
-// before they wait for that step's D_S.
+// the others at one barrier.  The outputs of chunk c are read out in step c + 1, before the state warps
+// wait for that step's D_S.
 //
 // The state operand is fp16(S_c 2^-sig_c).  sig_c comes from a bound on |S_c| that every thread computes
 // alike, with no reduction on the chain: at the start the exact maximum, then
@@ -849,7 +849,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         for (int j = 0; j < HALF; ++j)
             *reinterpret_cast<uint16_t*>(sop + (j >> 3) * Lay::SOP_SBO + (j & 7) * 16) = to_f16_bits(s[j] * f);
     };
-    // outputs of chunk c (lane quarters 2, 3: rows i = d - 64 of D_O), O = Q' S_c 2^(eq + sig_c) + A U
+    // outputs of chunk c: an M = 64 product puts row i in lane 32 (i / 16) + i % 16, so lanes 0-15 of every
+    // state warp read 16 rows (i = 16 wq + lane), O = Q' S_c 2^(eq + sig_c) + A U
     uint32_t ph_out = 0;
     auto outputs = [&](int c, float f_q) -> bool {
         const int par = (c - c_begin) & 1;
@@ -857,7 +858,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         fence_after_sync();
         if (!ok) return false;
         ph_out ^= 1u << par;
-        const int i = d - 64, n = min(CH, T - c * CH);
+        const int i = 16 * wq + lane, n = lane < 16 ? min(CH, T - c * CH) : 0;
         const float* sAU = reinterpret_cast<const float*>(smem + Lay::slot(slot_of(c)) + Lay::AU_OFF);
         constexpr int SUB = HALF < 16 ? HALF : 16;
 #pragma unroll
@@ -907,9 +908,9 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
             gemm_f16_bpad(tmem + Lay::D_S, sl, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO, idesc_f16(128, VB),
                           KD / 16, false);
             mma_commit(bar_chain);  // before the output product: the chain waits for G S alone
-            if (OUTS) {  // rows 64-191 of [G; Q']: D_O rows 64-127 hold Q' S
-                gemm_f16_bpad(tmem + Lay::D_O + par * VB, sl + 16384, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO,
-                              idesc_f16(128, VB), KD / 16, false);
+            if (OUTS) {  // M = 64 on the Q' rows: row i of D_O = Q' S sits in TMEM lane 32 (i / 16) + i % 16
+                gemm_f16_bpad(tmem + Lay::D_O + par * VB, sl + Rec::QP_OFF, KD / 8 * 128, sop, Lay::SOP_LBO,
+                              Lay::SOP_SBO, idesc_f16(64, VB), KD / 16, false);
                 mma_commit(bar_out0 + 8 * par);
             }
         }
@@ -926,7 +927,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         const int sig_next = fp16_scale_exponent(egmax * mS + 256.f * exp2i(14 + e_g) * mS +
                                                  (use_u ? 2.f * exp2i(14 + e_u) : 0.f));
         // ---- the previous chunk's outputs, while D_S runs -------------------------------------------
-        if (OUTS && state_warp && wq >= 2 && c > c_begin) ok = outputs(c - 1, fq_prev) && ok;
+        if (OUTS && state_warp && c > c_begin) ok = outputs(c - 1, fq_prev) && ok;
         // ---- state: S = e^{Gam_end} S - G S + KU ------------------------------------------------------
         const unsigned char* sKU = smem + Lay::slot(k) + Lay::KU_OFF;
         constexpr int PIECE = HALF < 32 ? HALF : 32;
@@ -976,7 +977,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         if (loader && c + 2 < c_end) load_rec(c + 2);  // into the slot of chunk c - 1 (outputs) or c (no outputs)
         fq_prev = fq;
     }
-    if (OUTS && !aborted && state_warp && wq >= 2 && c_end > c_begin) aborted = !outputs(c_end - 1, fq_prev);
+    if (OUTS && !aborted && state_warp && c_end > c_begin) aborted = !outputs(c_end - 1, fq_prev);
     aborted = __syncthreads_or(aborted) != 0;
 
     if (aborted) {

@@ -53,20 +53,26 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
+// The products below build each shared-memory descriptor once and step it along K by adding to its
+// start-address field (address / 16 in bits 0-13: shared memory stays below 256 KB, so the field does not
+// carry): the issuing thread then spends a few instructions per MMA, not a descriptor build.
+
 // D[M x N] (+)= A_tmem[M x 8*ksteps] * B[N x 8*ksteps]^T: one K = 8 step per 8 TMEM columns of A.
 __device__ __forceinline__ void gemm_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, uint32_t b_sbo,
                                              uint32_t idesc, int ksteps, bool accumulate) {
+    const uint64_t b0 = smem_desc(b_addr, b_sbo);
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks)
-        mma_tf32_ts(d_tmem, a_tmem + 8u * ks, smem_desc(b_addr + ks * 256u, b_sbo), idesc,
-                    (ks > 0 || accumulate) ? 1u : 0u);
+        mma_tf32_ts(d_tmem, a_tmem + 8u * ks, b0 + (uint64_t)(16 * ks), idesc, (ks > 0 || accumulate) ? 1u : 0u);
 }
 
 // D[M x N] (+)= A[M x 8*ksteps] * B[N x 8*ksteps]^T, operands in the tiling above.
 __device__ __forceinline__ void gemm_tf32(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
                                           uint32_t b_sbo, uint32_t idesc, int ksteps, bool accumulate) {
+    const uint64_t a0 = smem_desc(a_addr, a_sbo), b0 = smem_desc(b_addr, b_sbo);
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks)
-        mma_tf32(d_tmem, smem_desc(a_addr + ks * 256u, a_sbo), smem_desc(b_addr + ks * 256u, b_sbo), idesc,
-                 (ks > 0 || accumulate) ? 1u : 0u);
+        mma_tf32(d_tmem, a0 + (uint64_t)(16 * ks), b0 + (uint64_t)(16 * ks), idesc, (ks > 0 || accumulate) ? 1u : 0u);
 }
 
 // ---- kind::f16 with fp16 operands (both A and B fp16), fp32 accumulation ----------------------------
@@ -99,9 +105,10 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
 // D[M x N] (+)= A[M x 16*ksteps] * B[N x 16*ksteps]^T, fp16 operands in the tiling of cm_off16.
 __device__ __forceinline__ void gemm_f16(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
                                          uint32_t b_sbo, uint32_t idesc, int ksteps, bool accumulate) {
+    const uint64_t a0 = smem_desc(a_addr, a_sbo), b0 = smem_desc(b_addr, b_sbo);
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks)
-        mma_f16(d_tmem, smem_desc(a_addr + ks * 256u, a_sbo), smem_desc(b_addr + ks * 256u, b_sbo), idesc,
-                (ks > 0 || accumulate) ? 1u : 0u);
+        mma_f16(d_tmem, a0 + (uint64_t)(16 * ks), b0 + (uint64_t)(16 * ks), idesc, (ks > 0 || accumulate) ? 1u : 0u);
 }
 
 // gemm_f16 with a B operand whose K-adjacent core matrices are `b_lbo` bytes apart (a padded tiling:
@@ -110,9 +117,11 @@ __device__ __forceinline__ void gemm_f16(uint32_t d_tmem, uint32_t a_addr, uint3
 __device__ __forceinline__ void gemm_f16_bpad(uint32_t d_tmem, uint32_t a_addr, uint32_t a_sbo, uint32_t b_addr,
                                               uint32_t b_lbo, uint32_t b_sbo, uint32_t idesc, int ksteps,
                                               bool accumulate) {
+    const uint64_t a0 = smem_desc(a_addr, a_sbo), b0 = smem_desc_lbo(b_addr, b_lbo, b_sbo);
+    const uint64_t b_step = (2u * b_lbo) >> 4;
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks)
-        mma_f16(d_tmem, smem_desc(a_addr + ks * 256u, a_sbo), smem_desc_lbo(b_addr + ks * 2u * b_lbo, b_lbo, b_sbo),
-                idesc, (ks > 0 || accumulate) ? 1u : 0u);
+        mma_f16(d_tmem, a0 + (uint64_t)(16 * ks), b0 + b_step * (uint64_t)ks, idesc, (ks > 0 || accumulate) ? 1u : 0u);
 }
 
 // 2^e as a float, for -126 <= e <= 127 (exact).
