@@ -53,14 +53,15 @@ using bf16 = __nv_bfloat16;
 namespace {
 using namespace c64;
 
-// Per-chunk record in the workspace (bytes).  Value-column blocks of 16 (KU, AU) let a state CTA read
-// its columns with one contiguous copy per block.
+// Per-chunk record in the workspace (bytes).  KU and AU are stored as 16-byte chunks of consecutive value
+// columns, rows contiguous within a chunk column: a block of 16 value columns is one contiguous 4 KB range
+// (one copy per block), and 16-byte accesses by consecutive rows touch consecutive banks.
 struct Rec {
     static constexpr uint32_t WQ = 0;          // [192][128] fp16 tiles: G 2^-eg (rows 0-127), Q' 2^-eq (rows 128-191)
     static constexpr uint32_t WQ_BYTES = 49152;
     static constexpr uint32_t QP_OFF = 32768;  // row 128 of WQ
-    static constexpr uint32_t KU = 49152;      // fp16 [8][128][16]: KU 2^-eu by blocks of 16 value columns
-    static constexpr uint32_t AU = 81920;      // fp32 [8][64][16]: A U by blocks of 16 value columns
+    static constexpr uint32_t KU = 49152;      // fp16 [16][128][8]: KU 2^-eu, 8 value columns per row chunk
+    static constexpr uint32_t AU = 81920;      // fp32 [32][64][4]: A U, 4 value columns per row chunk
     static constexpr uint32_t VEC = 114688;    // [128] fp32 e^{Gam_end}, then the scale block at SCL
     static constexpr uint32_t SCL = VEC + 512; // int eg, eq, eu; float max e^{Gam_end}
     static constexpr uint32_t VEC_LOAD = 528;  // bytes of VEC the state pass reads
@@ -625,12 +626,12 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         *reinterpret_cast<uint4*>(smem + L::KA + cm_off16(d, 64 * wc + 32 * h + 8 * c, KD)) = w[c];
-                } else {    // KU row d, value columns v = 64 (wc - 2) + 32 h + 8 c: blocks of 16 columns
+                } else {    // KU row d, value columns v = 64 (wc - 2) + 32 h + 8 c
                     const int v0 = 64 * (wc - 2) + 32 * h;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int v = v0 + 8 * c;
-                        *reinterpret_cast<uint4*>(smem + L::CK + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2) = w[c];
+                        *reinterpret_cast<uint4*>(smem + L::CK + ((v >> 3) * KD + d) * 16) = w[c];
                     }
                 }
             }
@@ -654,7 +655,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
                             const int v = v0 + 4 * c;
-                            *reinterpret_cast<uint4*>(smem + L::VT + (((v >> 4) * 64 + i) * 16 + (v & 15)) * 4) =
+                            *reinterpret_cast<uint4*>(smem + L::VT + ((v >> 2) * 64 + i) * 16) =
                                 make_uint4(r[4 * c] ^ 0x80000000u, r[4 * c + 1] ^ 0x80000000u, r[4 * c + 2] ^ 0x80000000u,
                                            r[4 * c + 3] ^ 0x80000000u);
                         }
@@ -871,8 +872,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
 #pragma unroll
                 for (int j = 0; j < SUB; j += 8) {
                     const int v = c0 + j0 + j;  // column within the block; AU by blocks of 16 columns
-                    const float4 a0 = *reinterpret_cast<const float4*>(sAU + ((v >> 4) * 64 + i) * 16 + (v & 15));
-                    const float4 a1 = *reinterpret_cast<const float4*>(sAU + ((v >> 4) * 64 + i) * 16 + (v & 15) + 4);
+                    const float4 a0 = *reinterpret_cast<const float4*>(sAU + ((v >> 2) * 64 + i) * 4);
+                    const float4 a1 = *reinterpret_cast<const float4*>(sAU + (((v >> 2) + 1) * 64 + i) * 4);
                     const float au[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                     uint32_t w[4];
 #pragma unroll
@@ -935,7 +936,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
 #pragma unroll
         for (int j = 0; j < PIECE; j += 8) {
             const int v = c0 + j;
-            ku_first[j / 8] = use_u && state_warp ? *reinterpret_cast<const uint4*>(sKU + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2)
+            ku_first[j / 8] = use_u && state_warp ? *reinterpret_cast<const uint4*>(sKU + ((v >> 3) * KD + d) * 16)
                                                    : make_uint4(0u, 0u, 0u, 0u);
         }
         if (state_warp) ok = mbar_wait(bar_chain, ph_chain, WAIT_POLLS) && ok;
@@ -953,7 +954,7 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
                     if (use_u) {
                         const int v = c0 + j0 + j;
                         const uint4 u4 = j0 == 0 ? ku_first[j / 8]
-                                                 : *reinterpret_cast<const uint4*>(sKU + (((v >> 4) * KD + d) * 16 + (v & 15)) * 2);
+                                                 : *reinterpret_cast<const uint4*>(sKU + ((v >> 3) * KD + d) * 16);
                         f16x2_to_f32(u4.x, ku[0], ku[1]);
                         f16x2_to_f32(u4.y, ku[2], ku[3]);
                         f16x2_to_f32(u4.z, ku[4], ku[5]);
