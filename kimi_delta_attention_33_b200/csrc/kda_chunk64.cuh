@@ -218,5 +218,72 @@ __device__ __forceinline__ void tri_inverse_step32(float* sRT, float* sX, int ti
     __syncthreads();
 }
 
+// The same last doubling step, writing its lower-left entries straight into Tb = T diag(beta), a [64][64]
+// tf32 operand tile in the tiling of cm_off (tb: its shared-memory base), instead of back into sRT.  The
+// other entries of Tb (the diagonal blocks, final after step 16 -> 32, and the zero upper-right block)
+// are written by tb_outside_lower_left, before this; the caller's barrier completes Tb.
+__device__ __forceinline__ void tri_inverse_step32_tb(const float* sRT, float* sX, int tid, const float* sBeta,
+                                                      unsigned char* tb) {
+    const int r = tid >> 4, c = tid & 15;
+    const float* Crow = sRT + (32 + r) * RP;
+    float acc0 = Crow[c], acc1 = Crow[c + 16];
+#pragma unroll
+    for (int m4 = 0; m4 < 32; m4 += 4) {
+        const float4 cr = *reinterpret_cast<const float4*>(Crow + m4);
+        const float cm[4] = {cr.x, cr.y, cr.z, cr.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int m = m4 + t;
+            if (m > c) acc0 += cm[t] * sRT[m * RP + c];
+            if (m4 >= 16 && m > c + 16) acc1 += cm[t] * sRT[m * RP + c + 16];
+        }
+    }
+    sX[r * 32 + c] = acc0;
+    sX[r * 32 + c + 16] = acc1;
+    __syncthreads();
+    const float* Drow = sRT + (32 + r) * RP + 32;
+    acc0 = sX[r * 32 + c];
+    acc1 = sX[r * 32 + c + 16];
+    const int rmax = 2 * (tid >> 5) + 1;  // largest row of this warp: rows m < r <= rmax contribute
+#pragma unroll
+    for (int m4 = 0; m4 < 32; m4 += 4) {
+        if (m4 >= rmax) break;  // warp-uniform
+        const float4 dr = *reinterpret_cast<const float4*>(Drow + m4);
+        const float dm[4] = {dr.x, dr.y, dr.z, dr.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int m = m4 + t;
+            if (m < r) {
+                acc0 += dm[t] * sX[m * 32 + c];
+                acc1 += dm[t] * sX[m * 32 + c + 16];
+            }
+        }
+    }
+    *reinterpret_cast<uint32_t*>(tb + tc::cm_off(32 + r, c, 64)) = to_tf32(-acc0 * sBeta[c]);
+    *reinterpret_cast<uint32_t*>(tb + tc::cm_off(32 + r, c + 16, 64)) = to_tf32(-acc1 * sBeta[c + 16]);
+}
+
+// Tb entries outside the lower-left 32 x 32 block, from T after step 16 -> 32: the two diagonal blocks (strictly
+// lower part from sRT, unit diagonal, zeros above) and the zero upper-right block.  Units of four columns.
+__device__ __forceinline__ void tb_outside_lower_left(const float* sRT, int tid, const float* sBeta, unsigned char* tb) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int u = tid + INV_THREADS * x;
+        const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
+        if (i >= 32 && j4 < 8) continue;  // the lower-left block: step 32 -> 64 writes it
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if ((i >> 5) == (j4 >> 3)) {  // a diagonal block
+            const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
+            const float tr[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int j = 4 * j4 + t;
+                w[t] = to_tf32(((j < i) ? tr[t] : (j == i ? 1.f : 0.f)) * sBeta[j]);
+            }
+        }
+        *reinterpret_cast<uint4*>(tb + tc::cm_off(i, 4 * j4, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 }  // namespace c64
 }  // namespace kda

@@ -137,8 +137,8 @@ struct StateLayout {
 
 
 constexpr int STATE_WARPS = 8;                         // warps that own the state slice
-constexpr int STATE_THREADS = 32 * (STATE_WARPS + 1);  // and one that issues the copies and the products
-constexpr int ISSUER = 32 * STATE_WARPS;
+constexpr int STATE_THREADS = 32 * (STATE_WARPS + 2);  // and two that issue the chain and the output products
+constexpr int ISSUER = 32 * STATE_WARPS, OUT_ISSUER = ISSUER + 32;
 constexpr int PREP_THREADS = 512;
 static_assert(PREP_THREADS == INV_THREADS, "the triangular inverse assumes 512 threads");
 
@@ -519,23 +519,10 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
         // ---- T = (I + R)^{-1} in place; Tb = T diag(beta) -> KA rows 128-191 --------------------------
         tri_inverse_diag16(sRT, sX, tid);
         tri_inverse_step16(sRT, sX, tid);
-        tri_inverse_step32(sRT, sX, tid);
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const int u = tid + NT * x;
-            const int i = ((u >> 7) << 3) + (u & 7), j4 = (u >> 3) & 15;
-            uint32_t w[4];
-            const float4 t4 = *reinterpret_cast<const float4*>(sRT + i * RP + 4 * j4);
-            const float tr[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int j = 4 * j4 + t;
-                const float tv = (j < i) ? tr[t] : (j == i ? 1.f : 0.f);
-                w[t] = to_tf32(tv * sBeta[j]);
-            }
-            const uint4 w4 = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(smem + L::KA + 32768 + cm_off(i, 4 * j4, CH)) = w4;
-        }
+        // Tb = T diag(beta) into KA rows 128-191: the diagonal blocks (final now) while step 32 -> 64 runs, which
+        // writes the lower-left block itself
+        tb_outside_lower_left(sRT, tid, sBeta, smem + L::KA + 32768);
+        tri_inverse_step32_tb(sRT, sX, tid, sBeta, smem + L::KA + 32768);
         if (tid < 64) sSqQ[tid] = sSqK[tid] = 0.0f;  // read for the last time above; the next chunk's sums follow
         fence_proxy_async();
         cta_sync_tc();
@@ -796,8 +783,10 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         pending |= 1u << k;
     };
     // this thread's part of the state slice: key row d, columns vb0 + c0 .. + HALF, exact fp32 (state warps)
-    const bool issuer = tid == ISSUER, state_warp = warp < STATE_WARPS;
-    const bool loader = tid == 0;  // issues the record copies (its warp waits for D_S with time to spare)
+    const bool issuer = tid == ISSUER, out_issuer = tid == OUT_ISSUER, state_warp = warp < STATE_WARPS;
+    // the record copies come from the output issuer: its products are read out a step later, so a copy issued after the
+    // barrier delays nothing on the chain
+    const bool loader = tid == OUT_ISSUER;
     const int d = 32 * wq + lane;
     float s[HALF];
     {
@@ -888,7 +877,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         }
         return true;
     };
-    uint32_t ph_chain = 0;
+    uint32_t ph_chain = 0, out_commits = 0;
+    int last_out_par = -1;
     bool aborted = false;
     if (state_warp) warp_max_s(0);
     __syncthreads();
@@ -905,15 +895,19 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
         bool ok = mbar_wait(bar_rec0 + 8 * k, (ph_rec >> k) & 1u, WAIT_POLLS);
         ph_rec ^= 1u << k;
         if (loader && ok) pending &= ~(1u << k);
+        // two issuing threads on different schedulers: an MMA takes a thread about 100 cycles to issue here, and
+        // the chain's products should not queue behind the output's in one thread
         if (issuer && ok) {
             gemm_f16_bpad(tmem + Lay::D_S, sl, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO, idesc_f16(128, VB),
                           KD / 16, false);
-            mma_commit(bar_chain);  // before the output product: the chain waits for G S alone
-            if (OUTS) {  // M = 64 on the Q' rows: row i of D_O = Q' S sits in TMEM lane 32 (i / 16) + i % 16
-                gemm_f16_bpad(tmem + Lay::D_O + par * VB, sl + Rec::QP_OFF, KD / 8 * 128, sop, Lay::SOP_LBO,
-                              Lay::SOP_SBO, idesc_f16(64, VB), KD / 16, false);
-                mma_commit(bar_out0 + 8 * par);
-            }
+            mma_commit(bar_chain);
+        }
+        if (OUTS && out_issuer && ok) {  // M = 64 on the Q' rows: row i of D_O = Q' S sits in TMEM lane 32 (i / 16) + i % 16
+            gemm_f16_bpad(tmem + Lay::D_O + par * VB, sl + Rec::QP_OFF, KD / 8 * 128, sop, Lay::SOP_LBO, Lay::SOP_SBO,
+                          idesc_f16(64, VB), KD / 16, false);
+            mma_commit(bar_out0 + 8 * par);
+            out_commits += 1u << (16 * par);  // commits per parity, for the drain on abort
+            last_out_par = par;
         }
         fence_after_sync();
         const unsigned char* vec = smem + Lay::slot(k) + Lay::VEC_OFF;
@@ -989,6 +983,8 @@ chunk_state_kernel(const unsigned char* __restrict__ rec_base, const float* __re
                 if (pending & (1u << bb)) mbar_wait(bar_rec0 + 8 * bb, (ph_rec >> bb) & 1u, WAIT_POLLS);
         }
         if (issuer) mbar_wait(bar_chain, ph_chain, WAIT_POLLS);
+        if (OUTS && out_issuer && last_out_par >= 0)  // the output products: their last commit tracks them all
+            mbar_wait(bar_out0 + 8 * last_out_par, ((out_commits >> (16 * last_out_par)) - 1u) & 1u, WAIT_POLLS);
     } else if (state_warp) {
         float* dst = nullptr;
         if (!OUTS) dst = carry_slot(seg, half);
