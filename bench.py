@@ -419,6 +419,26 @@ def run_mla_only(args, ws, rank, local):
                           "gpu_launches": args.steps * 3}), flush=True)
 
 
+def measure_fallbacks(dev, kda, hbm_peak, peak_kind, steps=20):
+    """The paths outside the two tensor-core schedules, timed on workload 2's sizes: the CUDA-core kernel
+    (value/key width 64, and chunk 16, both bf16) and the two-pass schedule with every chunk on the exact
+    decay path (dt_bias far positive: every gate value near the lower bound, so the in-chunk decay span
+    exceeds the factorised operands' limit)."""
+    w2 = WORKLOADS[2]
+    cases = {"cuda_core_K64_V64": w2.scaled(K=64, V=64), "cuda_core_chunk16": w2.scaled(chunk=16),
+             "two_pass_exact_decay_path": w2.scaled(dt_bias_mean=6.0, dt_bias_std=0.0)}
+    out = {}
+    for name, w in cases.items():
+        pf = Prefill(w, rank_seed(w, 0), dev, kda)
+        v, mps, r = pf.measure(steps, 3, 1, None, hbm_peak, peak_kind)
+        out[name] = {"sizes": f"B{w.B} T{w.T} H{w.H} HV{w.HV} K{w.K} V{w.V} C{w.chunk}", "schedule": r["schedule"],
+                     "ms_per_step": round(mps, 5), "tokens_per_s": round(v, 1), "roofline_frac": r["frac"],
+                     "kernel_file": r["kernel_file"]}
+        del pf
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, ws, rank, local):
     from kimi_delta_attention_33_b200 import kda
     if args.workload == 6:
@@ -481,6 +501,8 @@ def run_ours(args, ws, rank, local):
         extras["mla_decode"] = measure_mla(dev, kda, hbm_peak, peak_kind, measured_peaks()[1])
         torch.cuda.empty_cache()
         extras["backward"] = measure_backward(dev, kda, hbm_peak, peak_kind)
+        torch.cuda.empty_cache()
+        extras["fallbacks"] = measure_fallbacks(dev, kda, hbm_peak, peak_kind)
         line.update(extras)
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(w) if (ws == 1 and not args.no_cpu_baseline) else None
@@ -566,7 +588,9 @@ def run_e2e(args, w, x, dev, kda):
     d2h = sum(t.numel() * t.element_size() for t in results_host[0])
     return {"value": round(units / sec, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": n, "overlap": "inputs of step i+1 and results of step i-1 "
-            "copy while step i runs (two buffer sets, three streams)"}
+            "copy while step i runs (two buffer sets, three streams)",
+            # the host link's rates over the timed steps: at a PCIe link's rate the call is copy-bound
+            "h2d_GBps": round(h2d / sec / 1e9, 1), "d2h_GBps": round(d2h / sec / 1e9, 1)}
 
 
 # ------------------------------------------------------------------------ CPU oracle legs -----
