@@ -7,12 +7,12 @@
 //   3. o_lat = softmax(scale score) . c    [B, H, r]
 //   4. o     = o_lat . W_UV^T              [B, H, d_v]    (W_UV [H, d_v, r])
 // (the K3 MLA layer: global softmax attention without positional encoding).  Three kernels:
-//   mla_qabs_kernel    step 1 on the CUDA cores; q_abs is kept as two bf16 terms, hi + lo, so that the
-//                      tensor-core scores carry about 16 mantissa bits of it;
+//   mla_qabs_kernel    step 1 with bf16 tensor-core MMAs; q_abs is kept as two bf16 terms, hi + lo, so that
+//                      the tensor-core scores carry about 16 mantissa bits of it;
 //   mla_attend_kernel  steps 2-3 with bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation):
 //                      one CTA per (sequence, group of 48 heads, split of the positions) streams its
 //                      latent tiles once through shared memory, with an online softmax;
-//   mla_out_kernel     merges the splits and applies step 4 on the CUDA cores.
+//   mla_out_kernel     merges the splits and applies step 4 with bf16 MMAs on the hi + lo terms of o_lat.
 // Every head reads the same latent vectors, so the CTA covers as many heads as its registers allow and
 // the cache crosses HBM once per head group.
 #include "kda_common.cuh"
@@ -75,42 +75,77 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
 }  // namespace
 
 // ---- step 1: q_abs = q W_UK per head, as bf16 hi + lo ------------------------------------------
-// Grid (H, R / 128, ceil(B / 32)); thread = one latent column, 32 sequences per CTA, so W_UK is read
-// ceil(B / 32) times; four key channels per step with the sequences' q values as float4.
+// Grid (H, ceil(B / 32)), 256 threads.  q (32 sequences x DQ) and W_UK[h] (DQ x R) go to shared memory by
+// 16-byte cp.async; the product runs on bf16 MMAs (m16n8k16, fp32 accumulation; both operands are bf16,
+// so the sums are those of the CUDA-core product up to their order).  Warp w: sequences 16 (w % 2) ..,
+// latent columns (w / 2) R / 4 ..; W_UK's rows are k, so its B fragments come from transposing loads.
 constexpr int QABS_B = 32;
+constexpr int PROJ_THREADS = 256;
 
 template <int DQ, int R>
-__global__ void __launch_bounds__(128)
+struct QabsSmem {
+    static constexpr int PQ = DQ + 8, PW = R + 8;  // row pitches (bf16): conflict-free fragment loads
+    static constexpr size_t SQ = 0, SW = SQ + (size_t)QABS_B * PQ * 2;
+    static constexpr size_t BYTES = SW + (size_t)DQ * PW * 2;
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+template <int DQ, int R>
+__global__ void __launch_bounds__(PROJ_THREADS)
 mla_qabs_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_UK, int B, int H, bf16* __restrict__ qa_hi,
                 bf16* __restrict__ qa_lo) {
-    __shared__ __align__(16) float sq[QABS_B][DQ];
-    const int h = blockIdx.x, col = blockIdx.y * 128 + threadIdx.x, b0 = blockIdx.z * QABS_B;
-    for (int i = threadIdx.x; i < QABS_B * DQ; i += 128) {
-        const int bb = i / DQ, d = i - bb * DQ;
-        sq[bb][d] = (b0 + bb < B) ? __bfloat162float(q[((size_t)(b0 + bb) * H + h) * DQ + d]) : 0.f;
+    using Sm = QabsSmem<DQ, R>;
+    constexpr int PQ = Sm::PQ, PW = Sm::PW, NT8 = R / 4 / 8;  // n8 tiles per warp
+    extern __shared__ __align__(16) unsigned char qsm[];
+    const uint32_t sq = (uint32_t)__cvta_generic_to_shared(qsm + Sm::SQ), sw = (uint32_t)__cvta_generic_to_shared(qsm + Sm::SW);
+    const int h = blockIdx.x, b0 = blockIdx.y * QABS_B, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < QABS_B * (DQ / 8); i += PROJ_THREADS) {  // rows past B read as zeros
+        const int bb = i / (DQ / 8), ch = i - bb * (DQ / 8);
+        const bool ok = b0 + bb < B;
+        cp_async16_zfill(sq + (uint32_t)((bb * PQ + 8 * ch) * 2),
+                         ok ? (const void*)(q + ((size_t)(b0 + bb) * H + h) * DQ + 8 * ch) : (const void*)q, ok);
     }
+    const bf16* w = W_UK + (size_t)h * DQ * R;
+    for (int i = tid; i < DQ * (R / 8); i += PROJ_THREADS) {
+        const int d = i / (R / 8), ch = i - d * (R / 8);
+        cp_async16_zfill(sw + (uint32_t)((d * PW + 8 * ch) * 2), w + (size_t)d * R + 8 * ch, true);
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
-    float acc[QABS_B];
+    const int mt = warp & 1, n0 = (warp >> 1) * (R / 4), g = lane >> 2, t4 = lane & 3;
+    float acc[NT8][4];
 #pragma unroll
-    for (int bb = 0; bb < QABS_B; ++bb) acc[bb] = 0.f;
-    const bf16* w = W_UK + (size_t)h * DQ * R + col;
-#pragma unroll 1
-    for (int d = 0; d < DQ; d += 4) {
-        const float w0 = __bfloat162float(w[(size_t)d * R]), w1 = __bfloat162float(w[(size_t)(d + 1) * R]);
-        const float w2 = __bfloat162float(w[(size_t)(d + 2) * R]), w3 = __bfloat162float(w[(size_t)(d + 3) * R]);
+    for (int j = 0; j < NT8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    const uint32_t a_off = (uint32_t)(((16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * PQ + 8 * (lane >> 4)) * 2);
+    const uint32_t b_off = (uint32_t)(((lane & 15) * PW + n0) * 2);  // rows k0 + (lane % 16) of [k][n]
 #pragma unroll
-        for (int bb = 0; bb < QABS_B; ++bb) {
-            const float4 qv = *reinterpret_cast<const float4*>(&sq[bb][d]);
-            acc[bb] = fmaf(qv.x, w0, fmaf(qv.y, w1, fmaf(qv.z, w2, fmaf(qv.w, w3, acc[bb]))));
+    for (int k = 0; k < DQ; k += 16) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(a0, a1, a2, a3, sq + a_off + (uint32_t)(k * 2));
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+            uint32_t b0f, b1f;
+            ldmatrix_x2_trans(b0f, b1f, sw + b_off + (uint32_t)((k * PW + 8 * j) * 2));
+            mma_bf16(acc[j], a0, a1, a2, a3, b0f, b1f);
         }
     }
+    // D fragment: rows 16 mt + g (+ 8), columns n0 + 8 j + 2 t4 (+ 1)
 #pragma unroll
-    for (int bb = 0; bb < QABS_B; ++bb) {
-        if (b0 + bb >= B) break;
-        const bf16 hi = __float2bfloat16_rn(acc[bb]);
-        const size_t idx = ((size_t)(b0 + bb) * H + h) * R + col;
-        qa_hi[idx] = hi;
-        qa_lo[idx] = __float2bfloat16_rn(acc[bb] - __bfloat162float(hi));
+    for (int half = 0; half < 2; ++half) {
+        const int b = b0 + 16 * mt + g + 8 * half;
+        if (b >= B) continue;
+        const size_t row = ((size_t)b * H + h) * R;
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+            const float x0 = acc[j][2 * half], x1 = acc[j][2 * half + 1];
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(hi);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+            const int col = n0 + 8 * j + 2 * t4;
+            *reinterpret_cast<__nv_bfloat162*>(qa_hi + row + col) = hi;
+            *reinterpret_cast<__nv_bfloat162*>(qa_lo + row + col) = lo;
+        }
     }
 }
 
@@ -195,7 +230,6 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
             asm volatile("cp.async.wait_group 0;\n" ::: "memory");
         }
         __syncthreads();  // this tile has landed for every thread
-        const bf16* cT = sC + buf * MLA_TP * P;
         // ---- partial scores: 16 heads x 32 positions over this warp's quarter of the latent columns,
         //      (q_hi + q_lo) . c with bf16 MMAs ----------------------------------------------------------
         {
@@ -345,97 +379,105 @@ mla_attend_kernel(const bf16* __restrict__ qa_hi, const bf16* __restrict__ qa_lo
 }
 
 // ---- merge the splits and step 4: o = (o_lat / l) W_UV^T ---------------------------------------
-// Grid (H, ceil(B / 32)); 256 threads.  The merged o_lat of 32 sequences goes to shared memory (dynamic);
-// W_UV[h] passes through shared memory in 32-column tiles loaded 16 bytes at a time, so it is read
-// ceil(B / 32) times.  Thread (v, part) accumulates the 32 sequences' outputs for value column v over its
-// part of each tile (float4 reads), and the parts are summed at the end.
+// Grid (H, ceil(B / 32)), 256 threads.  The merged o_lat of 32 sequences is split into bf16 hi + lo terms
+// (about 16 mantissa bits) in shared memory; W_UV[h] (DV x R, rows v, k contiguous) arrives by 16-byte
+// cp.async while the merge runs.  o = (hi + lo) W_UV^T on bf16 MMAs (m16n8k16, fp32 accumulation).
+// Warp w: sequences 16 (w % 2) .., value columns (w / 2) DV / 4 ...
 constexpr int OUT_B = 32;
 
 template <int DV, int R>
 struct MlaOutSmem {
-    static constexpr int PARTS = 256 / DV;
-    static constexpr size_t SO = 0;                                    // [32][R] fp32 merged o_lat
-    static constexpr size_t SW = SO + (size_t)OUT_B * R * 4;           // [DV][36] fp32 W tile
-    static constexpr size_t SR = SW + (size_t)DV * 36 * 4;             // [PARTS - 1][DV][32] partial sums
-    static constexpr size_t BYTES = SR + (size_t)(PARTS > 1 ? PARTS - 1 : 1) * DV * OUT_B * 4;
+    static constexpr int PA = R + 8;  // row pitch (bf16) of the o_lat terms and of W_UV
+    static constexpr size_t SH = 0, SL = SH + (size_t)OUT_B * PA * 2, SW = SL + (size_t)OUT_B * PA * 2;
+    static constexpr size_t BYTES = SW + (size_t)DV * PA * 2;
+    static_assert(BYTES <= 232448, "shared memory budget");
 };
 
 template <int DV, int R>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(PROJ_THREADS)
 mla_out_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, const bf16* __restrict__ W_UV,
                int B, int H, int nsplit, bf16* __restrict__ o) {
     using Sm = MlaOutSmem<DV, R>;
-    constexpr int PARTS = Sm::PARTS, KPT = 32 / PARTS;  // parts of each tile, columns per part
+    constexpr int PA = Sm::PA, NT8 = DV / 4 / 8;  // n8 tiles per warp
     extern __shared__ __align__(16) unsigned char osm[];
-    float (*so)[R] = reinterpret_cast<float (*)[R]>(osm + Sm::SO);
-    float (*sw)[36] = reinterpret_cast<float (*)[36]>(osm + Sm::SW);  // pitch 36: conflict-free float4 reads
-    float* sred = reinterpret_cast<float*>(osm + Sm::SR);
-    const int h = blockIdx.x, b0 = blockIdx.y * OUT_B, tid = threadIdx.x;
-    // merge: o_lat = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s
-    for (int i = tid; i < OUT_B * R; i += 256) {
-        const int bb = i / R, col = i - bb * R, b = b0 + bb;
-        float val = 0.f;
+    bf16* sH = reinterpret_cast<bf16*>(osm + Sm::SH);
+    bf16* sL = reinterpret_cast<bf16*>(osm + Sm::SL);
+    const uint32_t sh = (uint32_t)__cvta_generic_to_shared(sH), sl = (uint32_t)__cvta_generic_to_shared(sL);
+    const uint32_t sw = (uint32_t)__cvta_generic_to_shared(osm + Sm::SW);
+    const int h = blockIdx.x, b0 = blockIdx.y * OUT_B, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bf16* w = W_UV + (size_t)h * DV * R;
+    for (int i = tid; i < DV * (R / 8); i += PROJ_THREADS) {
+        const int v = i / (R / 8), ch = i - v * (R / 8);
+        cp_async16_zfill(sw + (uint32_t)((v * PA + 8 * ch) * 2), w + (size_t)v * R + 8 * ch, true);
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    // merge: o_lat = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s, four columns per item
+    for (int i = tid; i < OUT_B * (R / 4); i += PROJ_THREADS) {
+        const int bb = i / (R / 4), col = 4 * (i - bb * (R / 4)), b = b0 + bb;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
         if (b < B) {
             float M = -INFINITY;
             for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, part_ml[(((size_t)b * nsplit + sp) * H + h) * 2]);
-            float num = 0.f, den = 0.f;
+            float den = 0.f;
             for (int sp = 0; sp < nsplit; ++sp) {
                 const float* ml = part_ml + (((size_t)b * nsplit + sp) * H + h) * 2;
                 if (ml[0] == -INFINITY) continue;  // an empty split
-                const float w = exp2f(ml[0] - M);
-                num += w * part_o[(((size_t)b * nsplit + sp) * H + h) * R + col];
-                den += w * ml[1];
+                const float wt = exp2f(ml[0] - M);
+                const float4 x = *reinterpret_cast<const float4*>(part_o + (((size_t)b * nsplit + sp) * H + h) * R + col);
+                val.x += wt * x.x;
+                val.y += wt * x.y;
+                val.z += wt * x.z;
+                val.w += wt * x.w;
+                den += wt * ml[1];
             }
-            val = num / den;
+            const float inv = 1.f / den;
+            val = make_float4(val.x * inv, val.y * inv, val.z * inv, val.w * inv);
         }
-        so[bb][col] = val;
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(val.x, val.y), h23 = __floats2bfloat162_rn(val.z, val.w);
+        const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(val.x - f01.x, val.y - f01.y);
+        const __nv_bfloat162 l23 = __floats2bfloat162_rn(val.z - f23.x, val.w - f23.y);
+        *reinterpret_cast<uint2*>(sH + bb * PA + col) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+        *reinterpret_cast<uint2*>(sL + bb * PA + col) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
     }
-    const int v = tid % DV, part = tid / DV;
-    float acc[OUT_B];
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();
+    const int mt = warp & 1, n0 = (warp >> 1) * (DV / 4), g = lane >> 2, t4 = lane & 3;
+    float acc[NT8][4];
 #pragma unroll
-    for (int i = 0; i < OUT_B; ++i) acc[i] = 0.f;
-    const bf16* w = W_UV + (size_t)h * DV * R;
-    for (int k0 = 0; k0 < R; k0 += 32) {
-        __syncthreads();  // previous W tile consumed (and o_lat merged, on the first pass)
-        for (int i = tid; i < DV * 4; i += 256) {  // DV rows x 4 chunks of 8 bf16
-            const int vv = i >> 2, ch = i & 3;
-            const uint4 raw = *reinterpret_cast<const uint4*>(w + (size_t)vv * R + k0 + 8 * ch);
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
-            const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
-            *reinterpret_cast<float4*>(&sw[vv][8 * ch]) = make_float4(f0.x, f0.y, f1.x, f1.y);
-            *reinterpret_cast<float4*>(&sw[vv][8 * ch + 4]) = make_float4(f2.x, f2.y, f3.x, f3.y);
+    for (int j = 0; j < NT8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    const uint32_t a_off = (uint32_t)(((16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * PA + 8 * (lane >> 4)) * 2);
+    // B fragment addresses: lane l -> row (value column) n0 + 8 j + (l % 8), column k + 8 (l / 8): two k16 steps
+    const uint32_t b_off = (uint32_t)(((n0 + (lane & 7)) * PA + 8 * (lane >> 3)) * 2);
+#pragma unroll 2
+    for (int k = 0; k < R; k += 32) {
+        uint32_t ah[2][4], al[2][4];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            ldmatrix_x4(ah[h2][0], ah[h2][1], ah[h2][2], ah[h2][3], sh + a_off + (uint32_t)((k + 16 * h2) * 2));
+            ldmatrix_x4(al[h2][0], al[h2][1], al[h2][2], al[h2][3], sl + a_off + (uint32_t)((k + 16 * h2) * 2));
         }
-        __syncthreads();
 #pragma unroll
-        for (int kk = part * KPT; kk < part * KPT + KPT; kk += 4) {
-            const float4 wv = *reinterpret_cast<const float4*>(&sw[v][kk]);
+        for (int j = 0; j < NT8; ++j) {
+            uint32_t bf[4];
+            ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], sw + b_off + (uint32_t)((8 * j * PA + k) * 2));
 #pragma unroll
-            for (int i = 0; i < OUT_B; ++i) {
-                const float4 x = *reinterpret_cast<const float4*>(&so[i][k0 + kk]);
-                acc[i] = fmaf(x.x, wv.x, fmaf(x.y, wv.y, fmaf(x.z, wv.z, fmaf(x.w, wv.w, acc[i]))));
+            for (int h2 = 0; h2 < 2; ++h2) {
+                mma_bf16(acc[j], ah[h2][0], ah[h2][1], ah[h2][2], ah[h2][3], bf[2 * h2], bf[2 * h2 + 1]);
+                mma_bf16(acc[j], al[h2][0], al[h2][1], al[h2][2], al[h2][3], bf[2 * h2], bf[2 * h2 + 1]);
             }
         }
     }
-    if (PARTS > 1) {
-        if (part > 0) {
 #pragma unroll
-            for (int i = 0; i < OUT_B; ++i) sred[((part - 1) * DV + v) * OUT_B + i] = acc[i];
-        }
-        __syncthreads();
-        if (part == 0) {
-            for (int p2 = 0; p2 + 1 < PARTS; ++p2) {
+    for (int half = 0; half < 2; ++half) {
+        const int b = b0 + 16 * mt + g + 8 * half;
+        if (b >= B) continue;
 #pragma unroll
-                for (int i = 0; i < OUT_B; ++i) acc[i] += sred[(p2 * DV + v) * OUT_B + i];
-            }
-        }
-    }
-    if (part == 0) {
-#pragma unroll
-        for (int i = 0; i < OUT_B; ++i) {
-            const int b = b0 + i;
-            if (b < B) o[((size_t)b * H + h) * DV + v] = __float2bfloat16_rn(acc[i]);
-        }
+        for (int j = 0; j < NT8; ++j)
+            *reinterpret_cast<__nv_bfloat162*>(o + ((size_t)b * H + h) * DV + n0 + 8 * j + 2 * t4) =
+                __floats2bfloat162_rn(acc[j][2 * half], acc[j][2 * half + 1]);
     }
 }
 
@@ -467,10 +509,12 @@ cudaError_t launch_mla_t(const MlaArgs& a) {
     float* part_o = reinterpret_cast<float*>(qa_lo + (size_t)a.B * a.H * R);
     float* part_ml = part_o + (size_t)a.B * ns * a.H * R;
     const bf16* q = static_cast<const bf16*>(a.q);
-    mla_qabs_kernel<DQ, R><<<dim3(a.H, R / 128, (a.B + QABS_B - 1) / QABS_B), 128, 0, a.stream>>>(
-        q, static_cast<const bf16*>(a.W_UK), a.B, a.H, qa_hi, qa_lo);
-    cudaError_t e = cudaGetLastError();
+    using QSm = QabsSmem<DQ, R>;
+    cudaError_t e = cudaFuncSetAttribute(mla_qabs_kernel<DQ, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QSm::BYTES);
     if (e != cudaSuccess) return e;
+    mla_qabs_kernel<DQ, R><<<dim3(a.H, (a.B + QABS_B - 1) / QABS_B), PROJ_THREADS, QSm::BYTES, a.stream>>>(
+        q, static_cast<const bf16*>(a.W_UK), a.B, a.H, qa_hi, qa_lo);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     using Sm = MlaSmem<R>;
     e = cudaFuncSetAttribute(mla_attend_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sm::BYTES);
     if (e != cudaSuccess) return e;
@@ -481,7 +525,7 @@ cudaError_t launch_mla_t(const MlaArgs& a) {
     using OSm = MlaOutSmem<DV, R>;
     e = cudaFuncSetAttribute(mla_out_kernel<DV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OSm::BYTES);
     if (e != cudaSuccess) return e;
-    mla_out_kernel<DV, R><<<dim3(a.H, (a.B + OUT_B - 1) / OUT_B), 256, OSm::BYTES, a.stream>>>(
+    mla_out_kernel<DV, R><<<dim3(a.H, (a.B + OUT_B - 1) / OUT_B), PROJ_THREADS, OSm::BYTES, a.stream>>>(
         part_o, part_ml, static_cast<const bf16*>(a.W_UV), a.B, a.H, ns, static_cast<bf16*>(a.o));
     return cudaGetLastError();
 }
