@@ -140,6 +140,21 @@ def test_schedule_choice():
     assert kda.uses_tensor_cores(128, 128, 64) and not kda.uses_tensor_cores(64, 64, 64)
 
 
+def test_split_state_pass_plan():
+    # The state pass splits along the sequence only where the unsplit chains leave the SMs idle: a few (sequence, head)
+    # pairs with long sequences.  The benchmark workloads 2 (16 pairs x 16 chunks) and 4 (32 pairs x 1024 chunks) keep
+    # one chain per value block; 4 pairs x 79 chunks and 1 pair x 94 chunks split (the GPU scan tests' shapes).
+    L = kda.lib
+    def plan(B, T, H, HV):
+        return L.kda_chunk_fwd_schedule(B, T, H, HV, 128, 128, 64, kda.BF16, kda.workspace_size(B, T, H, HV, 128, 128, 64))
+    assert plan(2, 1024, 4, 8) == kda.SCHEDULE_TC_TWO_PASS
+    assert plan(1, 65536, 8, 32) == kda.SCHEDULE_TC_TWO_PASS
+    assert plan(1, 5000, 2, 4) == kda.SCHEDULE_TC_TWO_PASS_SCAN
+    assert plan(1, 6000, 1, 1) == kda.SCHEDULE_TC_TWO_PASS_SCAN
+    assert kda.schedule_launches(1, 5000, 2, 4, 128, 128, 64) == 4   # prep, carry, segment chain, outputs
+    assert kda.schedule_launches(1, 65536, 8, 32, 128, 128, 64) == 2  # prep, state
+
+
 def test_two_pass_limits():
     L = kda.lib
     # token stride (HV x 256 bytes) x T must stay below 2^40 bytes for the prep pass's tensor maps

@@ -65,7 +65,7 @@ def test_ragged_lengths_both_schedules(schedule, T):
     assert rel_err(S, S_ref) <= TOL[w.dtype]
 
 
-# (B, HV) reaching value blocks of 16 (<= 18 pairs), 32 (<= 37 pairs) and 64 columns
+# (B, HV) reaching value blocks of 16 (<= 18 pairs) and 32 columns (more pairs), and the single-pass schedule's counts
 @pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("B,H,HV", [(1, 1, 1), (2, 4, 8), (3, 5, 10), (1, 8, 32), (5, 8, 8), (2, 16, 48), (4, 8, 24)])
 def test_pair_counts_both_schedules(schedule, B, H, HV):
