@@ -21,6 +21,8 @@
 //   1. forward sweep over all tokens, the state saved every CK tokens to the workspace;
 //   2. the blocks of CK tokens in reverse: the block's states recomputed from its checkpoint into
 //      shared memory, then its tokens in reverse order.
+// The per-token inputs of a block (decay, k, q, v, dO, beta) are staged in shared memory once per block
+// by loads that are all in flight together, so a token step does not wait for its own global loads.
 // A second, elementwise kernel chains dg through the gate when the op applied it.
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -40,7 +42,10 @@ struct BwdShape {
     static constexpr int R = K / RPP;                                  // rows per thread
     static constexpr int NW = NT / 32;                                 // warps
     static_assert(NT % 32 == 0 && RPP * R == K && TPR * 4 == VB, "backward shape");
-    static constexpr size_t smem_floats = (size_t)BWD_CK * K * VB + (size_t)BWD_CK * VB + 2 * (size_t)NW * VB;
+    // sPrev [CK][K][VB], sR [CK][VB], sRed 2 x [NW][VB], then the staged block: decay, k, q [CK][K], v, dO [CK][VB],
+    // beta [CK], and dt_bias [K]
+    static constexpr size_t smem_floats = (size_t)BWD_CK * K * VB + (size_t)BWD_CK * VB + 2 * (size_t)NW * VB +
+                                          3 * (size_t)BWD_CK * K + 2 * (size_t)BWD_CK * VB + BWD_CK + K;
     static constexpr size_t smem_bytes = smem_floats * sizeof(float);
 };
 
@@ -93,6 +98,13 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     float* sPrev = bsm;                        // [CK][K][VB] state entering each token of the block
     float* sR = sPrev + BWD_CK * K * VB;       // [CK][VB] residuals
     float* sRed = sR + BWD_CK * VB;            // 2 x [NW][VB] reduction buffers
+    float* sA = sRed + 2 * NW * VB;            // staged block: [CK][K] decay exp(g)
+    float* sK = sA + BWD_CK * K;               //               [CK][K] k
+    float* sQ = sK + BWD_CK * K;               //               [CK][K] q
+    float* sV = sQ + BWD_CK * K;               //               [CK][VB] v (this CTA's columns)
+    float* sDO = sV + BWD_CK * VB;             //               [CK][VB] dO
+    float* sB = sDO + BWD_CK * VB;             //               [CK] beta
+    float* sBias = sB + BWD_CK;                // [K] dt_bias (zeros when absent)
 
     const int vbi = blockIdx.x % NVB, pair = blockIdx.x / NVB;
     const int b = pair / HV, hv = pair - b * HV, h = hv / (HV / H);
@@ -100,23 +112,30 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cg = tid % TPR, rg = tid / TPR;
     const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[hv]) : 0.0f;
-    float bias[R];
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-        bias[i] = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * K + rg + RPP * i] : 0.0f;
+    for (int d = tid; d < K; d += Sh::NT)
+        sBias[d] = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * K + d] : 0.0f;
     const int NCK = (T + BWD_CK - 1) / BWD_CK;
     float* my_ckpt = ckpt + (size_t)blockIdx.x * NCK * K * VB;
     int red = 0;  // which reduction buffer the next reduction uses
 
     auto tok_qk = [&](int t) { return ((size_t)b * T + t) * H + h; };      // row of q / k (times K)
     auto tok_v = [&](int t) { return ((size_t)b * T + t) * HV + hv; };     // row of v, g, dO (times V or K)
-    auto decay = [&](int t, float (&a)[R]) {
-#pragma unroll
-        for (int i = 0; i < R; ++i)
-            a[i] = expf(gate_value(to_f32(g[tok_v(t) * K + rg + RPP * i]), bias[i], rate, gate_mode, lower_bound));
-    };
-    auto load4 = [&](const Elt* p) {  // 4 consecutive elements as float4
-        return make_float4(to_f32(p[0]), to_f32(p[1]), to_f32(p[2]), to_f32(p[3]));
+    // the inputs of block blk's tokens into shared memory (rows past T left as they are: never read); callers
+    // put a barrier before (the previous block's values are read no more) and after
+    auto stage = [&](int blk, bool backward) {
+        const int t0 = blk * BWD_CK, n = min(BWD_CK, T - t0);
+        for (int idx = tid; idx < n * K; idx += Sh::NT) {
+            const int j = idx / K, row = idx - j * K, t = t0 + j;
+            sA[idx] = expf(gate_value(to_f32(g[tok_v(t) * K + row]), sBias[row], rate, gate_mode, lower_bound));
+            sK[idx] = to_f32(k[tok_qk(t) * K + row]);
+            if (backward) sQ[idx] = to_f32(q[tok_qk(t) * K + row]);
+        }
+        for (int idx = tid; idx < n * VB; idx += Sh::NT) {
+            const int j = idx / VB, c = idx - j * VB, t = t0 + j;
+            sV[idx] = to_f32(v[tok_v(t) * V + c0 + c]);
+            if (backward) sDO[idx] = to_f32(dO[tok_v(t) * V + c0 + c]);
+        }
+        if (tid < n) sB[tid] = to_f32(beta[tok_v(t0 + tid)]);
     };
     auto reduce = [&](float4 part) {
         const float4 s = reduce_over_rows<TPR, NW, VB>(part, sRed + red * NW * VB, lane, warp, cg);
@@ -124,23 +143,23 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
         return s;
     };
 
-    // one forward step on this thread's state rows: decay, residual (returned), rank-1 write
+    // one forward step on this thread's state rows, token j of the staged block: decay, residual (returned),
+    // rank-1 write
     float4 S[R];
-    auto forward_step = [&](int t) {
-        float a[R];
-        decay(t, a);
+    auto forward_step = [&](int j) {
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
         float kd[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            kd[i] = to_f32(k[tok_qk(t) * K + rg + RPP * i]);
-            S[i] = make_float4(a[i] * S[i].x, a[i] * S[i].y, a[i] * S[i].z, a[i] * S[i].w);
+            const float a = sA[j * K + rg + RPP * i];
+            kd[i] = sK[j * K + rg + RPP * i];
+            S[i] = make_float4(a * S[i].x, a * S[i].y, a * S[i].z, a * S[i].w);
             p = make_float4(p.x + kd[i] * S[i].x, p.y + kd[i] * S[i].y, p.z + kd[i] * S[i].z, p.w + kd[i] * S[i].w);
         }
         p = reduce(p);
-        const float4 vv = load4(v + tok_v(t) * V + c0 + 4 * cg);
+        const float4 vv = *reinterpret_cast<const float4*>(sV + j * VB + 4 * cg);
         const float4 r = make_float4(vv.x - p.x, vv.y - p.y, vv.z - p.z, vv.w - p.w);
-        const float bt = to_f32(beta[tok_v(t)]);
+        const float bt = sB[j];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const float w = bt * kd[i];
@@ -154,13 +173,15 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     for (int i = 0; i < R; ++i)
         S[i] = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * K + rg + RPP * i) * V + c0 + 4 * cg)
                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t = 0; t < T; ++t) {
-        if (t % BWD_CK == 0) {
+    for (int blk = 0; blk < NCK; ++blk) {
+        __syncthreads();  // the previous block's staged inputs are read no more (and sBias is written, at the start)
+        stage(blk, false);
+        __syncthreads();
 #pragma unroll
-            for (int i = 0; i < R; ++i)
-                *reinterpret_cast<float4*>(my_ckpt + ((size_t)(t / BWD_CK) * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-        }
-        forward_step(t);
+        for (int i = 0; i < R; ++i)
+            *reinterpret_cast<float4*>(my_ckpt + ((size_t)blk * K + rg + RPP * i) * VB + 4 * cg) = S[i];
+        const int n = min(BWD_CK, T - blk * BWD_CK);
+        for (int j = 0; j < n; ++j) forward_step(j);
     }
 
     // ---- 2. blocks in reverse ----------------------------------------------------------------------
@@ -171,6 +192,9 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                      : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int blk = NCK - 1; blk >= 0; --blk) {
         const int t0 = blk * BWD_CK, n = min(BWD_CK, T - t0);
+        __syncthreads();  // the previous block's staged inputs are read no more
+        stage(blk, true);
+        __syncthreads();
         // recompute: the state entering each token into shared memory (each thread its own entries),
         // the residuals too; S ends as the state after the block's last token
 #pragma unroll
@@ -180,20 +204,20 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
 #pragma unroll
             for (int i = 0; i < R; ++i)
                 *reinterpret_cast<float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-            const float4 r = forward_step(t0 + j);
+            const float4 r = forward_step(j);
             *reinterpret_cast<float4*>(sR + j * VB + 4 * cg) = r;  // same values from every row group
         }
         // reverse through the block; S holds the state after token t
         for (int j = n - 1; j >= 0; --j) {
             const int t = t0 + j;
             const size_t rq = tok_qk(t) * K, rv = tok_v(t);
-            const float4 dOc = load4(dO + rv * V + c0 + 4 * cg);
+            const float4 dOc = *reinterpret_cast<const float4*>(sDO + j * VB + 4 * cg);
             float qd[R], kd[R], a[R];
-            decay(t, a);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                qd[i] = to_f32(q[rq + rg + RPP * i]);
-                kd[i] = to_f32(k[rq + rg + RPP * i]);
+                a[i] = sA[j * K + rg + RPP * i];
+                qd[i] = sQ[j * K + rg + RPP * i];
+                kd[i] = sK[j * K + rg + RPP * i];
             }
             // dq_t = s S_t dO_t ; dS += s q_t dO_t^T
 #pragma unroll
@@ -211,7 +235,7 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                 u = make_float4(u.x + kd[i] * dS[i].x, u.y + kd[i] * dS[i].y, u.z + kd[i] * dS[i].z, u.w + kd[i] * dS[i].w);
             u = reduce(u);
             const float4 r = *reinterpret_cast<const float4*>(sR + j * VB + 4 * cg);
-            const float bt = to_f32(beta[rv]);
+            const float bt = sB[j];
             const float4 dr = make_float4(bt * u.x, bt * u.y, bt * u.z, bt * u.w);
             if (rg == 0) {  // dbeta_t = u . r over this CTA's columns; dv_t = dr
                 float db = dot4(u, r);
