@@ -481,8 +481,12 @@ def run_ours(args, ws, rank, local):
     # the other workloads, measured in the same run on rank 0 (extra keys, each with its roofline)
     if rank == 0 and not args.no_extras:
         extras = {}
+        want = set(args.extras.split(",")) if args.extras else None
+
+        def wanted(key):
+            return want is None or key in want
         for wid in (2, 3, 4):
-            if wid == w.wid:
+            if wid == w.wid or not wanted(f"workload{wid}"):
                 continue
             pf = Prefill(WORKLOADS[wid], rank_seed(WORKLOADS[wid], 0), dev, kda)
             v, mps, r = pf.measure(EXTRA_STEPS[wid], 3, 1, flush, hbm_peak, peak_kind)
@@ -491,18 +495,21 @@ def run_ours(args, ws, rank, local):
                                         "tokens_per_s": round(v, 1), "roofline": r}
             del pf
             torch.cuda.empty_cache()
-        if not w.is_decode:
+        if not w.is_decode and wanted("decode"):
             w5 = WORKLOADS[5]
             v, mps, r = measure_decode(w5, rank_seed(w5, 0), dev, kda, hbm_peak, peak_kind)
             extras["decode"] = {"workload": workload_config(w5, 1)["workload"], "steps": w5.decode_steps,
                                 "us_per_step": round(mps * 1e3, 2), "tokens_per_s": round(v, 1),
                                 "state_GBps": r["achieved"], "frac": r["frac"], "roofline": r}
         torch.cuda.empty_cache()
-        extras["mla_decode"] = measure_mla(dev, kda, hbm_peak, peak_kind, measured_peaks()[1])
-        torch.cuda.empty_cache()
-        extras["backward"] = measure_backward(dev, kda, hbm_peak, peak_kind)
-        torch.cuda.empty_cache()
-        extras["fallbacks"] = measure_fallbacks(dev, kda, hbm_peak, peak_kind)
+        if wanted("mla_decode"):
+            extras["mla_decode"] = measure_mla(dev, kda, hbm_peak, peak_kind, measured_peaks()[1])
+            torch.cuda.empty_cache()
+        if wanted("backward"):
+            extras["backward"] = measure_backward(dev, kda, hbm_peak, peak_kind)
+            torch.cuda.empty_cache()
+        if wanted("fallbacks"):
+            extras["fallbacks"] = measure_fallbacks(dev, kda, hbm_peak, peak_kind)
         line.update(extras)
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(w) if (ws == 1 and not args.no_cpu_baseline) else None
@@ -735,6 +742,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' extra keys")
+    ap.add_argument("--extras", default=None,
+                    help="comma-separated subset of the extra keys to measure (workload2, workload3, workload4, "
+                         "decode, mla_decode, backward, fallbacks); all by default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dry-plumbing", action="store_true",
                     help="multi-rank plumbing only, on CPU over gloo (no device is touched)")

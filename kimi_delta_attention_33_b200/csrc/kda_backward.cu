@@ -12,17 +12,23 @@
 // dq and dk of a q/k head add up over the value heads that read it (GVA), and every row quantity adds
 // up over the value columns.
 //
-// Layout: one CTA per (b, hv, block of VB = min(V, 8) value columns); value columns are independent in
-// the forward pass, so each CTA runs the recurrence on its columns alone.  Thread (row group rg, column
-// group cg) holds rows rg + RPP i (i < R) and columns 4 cg .. 4 cg + 3 of the state and of dS in
-// registers.  Reductions over key rows (the residual's prediction and u) go through warp shuffles and a
-// double-buffered shared array; row quantities summed over this CTA's columns are added into the fp32
-// outputs with atomics (the other column blocks and value heads add theirs).
+// Layout: one warp per (b, hv, block of VB value columns); value columns are independent in the forward
+// pass, so each warp runs the recurrence on its columns alone, and a CTA holds NWB such warps of one
+// (b, hv), which share the staged per-token inputs.  Lane (row group rg, column group cg) holds rows
+// rg + RG i (i < R) and columns 2 cg, 2 cg + 1 of the warp's block of the state and of dS in registers, as
+// pairs for the packed fp32x2 arithmetic, so reductions over key rows (the residual's prediction and u)
+// are warp shuffles, with no barrier on the per-token chain; two columns a lane keep the chain short and
+// give each SM sub-partition two warps to interleave.  Row quantities (dq, dk, dg) and dbeta, summed over each warp's columns, are kept per
+// warp in shared memory for the block of tokens, then summed over the CTA's warps and added into the fp32
+// outputs with one atomic per entry (the other CTAs of the value head, and the other value heads of a q/k
+// head, add theirs).
 //   1. forward sweep over all tokens, the state saved every CK tokens to the workspace;
 //   2. the blocks of CK tokens in reverse: the block's states recomputed from its checkpoint into
 //      shared memory, then its tokens in reverse order.
-// The per-token inputs of a block (decay, k, q, v, dO, beta) are staged in shared memory once per block
-// by loads that are all in flight together, so a token step does not wait for its own global loads.
+// The per-token inputs of a block (decay, k, q, v, dO, beta) are staged in shared memory once per block,
+// from 16-byte loads; the next block's are loaded into registers while this one is computed.  The decay
+// a = exp(gate) is computed once per (token, value head, key channel) by a small elementwise kernel into
+// the workspace, not again by every CTA that reads it.
 // A second, elementwise kernel chains dg through the gate when the op applied it.
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -35,237 +41,322 @@ constexpr int BWD_CK = 8;  // tokens between saved states
 
 template <int K, int V>
 struct BwdShape {
-    static constexpr int VB = V < 8 ? V : 8;                           // value columns per CTA
-    static constexpr int NT = (K * VB / 4 < 128) ? K * VB / 4 : 128;   // threads
-    static constexpr int TPR = VB / 4;                                 // threads per state row
-    static constexpr int RPP = NT / TPR;                               // row groups
-    static constexpr int R = K / RPP;                                  // rows per thread
-    static constexpr int NW = NT / 32;                                 // warps
-    static_assert(NT % 32 == 0 && RPP * R == K && TPR * 4 == VB, "backward shape");
-    // sPrev [CK][K][VB], sR [CK][VB], sRed 2 x [NW][VB], then the staged block: decay, k, q [CK][K], v, dO [CK][VB],
-    // beta [CK], and dt_bias [K]
-    static constexpr size_t smem_floats = (size_t)BWD_CK * K * VB + (size_t)BWD_CK * VB + 2 * (size_t)NW * VB +
-                                          3 * (size_t)BWD_CK * K + 2 * (size_t)BWD_CK * VB + BWD_CK + K;
+    static constexpr int RG = K < 32 ? K : 32;                       // row groups (lanes along the key rows)
+    static constexpr int TPR = 32 / RG;                              // lanes along the value columns
+    static constexpr int VB = 2 * TPR;                               // value columns per warp
+    static constexpr int R = K / RG;                                 // rows per lane
+    static constexpr int NCB = V / VB;                               // column blocks per (b, hv)
+    static constexpr int NWB = NCB < 4 ? NCB : 4;                    // warps (column blocks) per CTA
+    static constexpr int NT = 32 * NWB;                              // threads
+    static constexpr int CW = NWB * VB;                              // value columns per CTA
+    // 16-byte vectors a thread loads per block: decay (fp32) rows, k / q rows, v / dO columns (VN elements a vector)
+    template <typename Elt> static constexpr int VN = 16 / (int)sizeof(Elt);
+    static constexpr int EA = (BWD_CK * K / 4 + NT - 1) / NT;
+    template <typename Elt> static constexpr int EK = (BWD_CK * K / VN<Elt> + NT - 1) / NT;
+    template <typename Elt> static constexpr int EV = (BWD_CK * CW / VN<Elt> + NT - 1) / NT;
+    static_assert(RG * TPR == 32 && R * RG == K && NCB % NWB == 0, "backward shape");
+    static_assert(K % 16 == 0 && CW % 8 == 0, "16-byte staging vectors");
+    // sPrev [NWB][CK][K][VB], sR [NWB][CK][VB]; the staged block: decay, k, q [CK][K], v, dO [CK][CW], beta [CK];
+    // the block's per-warp row sums dq, dk, dg [NWB][CK][K] and dbeta [NWB][CK]
+    static constexpr size_t smem_floats = (size_t)NWB * BWD_CK * K * VB + (size_t)NWB * BWD_CK * VB +
+                                          3 * (size_t)BWD_CK * K + 2 * (size_t)BWD_CK * CW + BWD_CK +
+                                          3 * (size_t)NWB * BWD_CK * K + (size_t)NWB * BWD_CK;
     static constexpr size_t smem_bytes = smem_floats * sizeof(float);
 };
 
+// packed fp32x2 arithmetic (each half rounded as the scalar operation)
+__device__ __forceinline__ float2 f2_splat(float s) { return make_float2(s, s); }
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+
+// a 16-byte vector of inputs, as fp32, into shared memory (dst 16-byte aligned)
+__device__ __forceinline__ void put_f32(float* dst, uint4 raw, const float*) { *reinterpret_cast<uint4*>(dst) = raw; }
+__device__ __forceinline__ void put_f32(float* dst, uint4 raw, const __nv_bfloat16*) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);  // bf16 is the top half of an fp32
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+    *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
-__device__ __forceinline__ float4 f4_shfl_xor(float4 a, int off) {
-    return make_float4(__shfl_xor_sync(0xffffffffu, a.x, off), __shfl_xor_sync(0xffffffffu, a.y, off),
-                       __shfl_xor_sync(0xffffffffu, a.z, off), __shfl_xor_sync(0xffffffffu, a.w, off));
-}
 
-// Sum over all key rows of this CTA of a per-thread partial over its rows, for its four columns; every
-// thread gets the result for its own columns.  `buf` alternates between two [NW][VB] arrays.
-template <int TPR, int NW, int VB>
-__device__ __forceinline__ float4 reduce_over_rows(float4 part, float* buf, int lane, int warp, int cg) {
-#pragma unroll
-    for (int off = TPR; off < 32; off <<= 1) part = f4_add(part, f4_shfl_xor(part, off));
-    if (lane < TPR) *reinterpret_cast<float4*>(buf + warp * VB + 4 * cg) = part;
-    __syncthreads();
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < NW; ++w) s = f4_add(s, *reinterpret_cast<const float4*>(buf + w * VB + 4 * cg));
-    return s;
-}
-
-// Sum of x over this thread's four columns and the TPR lanes that share its rows (lanes cg = 0 .. TPR-1
-// are adjacent); lane cg = 0 holds the total for the CTA's VB columns.
+// Sum over the warp's key rows of a per-lane partial over its rows, for its two columns; every lane gets
+// the result for its own columns (the lanes of a column group differ in the bits from TPR up).
 template <int TPR>
-__device__ __forceinline__ float sum_over_cols(float4 x) {
-    float s = (x.x + x.y) + (x.z + x.w);
+__device__ __forceinline__ float2 sum_over_rows(float2 part) {
+#pragma unroll
+    for (int off = TPR; off < 32; off <<= 1)
+        part = f2_add(part, make_float2(__shfl_xor_sync(0xffffffffu, part.x, off), __shfl_xor_sync(0xffffffffu, part.y, off)));
+    return part;
+}
+
+// Sum of x over this lane's two columns and the TPR lanes that share its rows (lanes cg = 0 .. TPR-1
+// are adjacent); every one of them gets the total for the warp's VB columns.
+template <int TPR>
+__device__ __forceinline__ float sum_over_cols(float2 x) {
+    float s = x.x + x.y;
 #pragma unroll
     for (int off = 1; off < TPR; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     return s;
 }
-
-__device__ __forceinline__ float dot4(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 
 }  // namespace
 
 template <typename Elt, int K, int V>
 __global__ void __launch_bounds__(BwdShape<K, V>::NT)
 recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const Elt* __restrict__ v,
-                     const Elt* __restrict__ g, const Elt* __restrict__ beta, const float* __restrict__ A_log,
-                     const float* __restrict__ dt_bias, const float* __restrict__ S0, const Elt* __restrict__ dO,
-                     const float* __restrict__ dS_T, int T, int H, int HV, int gate_mode, float lower_bound,
-                     float scale, float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
-                     float* __restrict__ dg, float* __restrict__ dbeta, float* __restrict__ dS0,
-                     float* __restrict__ ckpt) {
+                     const float* __restrict__ decay, const Elt* __restrict__ beta, const float* __restrict__ S0,
+                     const Elt* __restrict__ dO, const float* __restrict__ dS_T, int T, int H, int HV, float scale,
+                     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg,
+                     float* __restrict__ dbeta, float* __restrict__ dS0, float* __restrict__ ckpt) {
     using Sh = BwdShape<K, V>;
-    constexpr int VB = Sh::VB, TPR = Sh::TPR, RPP = Sh::RPP, R = Sh::R, NW = Sh::NW, NVB = V / VB;
+    constexpr int VB = Sh::VB, TPR = Sh::TPR, RG = Sh::RG, R = Sh::R, NT = Sh::NT, NWB = Sh::NWB, CW = Sh::CW;
+    constexpr int CK = BWD_CK, VN = Sh::template VN<Elt>, EA = Sh::EA, EK = Sh::template EK<Elt>,
+                  EV = Sh::template EV<Elt>;
     extern __shared__ float bsm[];
-    float* sPrev = bsm;                        // [CK][K][VB] state entering each token of the block
-    float* sR = sPrev + BWD_CK * K * VB;       // [CK][VB] residuals
-    float* sRed = sR + BWD_CK * VB;            // 2 x [NW][VB] reduction buffers
-    float* sA = sRed + 2 * NW * VB;            // staged block: [CK][K] decay exp(g)
-    float* sK = sA + BWD_CK * K;               //               [CK][K] k
-    float* sQ = sK + BWD_CK * K;               //               [CK][K] q
-    float* sV = sQ + BWD_CK * K;               //               [CK][VB] v (this CTA's columns)
-    float* sDO = sV + BWD_CK * VB;             //               [CK][VB] dO
-    float* sB = sDO + BWD_CK * VB;             //               [CK] beta
-    float* sBias = sB + BWD_CK;                // [K] dt_bias (zeros when absent)
-
-    const int vbi = blockIdx.x % NVB, pair = blockIdx.x / NVB;
-    const int b = pair / HV, hv = pair - b * HV, h = hv / (HV / H);
-    const int c0 = vbi * VB;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cg = tid % TPR, rg = tid / TPR;
-    const float rate = (gate_mode != KDA_GATE_NONE) ? expf(A_log[hv]) : 0.0f;
-    for (int d = tid; d < K; d += Sh::NT)
-        sBias[d] = (dt_bias != nullptr && gate_mode != KDA_GATE_NONE) ? dt_bias[hv * K + d] : 0.0f;
-    const int NCK = (T + BWD_CK - 1) / BWD_CK;
-    float* my_ckpt = ckpt + (size_t)blockIdx.x * NCK * K * VB;
-    int red = 0;  // which reduction buffer the next reduction uses
+    float* sPrev = bsm + (size_t)warp * CK * K * VB;  // [CK][K][VB] state entering each token (this warp's)
+    float* sR = bsm + (size_t)NWB * CK * K * VB + warp * CK * VB;  // [CK][VB] residuals (this warp's)
+    float* sA = bsm + (size_t)NWB * CK * K * VB + NWB * CK * VB;   // staged block: [CK][K] decay exp(g)
+    float* sK = sA + CK * K;                   //               [CK][K] k
+    float* sQ = sK + CK * K;                   //               [CK][K] q
+    float* sV = sQ + CK * K;                   //               [CK][CW] v (this CTA's columns)
+    float* sDO = sV + CK * CW;                 //               [CK][CW] dO
+    float* sB = sDO + CK * CW;                 //               [CK] beta
+    float* sDq = sB + CK;                      // [NWB][CK][K] dq of the block, each warp's over its columns
+    float* sDk = sDq + NWB * CK * K;           // [NWB][CK][K] dk
+    float* sDg = sDk + NWB * CK * K;           // [NWB][CK][K] dg
+    float* sDb = sDg + NWB * CK * K;           // [NWB][CK] dbeta
+    float* wDq = sDq + warp * CK * K;          // this warp's
+    float* wDk = sDk + warp * CK * K;
+    float* wDg = sDg + warp * CK * K;
+
+    constexpr int CPP = Sh::NCB / NWB;         // CTAs per (b, hv)
+    const int pair = blockIdx.x / CPP;
+    const int b = pair / HV, hv = pair - b * HV, h = hv / (HV / H);
+    const int cc0 = (blockIdx.x - pair * CPP) * CW;  // first value column of the CTA
+    const int c0 = cc0 + warp * VB;                  // first value column of the warp
+    const int cg = lane % TPR, rg = lane / TPR;
+    const int NCK = (T + CK - 1) / CK;
+    float* my_ckpt = ckpt + ((size_t)pair * Sh::NCB + c0 / VB) * NCK * K * VB;
 
     auto tok_qk = [&](int t) { return ((size_t)b * T + t) * H + h; };      // row of q / k (times K)
     auto tok_v = [&](int t) { return ((size_t)b * T + t) * HV + hv; };     // row of v, g, dO (times V or K)
-    // the inputs of block blk's tokens into shared memory (rows past T left as they are: never read); callers
-    // put a barrier before (the previous block's values are read no more) and after
-    auto stage = [&](int blk, bool backward) {
-        const int t0 = blk * BWD_CK, n = min(BWD_CK, T - t0);
-        for (int idx = tid; idx < n * K; idx += Sh::NT) {
-            const int j = idx / K, row = idx - j * K, t = t0 + j;
-            sA[idx] = expf(gate_value(to_f32(g[tok_v(t) * K + row]), sBias[row], rate, gate_mode, lower_bound));
-            sK[idx] = to_f32(k[tok_qk(t) * K + row]);
-            if (backward) sQ[idx] = to_f32(q[tok_qk(t) * K + row]);
+
+    // the next block's inputs as loaded: 16-byte vectors of decay rows, k / q rows, and the CTA's v / dO columns
+    uint4 la[EA], lk[EK], lq[EK], lv[EV], lo[EV];
+    Elt lb;
+    constexpr int KV = K / VN, CV = CW / VN;  // vectors in a k / q row, in the CTA's v / dO columns
+    auto load_block = [&](int blk, bool backward) {
+        const int t0 = blk * CK, n = min(CK, T - t0);
+#pragma unroll
+        for (int e = 0; e < EA; ++e) {
+            const int idx = tid + e * NT, j = idx / (K / 4), x = idx - j * (K / 4);
+            if (idx < n * (K / 4)) la[e] = reinterpret_cast<const uint4*>(decay + tok_v(t0 + j) * K)[x];
         }
-        for (int idx = tid; idx < n * VB; idx += Sh::NT) {
-            const int j = idx / VB, c = idx - j * VB, t = t0 + j;
-            sV[idx] = to_f32(v[tok_v(t) * V + c0 + c]);
-            if (backward) sDO[idx] = to_f32(dO[tok_v(t) * V + c0 + c]);
+#pragma unroll
+        for (int e = 0; e < EK; ++e) {
+            const int idx = tid + e * NT, j = idx / KV, x = idx - j * KV;
+            if (idx < n * KV) {
+                lk[e] = reinterpret_cast<const uint4*>(k + tok_qk(t0 + j) * K)[x];
+                if (backward) lq[e] = reinterpret_cast<const uint4*>(q + tok_qk(t0 + j) * K)[x];
+            }
         }
-        if (tid < n) sB[tid] = to_f32(beta[tok_v(t0 + tid)]);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+            const int idx = tid + e * NT, j = idx / CV, x = idx - j * CV;
+            if (idx < n * CV) {
+                lv[e] = reinterpret_cast<const uint4*>(v + tok_v(t0 + j) * V + cc0)[x];
+                if (backward) lo[e] = reinterpret_cast<const uint4*>(dO + tok_v(t0 + j) * V + cc0)[x];
+            }
+        }
+        if (tid < n) lb = beta[tok_v(t0 + tid)];
     };
-    auto reduce = [&](float4 part) {
-        const float4 s = reduce_over_rows<TPR, NW, VB>(part, sRed + red * NW * VB, lane, warp, cg);
-        red ^= 1;
-        return s;
+    // the loaded block into shared memory as fp32 (rows past T are never read); callers put a barrier
+    // before (the previous block's staged values are read no more) and after
+    auto stage_block = [&](int n, bool backward) {
+#pragma unroll
+        for (int e = 0; e < EA; ++e) {
+            const int idx = tid + e * NT;
+            if (idx < n * (K / 4)) *reinterpret_cast<uint4*>(sA + 4 * idx) = la[e];
+        }
+#pragma unroll
+        for (int e = 0; e < EK; ++e) {
+            const int idx = tid + e * NT;
+            if (idx < n * KV) {
+                put_f32(sK + VN * idx, lk[e], k);
+                if (backward) put_f32(sQ + VN * idx, lq[e], q);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+            const int idx = tid + e * NT;
+            if (idx < n * CV) {
+                put_f32(sV + VN * idx, lv[e], v);
+                if (backward) put_f32(sDO + VN * idx, lo[e], dO);
+            }
+        }
+        if (tid < n) sB[tid] = to_f32(lb);
     };
 
-    // one forward step on this thread's state rows, token j of the staged block: decay, residual (returned),
-    // rank-1 write
-    float4 S[R];
+    // one forward step on this lane's state entries, token j of the staged block: decay, residual
+    // (returned), rank-1 write
+    float2 S[R];
     auto forward_step = [&](int j) {
-        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 p = make_float2(0.f, 0.f);
         float kd[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const float a = sA[j * K + rg + RPP * i];
-            kd[i] = sK[j * K + rg + RPP * i];
-            S[i] = make_float4(a * S[i].x, a * S[i].y, a * S[i].z, a * S[i].w);
-            p = make_float4(p.x + kd[i] * S[i].x, p.y + kd[i] * S[i].y, p.z + kd[i] * S[i].z, p.w + kd[i] * S[i].w);
+            const float a = sA[j * K + rg + RG * i];
+            kd[i] = sK[j * K + rg + RG * i];
+            S[i] = f2_mul(f2_splat(a), S[i]);
+            p = f2_fma(f2_splat(kd[i]), S[i], p);
         }
-        p = reduce(p);
-        const float4 vv = *reinterpret_cast<const float4*>(sV + j * VB + 4 * cg);
-        const float4 r = make_float4(vv.x - p.x, vv.y - p.y, vv.z - p.z, vv.w - p.w);
+        p = sum_over_rows<TPR>(p);
+        const float2 r = f2_sub(*reinterpret_cast<const float2*>(sV + j * CW + warp * VB + 2 * cg), p);
         const float bt = sB[j];
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const float w = bt * kd[i];
-            S[i] = make_float4(S[i].x + w * r.x, S[i].y + w * r.y, S[i].z + w * r.z, S[i].w + w * r.w);
-        }
+        for (int i = 0; i < R; ++i) S[i] = f2_fma(f2_splat(bt * kd[i]), r, S[i]);
         return r;
     };
+    auto state_row = [&](int i) { return (size_t)(rg + RG * i) * VB + 2 * cg; };  // offset in a [K][VB] block
 
     // ---- 1. forward sweep, the entering state of every block of CK tokens saved ---------------------
 #pragma unroll
     for (int i = 0; i < R; ++i)
-        S[i] = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)pair * K + rg + RPP * i) * V + c0 + 4 * cg)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[i] = S0 ? *reinterpret_cast<const float2*>(S0 + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg)
+                  : make_float2(0.f, 0.f);
+    load_block(0, false);
     for (int blk = 0; blk < NCK; ++blk) {
-        __syncthreads();  // the previous block's staged inputs are read no more (and sBias is written, at the start)
-        stage(blk, false);
+        const int n = min(CK, T - blk * CK);
+        __syncthreads();  // the previous block's staged inputs are read no more (sBias written, at the start)
+        stage_block(n, false);
         __syncthreads();
+        if (blk + 1 < NCK) load_block(blk + 1, false);
 #pragma unroll
         for (int i = 0; i < R; ++i)
-            *reinterpret_cast<float4*>(my_ckpt + ((size_t)blk * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-        const int n = min(BWD_CK, T - blk * BWD_CK);
+            *reinterpret_cast<float2*>(my_ckpt + (size_t)blk * K * VB + state_row(i)) = S[i];
         for (int j = 0; j < n; ++j) forward_step(j);
     }
 
     // ---- 2. blocks in reverse ----------------------------------------------------------------------
-    float4 dS[R];
+    float2 dS[R];
 #pragma unroll
     for (int i = 0; i < R; ++i)
-        dS[i] = dS_T ? *reinterpret_cast<const float4*>(dS_T + ((size_t)pair * K + rg + RPP * i) * V + c0 + 4 * cg)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        dS[i] = dS_T ? *reinterpret_cast<const float2*>(dS_T + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg)
+                     : make_float2(0.f, 0.f);
+    load_block(NCK - 1, true);
     for (int blk = NCK - 1; blk >= 0; --blk) {
-        const int t0 = blk * BWD_CK, n = min(BWD_CK, T - t0);
-        __syncthreads();  // the previous block's staged inputs are read no more
-        stage(blk, true);
+        const int t0 = blk * CK, n = min(CK, T - t0);
+        __syncthreads();  // the previous block's staged inputs and row sums are read no more
+        stage_block(n, true);
         __syncthreads();
-        // recompute: the state entering each token into shared memory (each thread its own entries),
-        // the residuals too; S ends as the state after the block's last token
+        if (blk > 0) load_block(blk - 1, true);
+        // recompute: the state entering each token into shared memory (each lane its own entries), the
+        // residuals too; S ends as the state after the block's last token
 #pragma unroll
-        for (int i = 0; i < R; ++i)
-            S[i] = *reinterpret_cast<const float4*>(my_ckpt + ((size_t)blk * K + rg + RPP * i) * VB + 4 * cg);
+        for (int i = 0; i < R; ++i) S[i] = *reinterpret_cast<const float2*>(my_ckpt + (size_t)blk * K * VB + state_row(i));
         for (int j = 0; j < n; ++j) {
 #pragma unroll
-            for (int i = 0; i < R; ++i)
-                *reinterpret_cast<float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg) = S[i];
-            const float4 r = forward_step(j);
-            *reinterpret_cast<float4*>(sR + j * VB + 4 * cg) = r;  // same values from every row group
+            for (int i = 0; i < R; ++i) *reinterpret_cast<float2*>(sPrev + (size_t)j * K * VB + state_row(i)) = S[i];
+            const float2 r = forward_step(j);
+            if (rg == 0) *reinterpret_cast<float2*>(sR + j * VB + 2 * cg) = r;  // same values in every row group
         }
+        __syncwarp();
         // reverse through the block; S holds the state after token t
         for (int j = n - 1; j >= 0; --j) {
-            const int t = t0 + j;
-            const size_t rq = tok_qk(t) * K, rv = tok_v(t);
-            const float4 dOc = *reinterpret_cast<const float4*>(sDO + j * VB + 4 * cg);
+            const float2 dOc = *reinterpret_cast<const float2*>(sDO + j * CW + warp * VB + 2 * cg);
             float qd[R], kd[R], a[R];
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                a[i] = sA[j * K + rg + RPP * i];
-                qd[i] = sQ[j * K + rg + RPP * i];
-                kd[i] = sK[j * K + rg + RPP * i];
+                a[i] = sA[j * K + rg + RG * i];
+                qd[i] = sQ[j * K + rg + RG * i];
+                kd[i] = sK[j * K + rg + RG * i];
             }
             // dq_t = s S_t dO_t ; dS += s q_t dO_t^T
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float part =
-                    sum_over_cols<TPR>(make_float4(S[i].x * dOc.x, S[i].y * dOc.y, S[i].z * dOc.z, S[i].w * dOc.w));
-                if (cg == 0) atomicAdd(dq + rq + rg + RPP * i, scale * part);
-                const float w = scale * qd[i];
-                dS[i] = make_float4(dS[i].x + w * dOc.x, dS[i].y + w * dOc.y, dS[i].z + w * dOc.z, dS[i].w + w * dOc.w);
+                const float part = sum_over_cols<TPR>(f2_mul(S[i], dOc));
+                if (cg == 0) wDq[j * K + rg + RG * i] = scale * part;
+                dS[i] = f2_fma(f2_splat(scale * qd[i]), dOc, dS[i]);
             }
             // u = dS^T k_t over the key rows
-            float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+            float2 u = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < R; ++i)
-                u = make_float4(u.x + kd[i] * dS[i].x, u.y + kd[i] * dS[i].y, u.z + kd[i] * dS[i].z, u.w + kd[i] * dS[i].w);
-            u = reduce(u);
-            const float4 r = *reinterpret_cast<const float4*>(sR + j * VB + 4 * cg);
+            for (int i = 0; i < R; ++i) u = f2_fma(f2_splat(kd[i]), dS[i], u);
+            u = sum_over_rows<TPR>(u);
+            const float2 r = *reinterpret_cast<const float2*>(sR + j * VB + 2 * cg);
             const float bt = sB[j];
-            const float4 dr = make_float4(bt * u.x, bt * u.y, bt * u.z, bt * u.w);
-            if (rg == 0) {  // dbeta_t = u . r over this CTA's columns; dv_t = dr
-                float db = dot4(u, r);
+            const float2 dr = f2_mul(f2_splat(bt), u);
+            if (rg == 0) {  // dbeta_t = u . r over this warp's columns; dv_t = dr
+                float db = u.x * r.x + u.y * r.y;
 #pragma unroll
                 for (int off = 1; off < TPR; off <<= 1) db += __shfl_xor_sync((1u << TPR) - 1u, db, off);
-                if (cg == 0) atomicAdd(dbeta + rv, db);
-                *reinterpret_cast<float4*>(dv + rv * V + c0 + 4 * cg) = dr;
+                if (cg == 0) sDb[warp * CK + j] = db;
+                *reinterpret_cast<float2*>(dv + tok_v(t0 + j) * V + c0 + 2 * cg) = dr;
             }
+            const float2 btr = f2_mul(f2_splat(bt), r);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float4 Sp = *reinterpret_cast<const float4*>(sPrev + ((size_t)j * K + rg + RPP * i) * VB + 4 * cg);
-                const float4 Sd = make_float4(a[i] * Sp.x, a[i] * Sp.y, a[i] * Sp.z, a[i] * Sp.w);
+                const float2 Sp = *reinterpret_cast<const float2*>(sPrev + (size_t)j * K * VB + state_row(i));
+                const float2 Sd = f2_mul(f2_splat(a[i]), Sp);
                 // dk_t = beta dS r - S_dec dr
-                const float pk = sum_over_cols<TPR>(make_float4(bt * dS[i].x * r.x - Sd.x * dr.x, bt * dS[i].y * r.y - Sd.y * dr.y,
-                                                                bt * dS[i].z * r.z - Sd.z * dr.z, bt * dS[i].w * r.w - Sd.w * dr.w));
-                if (cg == 0) atomicAdd(dk + rq + rg + RPP * i, pk);
+                const float pk = sum_over_cols<TPR>(f2_sub(f2_mul(dS[i], btr), f2_mul(Sd, dr)));
+                if (cg == 0) wDk[j * K + rg + RG * i] = pk;
                 // dS_dec = dS - k dr^T ; dg_t = a rowsum(dS_dec S_{t-1}) ; dS_{t-1} = a dS_dec
-                const float4 dSd = make_float4(dS[i].x - kd[i] * dr.x, dS[i].y - kd[i] * dr.y, dS[i].z - kd[i] * dr.z,
-                                               dS[i].w - kd[i] * dr.w);
-                const float pg = sum_over_cols<TPR>(make_float4(dSd.x * Sp.x, dSd.y * Sp.y, dSd.z * Sp.z, dSd.w * Sp.w));
-                if (cg == 0) atomicAdd(dg + rv * K + rg + RPP * i, a[i] * pg);
-                dS[i] = make_float4(a[i] * dSd.x, a[i] * dSd.y, a[i] * dSd.z, a[i] * dSd.w);
+                const float2 dSd = f2_fma(f2_splat(-kd[i]), dr, dS[i]);
+                const float pg = sum_over_cols<TPR>(f2_mul(dSd, Sp));
+                if (cg == 0) wDg[j * K + rg + RG * i] = a[i] * pg;
+                dS[i] = f2_mul(f2_splat(a[i]), dSd);
                 S[i] = Sp;
             }
+        }
+        __syncthreads();  // the block's row sums are complete
+        for (int idx = tid; idx < n * (K / 4); idx += NT) {  // four key channels at a time
+            const int j = idx / (K / 4), row = 4 * (idx - j * (K / 4));
+            float4 sq = make_float4(0.f, 0.f, 0.f, 0.f), sk = sq, sg = sq;
+#pragma unroll
+            for (int w = 0; w < NWB; ++w) {
+                sq = f4_add(sq, *reinterpret_cast<const float4*>(sDq + w * CK * K + 4 * idx));
+                sk = f4_add(sk, *reinterpret_cast<const float4*>(sDk + w * CK * K + 4 * idx));
+                sg = f4_add(sg, *reinterpret_cast<const float4*>(sDg + w * CK * K + 4 * idx));
+            }
+            atomicAdd(reinterpret_cast<float4*>(dq + tok_qk(t0 + j) * K + row), sq);
+            atomicAdd(reinterpret_cast<float4*>(dk + tok_qk(t0 + j) * K + row), sk);
+            atomicAdd(reinterpret_cast<float4*>(dg + tok_v(t0 + j) * K + row), sg);
+        }
+        if (tid < n) {
+            float sb = 0.f;
+#pragma unroll
+            for (int w = 0; w < NWB; ++w) sb += sDb[w * CK + tid];
+            atomicAdd(dbeta + tok_v(t0 + tid), sb);
         }
     }
     if (dS0) {
 #pragma unroll
         for (int i = 0; i < R; ++i)
-            *reinterpret_cast<float4*>(dS0 + ((size_t)pair * K + rg + RPP * i) * V + c0 + 4 * cg) = dS[i];
+            *reinterpret_cast<float2*>(dS0 + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg) = dS[i];
+    }
+}
+
+// a = exp(gate(g_raw)) per (b, t, hv, key channel), fp32: the per-token decays of the recurrence (with
+// GATE_NONE g is the log decay itself).
+template <typename Elt>
+__global__ void __launch_bounds__(256)
+decay_kernel(const Elt* __restrict__ g, const float* __restrict__ A_log, const float* __restrict__ dt_bias, long long n,
+             int HV, int K, int mode, float lower_bound, float* __restrict__ a) {
+    for (long long i = (long long)blockIdx.x * 256 + threadIdx.x; i < n; i += (long long)gridDim.x * 256) {
+        const int d = (int)(i % K), hv = (int)((i / K) % HV);
+        const float rate = mode != KDA_GATE_NONE ? expf(A_log[hv]) : 0.0f;
+        const float bias = (dt_bias != nullptr && mode != KDA_GATE_NONE) ? dt_bias[hv * K + d] : 0.0f;
+        a[i] = expf(gate_value(to_f32(g[i]), bias, rate, mode, lower_bound));
     }
 }
 
@@ -320,17 +411,29 @@ gate_bwd_kernel(const Elt* __restrict__ g_raw, const float* __restrict__ A_log, 
 
 namespace {
 
+// the states saved every CK tokens: [B][HV][V / VB][ceil(T / CK)][K][VB] floats
+size_t backward_ckpt_floats(int B, int T, int HV, int K, int V) {
+    const size_t nck = ((size_t)T + BWD_CK - 1) / BWD_CK;
+    return (size_t)B * HV * nck * K * V;
+}
+
 template <typename Elt, int K, int V>
 cudaError_t launch_bwd(const BackwardArgs& a) {
     using Sh = BwdShape<K, V>;
+    // workspace: the saved states, then the decays [B][T][HV][K]
+    float* ckpt = static_cast<float*>(a.workspace);
+    float* decay = ckpt + backward_ckpt_floats(a.B, a.T, a.HV, K, V);
+    const long long n = (long long)a.B * a.T * a.HV * K;
+    const unsigned dgrid = (unsigned)std::min<long long>((n + 255) / 256, 148ll * 16);
+    decay_kernel<Elt><<<dgrid, 256, 0, a.stream>>>(static_cast<const Elt*>(a.g), a.A_log, a.dt_bias, n, a.HV, K,
+                                                   a.gate_mode, a.lower_bound, decay);
     auto kern = recurrent_bwd_kernel<Elt, K, V>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::smem_bytes);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)((long long)a.B * a.HV * (V / Sh::VB)), Sh::NT, Sh::smem_bytes, a.stream>>>(
-        static_cast<const Elt*>(a.q), static_cast<const Elt*>(a.k), static_cast<const Elt*>(a.v),
-        static_cast<const Elt*>(a.g), static_cast<const Elt*>(a.beta), a.A_log, a.dt_bias, a.S0,
-        static_cast<const Elt*>(a.dO), a.dS_T, a.T, a.H, a.HV, a.gate_mode, a.lower_bound, a.scale, a.dq, a.dk, a.dv,
-        a.dg, a.dbeta, a.dS0, static_cast<float*>(a.workspace));
+    kern<<<(unsigned)((long long)a.B * a.HV * (Sh::NCB / Sh::NWB)), Sh::NT, Sh::smem_bytes, a.stream>>>(
+        static_cast<const Elt*>(a.q), static_cast<const Elt*>(a.k), static_cast<const Elt*>(a.v), decay,
+        static_cast<const Elt*>(a.beta), a.S0, static_cast<const Elt*>(a.dO), a.dS_T, a.T, a.H, a.HV, a.scale, a.dq,
+        a.dk, a.dv, a.dg, a.dbeta, a.dS0, ckpt);
     return cudaGetLastError();
 }
 
@@ -359,8 +462,7 @@ cudaError_t bwd_k(const BackwardArgs& a) {
 }  // namespace
 
 size_t backward_workspace(int B, int T, int HV, int K, int V) {
-    const size_t nck = ((size_t)T + BWD_CK - 1) / BWD_CK;
-    return (size_t)B * HV * nck * K * V * sizeof(float);
+    return (backward_ckpt_floats(B, T, HV, K, V) + (size_t)B * T * HV * K) * sizeof(float);
 }
 
 cudaError_t launch_backward(const BackwardArgs& a) {
