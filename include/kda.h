@@ -248,8 +248,9 @@ kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, co
 
 /*
  * kda_backward_workspace_size -- bytes of device workspace kda_backward needs for these sizes (the
- * state saved every 8 tokens, B * HV * ceil(T / 8) * K * V * 4 bytes, then the fp32 decays
- * exp(gate) of every token, B * T * HV * K * 4 bytes), or 0 for sizes it rejects.
+ * state saved every 8 tokens, B * HV * ceil(T / 8) * K * V * 4 bytes, the fp32 decays exp(gate)
+ * of every token, B * T * HV * K * 4 bytes, and the fp32 residuals of every token, B * T * HV * V * 4
+ * bytes), or 0 for sizes it rejects.
  */
 size_t kda_backward_workspace_size(int B, int T, int H, int HV, int K, int V);
 

@@ -15,16 +15,18 @@
 // Layout: one warp per (b, hv, block of VB value columns); value columns are independent in the forward
 // pass, so each warp runs the recurrence on its columns alone, and a CTA holds NWB such warps of one
 // (b, hv), which share the staged per-token inputs.  Lane (row group rg, column group cg) holds rows
-// rg + RG i (i < R) and columns 2 cg, 2 cg + 1 of the warp's block of the state and of dS in registers, as
+// R rg .. R rg + R - 1 and columns 2 cg, 2 cg + 1 of the warp's block of the state and of dS in registers, as
 // pairs for the packed fp32x2 arithmetic, so reductions over key rows (the residual's prediction and u)
 // are warp shuffles, with no barrier on the per-token chain; two columns a lane keep the chain short and
 // give each SM sub-partition two warps to interleave.  Row quantities (dq, dk, dg) and dbeta, summed over each warp's columns, are kept per
 // warp in shared memory for the block of tokens, then summed over the CTA's warps and added into the fp32
 // outputs with one atomic per entry (the other CTAs of the value head, and the other value heads of a q/k
 // head, add theirs).
-//   1. forward sweep over all tokens, the state saved every CK tokens to the workspace;
+//   1. forward sweep over all tokens, the state saved every CK tokens and the residual r of every token
+//      to the workspace;
 //   2. the blocks of CK tokens in reverse: the block's states recomputed from its checkpoint into
-//      shared memory, then its tokens in reverse order.
+//      shared memory (with the saved residuals this is a rank-1 update a token, no reduction), then its
+//      tokens in reverse order.
 // The per-token inputs of a block (decay, k, q, v, dO, beta) are staged in shared memory once per block,
 // from 16-byte loads; the next block's are loaded into registers while this one is computed.  The decay
 // a = exp(gate) is computed once per (token, value head, key channel) by a small elementwise kernel into
@@ -54,13 +56,14 @@ struct BwdShape {
     static constexpr int EA = (BWD_CK * K / 4 + NT - 1) / NT;
     template <typename Elt> static constexpr int EK = (BWD_CK * K / VN<Elt> + NT - 1) / NT;
     template <typename Elt> static constexpr int EV = (BWD_CK * CW / VN<Elt> + NT - 1) / NT;
+    static constexpr int ER = (BWD_CK * CW / 4 + NT - 1) / NT;  // saved residuals (fp32)
     static_assert(RG * TPR == 32 && R * RG == K && NCB % NWB == 0, "backward shape");
     static_assert(K % 16 == 0 && CW % 8 == 0, "16-byte staging vectors");
-    // sPrev [NWB][CK][K][VB], sR [NWB][CK][VB]; the staged block: decay, k, q [CK][K], v, dO [CK][CW], beta [CK];
-    // the block's per-warp row sums dq, dk, dg [NWB][CK][K] and dbeta [NWB][CK]
-    static constexpr size_t smem_floats = (size_t)NWB * BWD_CK * K * VB + (size_t)NWB * BWD_CK * VB +
-                                          3 * (size_t)BWD_CK * K + 2 * (size_t)BWD_CK * CW + BWD_CK +
-                                          3 * (size_t)NWB * BWD_CK * K + (size_t)NWB * BWD_CK;
+    // sPrev [NWB][CK][K][VB]; the staged block: decay, k, q [CK][K], v, dO, r [CK][CW], beta [CK]; the block's
+    // per-warp row sums dq, dk, dg [NWB][CK][K] and dbeta [NWB][CK]
+    static constexpr size_t smem_floats = (size_t)NWB * BWD_CK * K * VB + 3 * (size_t)BWD_CK * K +
+                                          3 * (size_t)BWD_CK * CW + BWD_CK + 3 * (size_t)NWB * BWD_CK * K +
+                                          (size_t)NWB * BWD_CK;
     static constexpr size_t smem_bytes = smem_floats * sizeof(float);
 };
 
@@ -107,6 +110,27 @@ __device__ __forceinline__ float sum_over_cols(float2 x) {
     return s;
 }
 
+// R consecutive floats (a lane's key rows) from / to shared memory, as one vector access (R in {1, 2, 4};
+// the address is R-float aligned)
+template <int R>
+__device__ __forceinline__ void rows_of(const float* p, float (&x)[R]) {
+    if constexpr (R == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
+    } else if constexpr (R == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        x[0] = v.x, x[1] = v.y;
+    } else {
+        x[0] = *p;
+    }
+}
+template <int R>
+__device__ __forceinline__ void put_rows(float* p, const float (&x)[R]) {
+    if constexpr (R == 4) *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else if constexpr (R == 2) *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+    else *p = x[0];
+}
+
 }  // namespace
 
 template <typename Elt, int K, int V>
@@ -115,21 +139,22 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                      const float* __restrict__ decay, const Elt* __restrict__ beta, const float* __restrict__ S0,
                      const Elt* __restrict__ dO, const float* __restrict__ dS_T, int T, int H, int HV, float scale,
                      float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg,
-                     float* __restrict__ dbeta, float* __restrict__ dS0, float* __restrict__ ckpt) {
+                     float* __restrict__ dbeta, float* __restrict__ dS0, float* __restrict__ ckpt,
+                     float* __restrict__ rres) {
     using Sh = BwdShape<K, V>;
     constexpr int VB = Sh::VB, TPR = Sh::TPR, RG = Sh::RG, R = Sh::R, NT = Sh::NT, NWB = Sh::NWB, CW = Sh::CW;
     constexpr int CK = BWD_CK, VN = Sh::template VN<Elt>, EA = Sh::EA, EK = Sh::template EK<Elt>,
-                  EV = Sh::template EV<Elt>;
+                  EV = Sh::template EV<Elt>, ER = Sh::ER;
     extern __shared__ float bsm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float* sPrev = bsm + (size_t)warp * CK * K * VB;  // [CK][K][VB] state entering each token (this warp's)
-    float* sR = bsm + (size_t)NWB * CK * K * VB + warp * CK * VB;  // [CK][VB] residuals (this warp's)
-    float* sA = bsm + (size_t)NWB * CK * K * VB + NWB * CK * VB;   // staged block: [CK][K] decay exp(g)
+    float* sPrev = bsm + (size_t)warp * CK * K * VB;  // [CK][R][32 lanes][2] state entering each token (this warp's)
+    float* sA = bsm + (size_t)NWB * CK * K * VB;  // staged block: [CK][K] decay exp(g)
     float* sK = sA + CK * K;                   //               [CK][K] k
     float* sQ = sK + CK * K;                   //               [CK][K] q
     float* sV = sQ + CK * K;                   //               [CK][CW] v (this CTA's columns)
     float* sDO = sV + CK * CW;                 //               [CK][CW] dO
-    float* sB = sDO + CK * CW;                 //               [CK] beta
+    float* sRr = sDO + CK * CW;                //               [CK][CW] r (saved by the forward sweep)
+    float* sB = sRr + CK * CW;                 //               [CK] beta
     float* sDq = sB + CK;                      // [NWB][CK][K] dq of the block, each warp's over its columns
     float* sDk = sDq + NWB * CK * K;           // [NWB][CK][K] dk
     float* sDg = sDk + NWB * CK * K;           // [NWB][CK][K] dg
@@ -152,6 +177,7 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
 
     // the next block's inputs as loaded: 16-byte vectors of decay rows, k / q rows, and the CTA's v / dO columns
     uint4 la[EA], lk[EK], lq[EK], lv[EV], lo[EV];
+    float4 lr[ER];
     Elt lb;
     constexpr int KV = K / VN, CV = CW / VN;  // vectors in a k / q row, in the CTA's v / dO columns
     auto load_block = [&](int blk, bool backward) {
@@ -175,6 +201,13 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
             if (idx < n * CV) {
                 lv[e] = reinterpret_cast<const uint4*>(v + tok_v(t0 + j) * V + cc0)[x];
                 if (backward) lo[e] = reinterpret_cast<const uint4*>(dO + tok_v(t0 + j) * V + cc0)[x];
+            }
+        }
+        if (backward) {
+#pragma unroll
+            for (int e = 0; e < ER; ++e) {  // written by this CTA in the forward sweep: read through L2
+                const int idx = tid + e * NT, j = idx / (CW / 4), x = idx - j * (CW / 4);
+                if (idx < n * (CW / 4)) lr[e] = __ldcg(reinterpret_cast<const float4*>(rres + tok_v(t0 + j) * V + cc0) + x);
             }
         }
         if (tid < n) lb = beta[tok_v(t0 + tid)];
@@ -203,6 +236,13 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                 if (backward) put_f32(sDO + VN * idx, lo[e], dO);
             }
         }
+        if (backward) {
+#pragma unroll
+            for (int e = 0; e < ER; ++e) {
+                const int idx = tid + e * NT;
+                if (idx < n * (CW / 4)) *reinterpret_cast<float4*>(sRr + 4 * idx) = lr[e];
+            }
+        }
         if (tid < n) sB[tid] = to_f32(lb);
     };
 
@@ -210,13 +250,13 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     // (returned), rank-1 write
     float2 S[R];
     auto forward_step = [&](int j) {
+        float a[R], kd[R];
+        rows_of<R>(sA + j * K + R * rg, a);
+        rows_of<R>(sK + j * K + R * rg, kd);
         float2 p = make_float2(0.f, 0.f);
-        float kd[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const float a = sA[j * K + rg + RG * i];
-            kd[i] = sK[j * K + rg + RG * i];
-            S[i] = f2_mul(f2_splat(a), S[i]);
+            S[i] = f2_mul(f2_splat(a[i]), S[i]);
             p = f2_fma(f2_splat(kd[i]), S[i], p);
         }
         p = sum_over_rows<TPR>(p);
@@ -226,75 +266,104 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
         for (int i = 0; i < R; ++i) S[i] = f2_fma(f2_splat(bt * kd[i]), r, S[i]);
         return r;
     };
-    auto state_row = [&](int i) { return (size_t)(rg + RG * i) * VB + 2 * cg; };  // offset in a [K][VB] block
+    // this lane's state entries in a warp-private copy (saved states, sPrev): entry i of lane l is the pair
+    // 32 i + l, so a warp's access to one entry covers 256 contiguous bytes
+    auto put_state = [&](float* dst, const float2 (&x)[R]) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) reinterpret_cast<float2*>(dst)[32 * i + lane] = x[i];
+    };
+    auto get_state = [&](const float* src, float2 (&x)[R]) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) x[i] = reinterpret_cast<const float2*>(src)[32 * i + lane];
+    };
+    constexpr int KVB = K * VB;  // floats of one warp's state block
 
     // ---- 1. forward sweep, the entering state of every block of CK tokens saved ---------------------
 #pragma unroll
     for (int i = 0; i < R; ++i)
-        S[i] = S0 ? *reinterpret_cast<const float2*>(S0 + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg)
+        S[i] = S0 ? *reinterpret_cast<const float2*>(S0 + ((size_t)pair * K + R * rg + i) * V + c0 + 2 * cg)
                   : make_float2(0.f, 0.f);
+    // the residuals of a block gather in sRr and go to the workspace after the next barrier
+    auto store_residuals = [&](int blk) {
+        const int t0 = blk * CK, n = min(CK, T - t0);
+        for (int idx = tid; idx < n * (CW / 4); idx += NT) {
+            const int j = idx / (CW / 4), x = idx - j * (CW / 4);
+            reinterpret_cast<float4*>(rres + tok_v(t0 + j) * V + cc0)[x] = *reinterpret_cast<const float4*>(sRr + 4 * idx);
+        }
+    };
     load_block(0, false);
     for (int blk = 0; blk < NCK; ++blk) {
         const int n = min(CK, T - blk * CK);
-        __syncthreads();  // the previous block's staged inputs are read no more (sBias written, at the start)
+        __syncthreads();  // the previous block's staged inputs are read no more, its residuals are complete
+        if (blk > 0) store_residuals(blk - 1);  // (the forward stage leaves sRr alone)
         stage_block(n, false);
-        __syncthreads();
+        __syncthreads();  // and stored: sRr is rewritten from here
         if (blk + 1 < NCK) load_block(blk + 1, false);
-#pragma unroll
-        for (int i = 0; i < R; ++i)
-            *reinterpret_cast<float2*>(my_ckpt + (size_t)blk * K * VB + state_row(i)) = S[i];
-        for (int j = 0; j < n; ++j) forward_step(j);
+        put_state(my_ckpt + (size_t)blk * KVB, S);
+        for (int j = 0; j < n; ++j) {
+            const float2 r = forward_step(j);
+            if (rg == 0) *reinterpret_cast<float2*>(sRr + j * CW + warp * VB + 2 * cg) = r;
+        }
     }
+    __syncthreads();
+    store_residuals(NCK - 1);
+    __syncthreads();  // the last block's residuals are read back below, by other threads
 
     // ---- 2. blocks in reverse ----------------------------------------------------------------------
     float2 dS[R];
 #pragma unroll
     for (int i = 0; i < R; ++i)
-        dS[i] = dS_T ? *reinterpret_cast<const float2*>(dS_T + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg)
+        dS[i] = dS_T ? *reinterpret_cast<const float2*>(dS_T + ((size_t)pair * K + R * rg + i) * V + c0 + 2 * cg)
                      : make_float2(0.f, 0.f);
     load_block(NCK - 1, true);
+    float2 Sck[R];  // the checkpoint of the block processed next, loaded a block ahead
+    get_state(my_ckpt + (size_t)(NCK - 1) * KVB, Sck);
     for (int blk = NCK - 1; blk >= 0; --blk) {
         const int t0 = blk * CK, n = min(CK, T - t0);
         __syncthreads();  // the previous block's staged inputs and row sums are read no more
         stage_block(n, true);
         __syncthreads();
         if (blk > 0) load_block(blk - 1, true);
-        // recompute: the state entering each token into shared memory (each lane its own entries), the
-        // residuals too; S ends as the state after the block's last token
+        // recompute: the state entering each token into shared memory (each lane its own entries), from the
+        // saved residuals (the same operations as the forward sweep, so the same values); S ends as the state
+        // after the block's last token
 #pragma unroll
-        for (int i = 0; i < R; ++i) S[i] = *reinterpret_cast<const float2*>(my_ckpt + (size_t)blk * K * VB + state_row(i));
+        for (int i = 0; i < R; ++i) S[i] = Sck[i];
+        if (blk > 0) get_state(my_ckpt + (size_t)(blk - 1) * KVB, Sck);
         for (int j = 0; j < n; ++j) {
+            put_state(sPrev + j * KVB, S);
+            float a[R], kd[R];
+            rows_of<R>(sA + j * K + R * rg, a);
+            rows_of<R>(sK + j * K + R * rg, kd);
+            const float2 r = *reinterpret_cast<const float2*>(sRr + j * CW + warp * VB + 2 * cg);
+            const float bt = sB[j];
 #pragma unroll
-            for (int i = 0; i < R; ++i) *reinterpret_cast<float2*>(sPrev + (size_t)j * K * VB + state_row(i)) = S[i];
-            const float2 r = forward_step(j);
-            if (rg == 0) *reinterpret_cast<float2*>(sR + j * VB + 2 * cg) = r;  // same values in every row group
+            for (int i = 0; i < R; ++i) S[i] = f2_fma(f2_splat(bt * kd[i]), r, f2_mul(f2_splat(a[i]), S[i]));
         }
-        __syncwarp();
         // reverse through the block; S holds the state after token t
         for (int j = n - 1; j >= 0; --j) {
-            const float2 dOc = *reinterpret_cast<const float2*>(sDO + j * CW + warp * VB + 2 * cg);
-            float qd[R], kd[R], a[R];
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                a[i] = sA[j * K + rg + RG * i];
-                qd[i] = sQ[j * K + rg + RG * i];
-                kd[i] = sK[j * K + rg + RG * i];
-            }
+            // dOs = s dO_t (this lane's columns)
+            const float2 dOs = f2_mul(f2_splat(scale), *reinterpret_cast<const float2*>(sDO + j * CW + warp * VB + 2 * cg));
+            float a[R], qd[R], kd[R];
+            rows_of<R>(sA + j * K + R * rg, a);
+            rows_of<R>(sQ + j * K + R * rg, qd);
+            rows_of<R>(sK + j * K + R * rg, kd);
             // dq_t = s S_t dO_t ; dS += s q_t dO_t^T
+            float pq[R];
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float part = sum_over_cols<TPR>(f2_mul(S[i], dOc));
-                if (cg == 0) wDq[j * K + rg + RG * i] = scale * part;
-                dS[i] = f2_fma(f2_splat(scale * qd[i]), dOc, dS[i]);
+                pq[i] = sum_over_cols<TPR>(f2_mul(S[i], dOs));
+                dS[i] = f2_fma(f2_splat(qd[i]), dOs, dS[i]);
             }
+            if (cg == 0) put_rows<R>(wDq + j * K + R * rg, pq);
             // u = dS^T k_t over the key rows
             float2 u = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < R; ++i) u = f2_fma(f2_splat(kd[i]), dS[i], u);
             u = sum_over_rows<TPR>(u);
-            const float2 r = *reinterpret_cast<const float2*>(sR + j * VB + 2 * cg);
+            const float2 r = *reinterpret_cast<const float2*>(sRr + j * CW + warp * VB + 2 * cg);
             const float bt = sB[j];
-            const float2 dr = f2_mul(f2_splat(bt), u);
+            const float2 dr = f2_mul(f2_splat(bt), u), ndr = make_float2(-dr.x, -dr.y);
             if (rg == 0) {  // dbeta_t = u . r over this warp's columns; dv_t = dr
                 float db = u.x * r.x + u.y * r.y;
 #pragma unroll
@@ -303,19 +372,22 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                 *reinterpret_cast<float2*>(dv + tok_v(t0 + j) * V + c0 + 2 * cg) = dr;
             }
             const float2 btr = f2_mul(f2_splat(bt), r);
+            float pk[R], pg[R];
+            float2 Sp[R];
+            get_state(sPrev + j * KVB, Sp);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float2 Sp = *reinterpret_cast<const float2*>(sPrev + (size_t)j * K * VB + state_row(i));
-                const float2 Sd = f2_mul(f2_splat(a[i]), Sp);
-                // dk_t = beta dS r - S_dec dr
-                const float pk = sum_over_cols<TPR>(f2_sub(f2_mul(dS[i], btr), f2_mul(Sd, dr)));
-                if (cg == 0) wDk[j * K + rg + RG * i] = pk;
+                // dk_t = beta dS r - S_dec dr,  S_dec = a S_{t-1}
+                pk[i] = sum_over_cols<TPR>(f2_fma(dS[i], btr, f2_mul(f2_mul(f2_splat(a[i]), Sp[i]), ndr)));
                 // dS_dec = dS - k dr^T ; dg_t = a rowsum(dS_dec S_{t-1}) ; dS_{t-1} = a dS_dec
-                const float2 dSd = f2_fma(f2_splat(-kd[i]), dr, dS[i]);
-                const float pg = sum_over_cols<TPR>(f2_mul(dSd, Sp));
-                if (cg == 0) wDg[j * K + rg + RG * i] = a[i] * pg;
+                const float2 dSd = f2_fma(f2_splat(kd[i]), ndr, dS[i]);
+                pg[i] = a[i] * sum_over_cols<TPR>(f2_mul(dSd, Sp[i]));
                 dS[i] = f2_mul(f2_splat(a[i]), dSd);
-                S[i] = Sp;
+                S[i] = Sp[i];
+            }
+            if (cg == 0) {
+                put_rows<R>(wDk + j * K + R * rg, pk);
+                put_rows<R>(wDg + j * K + R * rg, pg);
             }
         }
         __syncthreads();  // the block's row sums are complete
@@ -342,7 +414,7 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
     if (dS0) {
 #pragma unroll
         for (int i = 0; i < R; ++i)
-            *reinterpret_cast<float2*>(dS0 + ((size_t)pair * K + rg + RG * i) * V + c0 + 2 * cg) = dS[i];
+            *reinterpret_cast<float2*>(dS0 + ((size_t)pair * K + R * rg + i) * V + c0 + 2 * cg) = dS[i];
     }
 }
 
@@ -420,9 +492,10 @@ size_t backward_ckpt_floats(int B, int T, int HV, int K, int V) {
 template <typename Elt, int K, int V>
 cudaError_t launch_bwd(const BackwardArgs& a) {
     using Sh = BwdShape<K, V>;
-    // workspace: the saved states, then the decays [B][T][HV][K]
+    // workspace: the saved states, the decays [B][T][HV][K], the residuals [B][T][HV][V]
     float* ckpt = static_cast<float*>(a.workspace);
     float* decay = ckpt + backward_ckpt_floats(a.B, a.T, a.HV, K, V);
+    float* rres = decay + (size_t)a.B * a.T * a.HV * K;
     const long long n = (long long)a.B * a.T * a.HV * K;
     const unsigned dgrid = (unsigned)std::min<long long>((n + 255) / 256, 148ll * 16);
     decay_kernel<Elt><<<dgrid, 256, 0, a.stream>>>(static_cast<const Elt*>(a.g), a.A_log, a.dt_bias, n, a.HV, K,
@@ -433,7 +506,7 @@ cudaError_t launch_bwd(const BackwardArgs& a) {
     kern<<<(unsigned)((long long)a.B * a.HV * (Sh::NCB / Sh::NWB)), Sh::NT, Sh::smem_bytes, a.stream>>>(
         static_cast<const Elt*>(a.q), static_cast<const Elt*>(a.k), static_cast<const Elt*>(a.v), decay,
         static_cast<const Elt*>(a.beta), a.S0, static_cast<const Elt*>(a.dO), a.dS_T, a.T, a.H, a.HV, a.scale, a.dq,
-        a.dk, a.dv, a.dg, a.dbeta, a.dS0, ckpt);
+        a.dk, a.dv, a.dg, a.dbeta, a.dS0, ckpt, rres);
     return cudaGetLastError();
 }
 
@@ -462,7 +535,7 @@ cudaError_t bwd_k(const BackwardArgs& a) {
 }  // namespace
 
 size_t backward_workspace(int B, int T, int HV, int K, int V) {
-    return (backward_ckpt_floats(B, T, HV, K, V) + (size_t)B * T * HV * K) * sizeof(float);
+    return (backward_ckpt_floats(B, T, HV, K, V) + (size_t)B * T * HV * (K + V)) * sizeof(float);
 }
 
 cudaError_t launch_backward(const BackwardArgs& a) {

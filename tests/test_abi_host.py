@@ -187,8 +187,9 @@ def test_input_option_entry_points_validate_before_launch():
 
 def test_backward_validates_before_launch():
     L = kda.lib
-    # the states saved every 8 tokens, then the fp32 decays of every (token, value head, key channel)
-    assert kda.backward_workspace_size(2, 100, 2, 4, 128, 64) == 2 * 4 * 13 * 128 * 64 * 4 + 2 * 100 * 4 * 128 * 4
+    # the states saved every 8 tokens, the fp32 decays of every (token, value head, key channel) and the fp32
+    # residuals of every (token, value head, value column)
+    assert kda.backward_workspace_size(2, 100, 2, 4, 128, 64) == (2 * 4 * 13 * 128 * 64 + 2 * 100 * 4 * (128 + 64)) * 4
     assert kda.backward_workspace_size(2, 100, 3, 4, 128, 64) == 0
 
     def call(**over):
