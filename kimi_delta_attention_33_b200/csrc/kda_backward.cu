@@ -39,7 +39,8 @@ namespace kda {
 
 namespace {
 
-constexpr int BWD_CK = 8;  // tokens between saved states
+constexpr int BWD_CK = 8;          // tokens between saved states
+constexpr int GATE_BWD_ROWS = 16;  // (b, t) rows per CTA of the gate's backward
 
 template <int K, int V>
 struct BwdShape {
@@ -436,8 +437,8 @@ decay_kernel(const Elt* __restrict__ g, const float* __restrict__ A_log, const f
 // parameter gradients (KDA notes, "Gate 激活": input x = g_raw + dt_bias, rate = exp(A_log)):
 //   SAFE      g = L sigmoid(rate x):  dg/dx = L s (1 - s) rate,  dg/dA_log = L s (1 - s) rate x
 //   STANDARD  g = -rate softplus(x):  dg/dx = -rate sigmoid(x),  dg/dA_log = -rate softplus(x)
-// One CTA per (block of 64 tokens, value head), thread = key channel: the token loop sums ddt_bias and
-// dA_log per channel, then one atomic per channel and one per CTA.
+// One CTA per (block of GATE_BWD_ROWS (b, t) rows, value head), thread = key channel: the row loop sums
+// ddt_bias and dA_log per channel, then one atomic per channel and one per CTA.
 template <typename Elt>
 __global__ void __launch_bounds__(128)
 gate_bwd_kernel(const Elt* __restrict__ g_raw, const float* __restrict__ A_log, const float* __restrict__ dt_bias,
@@ -445,13 +446,13 @@ gate_bwd_kernel(const Elt* __restrict__ g_raw, const float* __restrict__ A_log, 
                 float* __restrict__ ddt_bias, float* __restrict__ dA_log) {
     __shared__ float s_part[4];
     const int hv = blockIdx.y;
-    const long long r0 = (long long)blockIdx.x * 64;
+    const long long r0 = (long long)blockIdx.x * GATE_BWD_ROWS;
     const float rate = expf(A_log[hv]);
     float acc_a = 0.f;
     for (int d = threadIdx.x; d < K; d += blockDim.x) {
         const float bias = dt_bias ? dt_bias[hv * K + d] : 0.0f;
         float sb = 0.f;
-        for (long long rr = r0; rr < r0 + 64 && rr < rows; ++rr) {
+        for (long long rr = r0; rr < r0 + GATE_BWD_ROWS && rr < rows; ++rr) {
             const size_t idx = ((size_t)rr * HV + hv) * K + d;
             const float x = to_f32(g_raw[idx]) + bias;
             float dgdx, dgda;
@@ -552,7 +553,7 @@ cudaError_t launch_backward(const BackwardArgs& a) {
         return e;
     if (a.dA_log && (e = cudaMemsetAsync(a.dA_log, 0, (size_t)a.HV * sizeof(float), a.stream)) != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.T;
-    const dim3 grid((unsigned)((rows + 63) / 64), (unsigned)a.HV);
+    const dim3 grid((unsigned)((rows + GATE_BWD_ROWS - 1) / GATE_BWD_ROWS), (unsigned)a.HV);
     if (a.dtype == KDA_BF16)
         gate_bwd_kernel<__nv_bfloat16><<<grid, 128, 0, a.stream>>>(static_cast<const __nv_bfloat16*>(a.g), a.A_log,
                                                                    a.dt_bias, rows, a.HV, a.K, a.gate_mode,
