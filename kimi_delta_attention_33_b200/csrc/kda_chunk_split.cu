@@ -400,7 +400,8 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                       false);
             mma_commit(mbar);
         }
-        // Qtil (fp32) into TMEM rows 64-127, columns 256-383, while M1 runs: M12 accumulates -A Wtil onto it
+        // Qtil (fp32) into TMEM rows 64-127, columns 256-383, and zeros into columns 384-511, while M1 runs: M12
+        // accumulates [-A Wtil | -A U] onto them
         if (wq >= 2) {
             const int i = 32 * (wq - 2) + lane;
             uint32_t x[32];
@@ -413,6 +414,9 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
                 x[4 * c4 + 3] = v4.w;
             }
             tmem_st32(taddr(tmem, 32 * wq, 256 + 32 * wc), x);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) x[t] = 0u;
+            tmem_st32(taddr(tmem, 32 * wq, 384 + 32 * wc), x);
             tmem_wait_st();
         }
 
@@ -573,9 +577,7 @@ chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const 
             gemm_tf32(tmem, s_base + L::KA, CH / 4 * 128, s_base + L::GM, CH / 4 * 128, idesc_tf32(128, 256), CH / 8,
                       false);
             gemm_tf32(tmem + 256, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::GM, CH / 4 * 128,
-                      idesc_tf32(128, 128), CH / 8, true);
-            gemm_tf32(tmem + 384, s_base + L::KA + 32768, CH / 4 * 128, s_base + L::VT, CH / 4 * 128,
-                      idesc_tf32(128, 128), CH / 8, false);
+                      idesc_tf32(128, 256), CH / 8, true);  // B = BT rows 0-255 (GM, then VT)
             mma_commit(mbar);
         }
         {
