@@ -143,7 +143,7 @@ recurrent_bwd_kernel(const Elt* __restrict__ q, const Elt* __restrict__ k, const
                      float* __restrict__ dbeta, float* __restrict__ dS0, float* __restrict__ ckpt,
                      float* __restrict__ rres) {
     using Sh = BwdShape<K, V>;
-    constexpr int VB = Sh::VB, TPR = Sh::TPR, RG = Sh::RG, R = Sh::R, NT = Sh::NT, NWB = Sh::NWB, CW = Sh::CW;
+    constexpr int VB = Sh::VB, TPR = Sh::TPR, R = Sh::R, NT = Sh::NT, NWB = Sh::NWB, CW = Sh::CW;
     constexpr int CK = BWD_CK, VN = Sh::template VN<Elt>, EA = Sh::EA, EK = Sh::template EK<Elt>,
                   EV = Sh::template EV<Elt>, ER = Sh::ER;
     extern __shared__ float bsm[];
