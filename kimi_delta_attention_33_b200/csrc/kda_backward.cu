@@ -18,10 +18,10 @@
 // R rg .. R rg + R - 1 and columns 2 cg, 2 cg + 1 of the warp's block of the state and of dS in registers, as
 // pairs for the packed fp32x2 arithmetic, so reductions over key rows (the residual's prediction and u)
 // are warp shuffles, with no barrier on the per-token chain; two columns a lane keep the chain short and
-// give each SM sub-partition two warps to interleave.  Row quantities (dq, dk, dg) and dbeta, summed over each warp's columns, are kept per
-// warp in shared memory for the block of tokens, then summed over the CTA's warps and added into the fp32
-// outputs with one atomic per entry (the other CTAs of the value head, and the other value heads of a q/k
-// head, add theirs).
+// give each SM sub-partition two warps to interleave.  Row quantities (dq, dk, dg) and dbeta, summed over
+// each warp's columns, are kept per warp in shared memory for the block of tokens, then summed over the
+// CTA's warps and added into the fp32 outputs (one float4 atomic per four key channels; the other CTAs
+// of the value head, and the other value heads of a q/k head, add theirs).
 //   1. forward sweep over all tokens, the state saved every CK tokens and the residual r of every token
 //      to the workspace;
 //   2. the blocks of CK tokens in reverse: the block's states recomputed from its checkpoint into
